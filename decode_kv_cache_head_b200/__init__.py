@@ -1,0 +1,225 @@
+"""Python binding of librkv.so, the B200 R-KV decode-time KV compression step.
+
+Argument marshalling only: every function here turns torch tensors into raw
+device pointers and calls the C-ABI function of the same name (declared in
+``include/rkv.h``).  All computation runs in the library's CUDA kernels; there
+is no CPU fallback, and importing this package fails if ``librkv.so`` has not
+been built (``python -m decode_kv_cache_head_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+__all__ = [
+    "RKV_OK", "RKV_STATUS_DISABLED", "RKV_RED_MEAN", "RKV_RED_MAX", "RKV_GQA_MAX", "RKV_GQA_MEAN",
+    "RkvError", "rkv_config", "rkv_step_options", "make_config", "library_path",
+    "rkv_status_string", "rkv_version", "rkv_workspace_size", "rkv_workspace_status",
+    "rkv_score_importance", "rkv_score_redundancy", "rkv_select_topk", "rkv_compact_kv",
+    "rkv_compress_step",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "librkv.so")
+
+RKV_OK = 0
+RKV_STATUS_DISABLED = 1
+RKV_RED_MEAN, RKV_RED_MAX = 0, 1
+RKV_GQA_MAX, RKV_GQA_MEAN = 0, 1
+
+
+class rkv_config(ctypes.Structure):
+    _fields_ = [
+        ("budget", ctypes.c_int32),
+        ("buffer", ctypes.c_int32),
+        ("window", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("n_kv_heads", ctypes.c_int32),
+        ("n_q_heads", ctypes.c_int32),
+        ("mix_lambda", ctypes.c_float),
+        ("redundancy_mode", ctypes.c_int32),
+        ("gqa_pool", ctypes.c_int32),
+    ]
+
+
+class rkv_step_options(ctypes.Structure):
+    _fields_ = [
+        ("kept_out", ctypes.c_void_p),
+        ("scores_out", ctypes.c_void_p),
+        ("main_begin", ctypes.c_void_p),
+        ("main_end", ctypes.c_void_p),
+        ("cluster_size", ctypes.c_int32),
+    ]
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"{_LIB_PATH} is missing: build it with "
+                          "`python -m decode_kv_cache_head_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(_LIB_PATH)
+    P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    CFG = ctypes.POINTER(rkv_config)
+    sig = {
+        "rkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "rkv_version": (I32, []),
+        "rkv_workspace_size": (SZ, [CFG, I32, I32, I32]),
+        "rkv_workspace_status": (ctypes.c_int, [P, P]),
+        "rkv_score_importance": (ctypes.c_int, [CFG, P, P, I64, I32, P, P, P, SZ, P]),
+        "rkv_score_redundancy": (ctypes.c_int, [CFG, P, I64, I32, P, P, P, SZ, P]),
+        "rkv_select_topk": (ctypes.c_int, [CFG, P, P, I32, P, P, P, SZ, P]),
+        "rkv_compact_kv": (ctypes.c_int, [CFG, P, P, P, P, P, I64, I32, P, SZ, P]),
+        "rkv_compress_step": (ctypes.c_int, [CFG, I32, I32, I32, P, P, P, P, P, P,
+                                             ctypes.POINTER(rkv_step_options), P, SZ, P]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+class RkvError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {rkv_status_string(status)} ({status})")
+
+
+def rkv_status_string(status: int) -> str:
+    return _lib.rkv_status_string(int(status)).decode()
+
+
+def rkv_version() -> int:
+    return int(_lib.rkv_version())
+
+
+def make_config(budget=1024, buffer=128, window=8, head_dim=128, n_kv_heads=8, n_q_heads=32,
+                mix_lambda=0.1, redundancy_mode=RKV_RED_MEAN, gqa_pool=RKV_GQA_MAX) -> rkv_config:
+    return rkv_config(int(budget), int(buffer), int(window), int(head_dim), int(n_kv_heads),
+                      int(n_q_heads), float(mix_lambda), int(redundancy_mode), int(gqa_pool))
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to librkv must be contiguous")
+    return t.data_ptr()
+
+
+def _dtype(t: Optional[torch.Tensor], dt: torch.dtype, name: str) -> None:
+    if t is not None and t.dtype != dt:
+        raise TypeError(f"{name} must be {dt}, got {t.dtype}")
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _check(status: int, where: str, allow_disabled: bool = False) -> int:
+    if status == RKV_OK or (allow_disabled and status == RKV_STATUS_DISABLED):
+        return status
+    raise RkvError(status, where)
+
+
+def rkv_workspace_size(cfg: rkv_config, n_layers: int, batch: int, cap: int) -> int:
+    return int(_lib.rkv_workspace_size(ctypes.byref(cfg), n_layers, batch, cap))
+
+
+def rkv_workspace_status(workspace: torch.Tensor, stream=None) -> int:
+    return int(_lib.rkv_workspace_status(_ptr(workspace), _stream(stream)))
+
+
+def rkv_score_importance(cfg, q, k, n_tokens, I, inv_norm=None, workspace=None, stream=None):
+    """q [Hq, w, 128] bf16; k [Hkv, cap, 128] bf16; I [Hkv, N-w] fp32; inv_norm [Hkv, N] fp32."""
+    _dtype(q, torch.bfloat16, "q"); _dtype(k, torch.bfloat16, "k")
+    _dtype(I, torch.float32, "I"); _dtype(inv_norm, torch.float32, "inv_norm")
+    ws = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    return _check(_lib.rkv_score_importance(ctypes.byref(cfg), _ptr(q), _ptr(k), k.shape[-2] * 128,
+                                            int(n_tokens), _ptr(I), _ptr(inv_norm), _ptr(workspace),
+                                            ws, _stream(stream)), "rkv_score_importance")
+
+
+def rkv_score_redundancy(cfg, k, n_tokens, r=None, R=None, workspace=None, stream=None):
+    """k [Hkv, cap, 128] bf16; r, R [Hkv, N-w] fp32."""
+    _dtype(k, torch.bfloat16, "k"); _dtype(r, torch.float32, "r"); _dtype(R, torch.float32, "R")
+    ws = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    return _check(_lib.rkv_score_redundancy(ctypes.byref(cfg), _ptr(k), k.shape[-2] * 128,
+                                            int(n_tokens), _ptr(r), _ptr(R), _ptr(workspace), ws,
+                                            _stream(stream)), "rkv_score_redundancy")
+
+
+def rkv_select_topk(cfg, I, R, n_tokens, kept, Z=None, workspace=None, stream=None):
+    """I, R [Hkv, N-w] fp32; kept [Hkv, budget] int32; Z [Hkv, N-w] fp32 or None."""
+    _dtype(I, torch.float32, "I"); _dtype(R, torch.float32, "R")
+    _dtype(kept, torch.int32, "kept"); _dtype(Z, torch.float32, "Z")
+    ws = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    return _check(_lib.rkv_select_topk(ctypes.byref(cfg), _ptr(I), _ptr(R), int(n_tokens),
+                                       _ptr(kept), _ptr(Z), _ptr(workspace), ws, _stream(stream)),
+                  "rkv_select_topk", allow_disabled=True)
+
+
+def rkv_compact_kv(cfg, k_src, v_src, kept, k_dst, v_dst, n_tokens, workspace=None, stream=None):
+    """k/v [Hkv, cap, 128] bf16 (dst may be src: in place); kept [Hkv, budget] int32."""
+    for n, t in (("k_src", k_src), ("v_src", v_src), ("k_dst", k_dst), ("v_dst", v_dst)):
+        _dtype(t, torch.bfloat16, n)
+    _dtype(kept, torch.int32, "kept")
+    ws = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    return _check(_lib.rkv_compact_kv(ctypes.byref(cfg), _ptr(k_src), _ptr(v_src), _ptr(kept),
+                                      _ptr(k_dst), _ptr(v_dst), k_src.shape[-2] * 128,
+                                      int(n_tokens), _ptr(workspace), ws, _stream(stream)),
+                  "rkv_compact_kv", allow_disabled=True)
+
+
+def _ptr_array(ts: Sequence[torch.Tensor]):
+    arr = (ctypes.c_void_p * len(ts))()
+    for i, t in enumerate(ts):
+        arr[i] = _ptr(t)
+    return arr
+
+
+def rkv_compress_step(cfg, k_layers, v_layers, q_layers, cur_len, workspace, budgets=None,
+                      lambdas=None, kept_out=None, scores_out=None, events=None,
+                      cluster_size=0, stream=None):
+    """The whole step over all layers of a batch, in place.
+
+    k_layers / v_layers: sequences of [batch, Hkv, cap, 128] bf16 tensors (one
+    per layer, or one [n_layers, batch, Hkv, cap, 128] tensor); q_layers:
+    [batch, Hq, w, 128] per layer; cur_len [batch] int32 (updated);
+    budgets [batch] int32 / lambdas [batch] fp32 or None; kept_out
+    [n_layers, batch, Hkv, cap] int32 and scores_out [n_layers, batch, Hkv, 4,
+    cap] fp32 optional; events: (begin, end) torch.cuda.Event recorded around
+    the main kernel, or None.
+    """
+    k_layers, v_layers, q_layers = list(k_layers), list(v_layers), list(q_layers)
+    n_layers = len(k_layers)
+    batch, _, cap, _ = k_layers[0].shape
+    for t in k_layers + v_layers + q_layers:
+        _dtype(t, torch.bfloat16, "k/v/q")
+    _dtype(cur_len, torch.int32, "cur_len"); _dtype(budgets, torch.int32, "budgets")
+    _dtype(lambdas, torch.float32, "lambdas"); _dtype(kept_out, torch.int32, "kept_out")
+    _dtype(scores_out, torch.float32, "scores_out")
+    opts = rkv_step_options(_ptr(kept_out), _ptr(scores_out), None, None, int(cluster_size))
+    if events is not None:
+        opts.main_begin = events[0].cuda_event
+        opts.main_end = events[1].cuda_event
+    ws = workspace.numel() * workspace.element_size()
+    return _check(_lib.rkv_compress_step(ctypes.byref(cfg), n_layers, batch, cap,
+                                         _ptr_array(k_layers), _ptr_array(v_layers),
+                                         _ptr_array(q_layers), _ptr(budgets), _ptr(lambdas),
+                                         _ptr(cur_len), ctypes.byref(opts), _ptr(workspace), ws,
+                                         _stream(stream)), "rkv_compress_step",
+                  allow_disabled=True)

@@ -1,0 +1,423 @@
+// rkv_abi.cu -- the extern "C" entry points declared in include/rkv.h:
+// argument validation (synchronous, before anything is enqueued), TMA
+// descriptor encoding, shape selection and kernel launches on the caller's
+// stream.  No allocation, no synchronisation, no state kept between calls.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "rkv_internal.h"
+#include "rkv_ptx.cuh"
+
+using namespace rkv;
+
+namespace {
+
+constexpr int32_t kVersion = 1 * 10000 + 0 * 100 + 0;
+constexpr int kSmemPerSM = 233472;            // 228 KB of shared memory per SM
+constexpr int kSmemPerCtaMax = 232448;        // 227 KB opt-in limit per CTA
+constexpr int kSmemTwoPerSM = kSmemPerSM / 2 - 1024;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// A [rows, 128] bf16 row-major matrix read in boxes of 64 columns x box_rows
+// rows with the 128-byte swizzle (one box row = 128 bytes = one swizzle span).
+bool encode_rows128(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(kHeadDim * 2)};
+    cuuint32_t box[2] = {64u, box_rows};
+    cuuint32_t es[2] = {1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+              box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlap(const void *a, size_t na, const void *b, size_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+int nqp_of(int nq) { return (nq + 15) / 16 * 16; }
+
+rkv_status check_cfg(const rkv_config *c) {
+    if (!c) return RKV_ERR_NULL;
+    if (c->head_dim != kHeadDim) return RKV_ERR_UNSUPPORTED;
+    if (c->n_kv_heads < 1 || c->n_q_heads < 1 || c->n_q_heads % c->n_kv_heads != 0)
+        return RKV_ERR_INVALID;
+    if (c->window < 1) return RKV_ERR_INVALID;
+    if (static_cast<int64_t>(c->n_q_heads / c->n_kv_heads) * c->window > kMaxQCols)
+        return RKV_ERR_UNSUPPORTED;
+    if (!std::isfinite(c->mix_lambda)) return RKV_ERR_INVALID;
+    if (c->redundancy_mode != RKV_RED_MEAN && c->redundancy_mode != RKV_RED_MAX)
+        return RKV_ERR_INVALID;
+    if (c->gqa_pool != RKV_GQA_MAX && c->gqa_pool != RKV_GQA_MEAN) return RKV_ERR_INVALID;
+    return RKV_OK;
+}
+
+struct Shape {
+    int cs, rmax, rp, tmem_cols, nqp;
+    size_t smem;
+};
+
+int pow2_at_least(int x) {
+    int p = 32;
+    while (p < x) p <<= 1;
+    return p;
+}
+
+Shape shape_for(int cap, int nqp, int cs) {
+    Shape s;
+    s.cs = cs;
+    s.nqp = nqp;
+    s.rmax = ((cap + cs - 1) / cs + 15) / 16 * 16;
+    s.rp = s.rmax < 128 ? 128 : s.rmax;
+    const int ntiles = (s.rmax + 127) / 128;
+    s.tmem_cols = pow2_at_least(ntiles * nqp);
+    s.smem = step_smem_bytes(s.rp, s.rmax, cap, nqp);
+    // TMEM holds 512 columns per SM: never let more CTAs share an SM than fit,
+    // by asking for enough shared memory to cap residency.
+    const int max_res = 512 / s.tmem_cols;
+    const size_t floor_smem = static_cast<size_t>(kSmemPerSM / (max_res + 1) - 1024 + 16);
+    if (s.smem < floor_smem) s.smem = floor_smem;
+    return s;
+}
+
+// Picks the cluster size: the smallest of 8, 16, 4, 2 whose layout lets two
+// CTAs share an SM, else the smallest that fits at all.  cs = 0 if none fits.
+Shape choose_shape(int cap, int nqp, int cs_req) {
+    if (cs_req) {
+        Shape s = shape_for(cap, nqp, cs_req);
+        if (s.smem > static_cast<size_t>(kSmemPerCtaMax) || s.rmax > 512) s.cs = 0;
+        return s;
+    }
+    const int order[4] = {8, 16, 4, 2};
+    for (int i = 0; i < 4; ++i) {
+        Shape s = shape_for(cap, nqp, order[i]);
+        if (s.smem <= static_cast<size_t>(kSmemTwoPerSM) && s.rmax <= 512) return s;
+    }
+    for (int i = 0; i < 4; ++i) {
+        Shape s = shape_for(cap, nqp, order[i]);
+        if (s.smem <= static_cast<size_t>(kSmemPerCtaMax) && s.rmax <= 512) return s;
+    }
+    Shape none = {};
+    return none;
+}
+
+size_t ws_bytes_for(const rkv_config *cfg, int32_t n_layers, int32_t batch, int32_t cap) {
+    size_t n = kStatusBytes;
+    n += align256(static_cast<size_t>(batch) * 4);
+    if (cfg->redundancy_mode == RKV_RED_MAX)
+        n += align256(static_cast<size_t>(n_layers) * batch * cfg->n_kv_heads * cap * 4);
+    return n;
+}
+
+void fill_common(StepParams &p, const rkv_config *cfg, const Shape &s, int batch, int cap) {
+    p.batch = batch;
+    p.n_kv = cfg->n_kv_heads;
+    p.group = cfg->n_q_heads / cfg->n_kv_heads;
+    p.window = cfg->window;
+    p.cap = cap;
+    p.cs = s.cs;
+    p.rmax = s.rmax;
+    p.rp = s.rp;
+    p.tmem_cols = s.tmem_cols;
+    p.budget_cfg = cfg->budget;
+    p.lambda_cfg = cfg->mix_lambda;
+    p.logit_scale_log2 =
+        static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(kHeadDim)));
+    p.red_mode = cfg->redundancy_mode;
+    p.gqa_pool = cfg->gqa_pool;
+}
+
+rkv_status cuda_status(cudaError_t e) { return e == cudaSuccess ? RKV_OK : RKV_ERR_CUDA; }
+
+// Per-head entry points share this: one (sequence, layer), all KV heads.
+rkv_status run_per_head_scores(const rkv_config *cfg, const rkv_bf16 *q, const rkv_bf16 *k,
+                               int64_t head_stride, int32_t n_tokens, int32_t flags, float *I,
+                               float *inv, float *r, float *R, void *ws, size_t ws_bytes,
+                               cudaStream_t stream) {
+    const int cap = static_cast<int>(head_stride / kHeadDim);
+    const int nqp = nqp_of((cfg->n_q_heads / cfg->n_kv_heads) * cfg->window);
+    const Shape s = choose_shape(cap, nqp, 0);
+    if (s.cs == 0) return RKV_ERR_UNSUPPORTED;
+    if (cfg->redundancy_mode == RKV_RED_MAX && (flags & ~kFlagImportance) != 0 && (r || R))
+        return RKV_ERR_UNSUPPORTED;   // the MAX-mode similarity kernel is separate
+    StepParams *pp = new StepParams();
+    StepParams &p = *pp;
+    std::memset(&p, 0, sizeof(p));
+    fill_common(p, cfg, s, 1, cap);
+    p.n_layers = 1;
+    p.n_tokens_fixed = n_tokens;
+    p.flags = flags;
+    p.out_I = I;
+    p.out_inv = inv;
+    p.out_r = r;
+    p.out_R = R;
+    p.status = static_cast<uint32_t *>(ws);
+    p.red_mode = RKV_RED_MEAN;
+    bool ok = encode_rows128(&p.tmap_k[0], k, static_cast<uint64_t>(cfg->n_kv_heads) * cap, 16);
+    if (flags & kFlagImportance)
+        ok = ok && encode_rows128(&p.tmap_q[0], q,
+                                  static_cast<uint64_t>(cfg->n_q_heads) * cfg->window,
+                                  static_cast<uint32_t>(nqp));
+    if (!ok) {
+        delete pp;
+        return RKV_ERR_CUDA;
+    }
+    p.k[0] = const_cast<uint16_t *>(k);
+    cudaError_t e = cudaMemsetAsync(ws, 0, kStatusBytes, stream);
+    if (e == cudaSuccess) e = launch_step(p, cfg->n_kv_heads, nqp, s.smem, stream);
+    delete pp;
+    (void)ws_bytes;
+    return cuda_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *rkv_status_string(rkv_status s) {
+    switch (s) {
+        case RKV_OK: return "RKV_OK";
+        case RKV_STATUS_DISABLED: return "RKV_STATUS_DISABLED: budget or buffer <= 0, compression off";
+        case RKV_ERR_NULL: return "RKV_ERR_NULL: a required pointer is NULL";
+        case RKV_ERR_INVALID: return "RKV_ERR_INVALID: inconsistent sizes";
+        case RKV_ERR_ALIGN: return "RKV_ERR_ALIGN: a device pointer or stride is not 16-byte aligned";
+        case RKV_ERR_ALIAS: return "RKV_ERR_ALIAS: outputs overlap inputs";
+        case RKV_ERR_WORKSPACE: return "RKV_ERR_WORKSPACE: workspace missing or too small";
+        case RKV_ERR_UNSUPPORTED: return "RKV_ERR_UNSUPPORTED: shape outside the supported range";
+        case RKV_ERR_CUDA: return "RKV_ERR_CUDA: a CUDA call or launch failed";
+        case RKV_STATUS_DEVICE_TIMEOUT: return "RKV_STATUS_DEVICE_TIMEOUT: a device-side wait ran out";
+        case RKV_ERR_DEVICE_INPUT: return "RKV_ERR_DEVICE_INPUT: invalid device-side input";
+    }
+    return "unknown rkv_status";
+}
+
+int32_t rkv_version(void) { return kVersion; }
+
+size_t rkv_workspace_size(const rkv_config *cfg, int32_t n_layers, int32_t batch, int32_t cap) {
+    if (check_cfg(cfg) != RKV_OK || n_layers < 1 || batch < 1 || cap < 2) return 0;
+    return ws_bytes_for(cfg, n_layers, batch, cap);
+}
+
+rkv_status rkv_workspace_status(const void *workspace, rkv_stream_t stream) {
+    if (!workspace) return RKV_ERR_NULL;
+    uint32_t word = 0;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return RKV_ERR_CUDA;
+    if (word & kDevFlagTimeout) return RKV_STATUS_DEVICE_TIMEOUT;
+    if (word) return RKV_ERR_DEVICE_INPUT;
+    return RKV_OK;
+}
+
+rkv_status rkv_score_importance(const rkv_config *cfg, const rkv_bf16 *q, const rkv_bf16 *k,
+                                int64_t k_head_stride, int32_t n_tokens, float *I,
+                                float *inv_norm, void *workspace, size_t ws_bytes,
+                                rkv_stream_t stream) {
+    rkv_status st = check_cfg(cfg);
+    if (st != RKV_OK) return st;
+    if (!q || !k || !I) return RKV_ERR_NULL;
+    if (!workspace) return RKV_ERR_WORKSPACE;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(workspace)) return RKV_ERR_ALIGN;
+    if (k_head_stride % kHeadDim != 0) return RKV_ERR_ALIGN;
+    if (n_tokens <= cfg->window || k_head_stride < static_cast<int64_t>(n_tokens) * kHeadDim)
+        return RKV_ERR_INVALID;
+    const int cap = static_cast<int>(k_head_stride / kHeadDim);
+    if (ws_bytes < ws_bytes_for(cfg, 1, 1, cap)) return RKV_ERR_WORKSPACE;
+    return run_per_head_scores(cfg, q, k, k_head_stride, n_tokens, kFlagImportance | kFlagOutScores,
+                               I, inv_norm, nullptr, nullptr, workspace, ws_bytes,
+                               reinterpret_cast<cudaStream_t>(stream));
+}
+
+rkv_status rkv_score_redundancy(const rkv_config *cfg, const rkv_bf16 *k, int64_t k_head_stride,
+                                int32_t n_tokens, float *r, float *R, void *workspace,
+                                size_t ws_bytes, rkv_stream_t stream) {
+    rkv_status st = check_cfg(cfg);
+    if (st != RKV_OK) return st;
+    if (!workspace) return RKV_ERR_WORKSPACE;
+    if (!k || (!r && !R)) return RKV_ERR_NULL;
+    if (!aligned16(k) || !aligned16(workspace)) return RKV_ERR_ALIGN;
+    if (k_head_stride % kHeadDim != 0) return RKV_ERR_ALIGN;
+    if (n_tokens <= cfg->window || k_head_stride < static_cast<int64_t>(n_tokens) * kHeadDim)
+        return RKV_ERR_INVALID;
+    const int cap = static_cast<int>(k_head_stride / kHeadDim);
+    if (ws_bytes < ws_bytes_for(cfg, 1, 1, cap)) return RKV_ERR_WORKSPACE;
+    return run_per_head_scores(cfg, nullptr, k, k_head_stride, n_tokens, kFlagOutScores, nullptr,
+                               nullptr, r, R, workspace, ws_bytes,
+                               reinterpret_cast<cudaStream_t>(stream));
+}
+
+rkv_status rkv_select_topk(const rkv_config *cfg, const float *I, const float *R,
+                           int32_t n_tokens, int32_t *kept, float *Z, void *workspace,
+                           size_t ws_bytes, rkv_stream_t stream) {
+    rkv_status st = check_cfg(cfg);
+    if (st != RKV_OK) return st;
+    if (cfg->budget <= 0 || cfg->buffer <= 0) return RKV_STATUS_DISABLED;
+    if (!I || !R || !kept) return RKV_ERR_NULL;
+    if (!workspace) return RKV_ERR_WORKSPACE;
+    if (cfg->budget < cfg->window || cfg->budget > n_tokens || n_tokens <= cfg->window)
+        return RKV_ERR_INVALID;
+    const int M = n_tokens - cfg->window;
+    if (static_cast<size_t>(M) * 4 > static_cast<size_t>(kSmemPerCtaMax) - 4096)
+        return RKV_ERR_UNSUPPORTED;
+    if (ws_bytes < kStatusBytes) return RKV_ERR_WORKSPACE;
+    if (Z && (overlap(Z, static_cast<size_t>(M) * cfg->n_kv_heads * 4, I,
+                      static_cast<size_t>(M) * cfg->n_kv_heads * 4) ||
+              overlap(Z, static_cast<size_t>(M) * cfg->n_kv_heads * 4, R,
+                      static_cast<size_t>(M) * cfg->n_kv_heads * 4)))
+        return RKV_ERR_ALIAS;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytes, s);
+    if (e == cudaSuccess)
+        e = launch_select(I, R, cfg->n_kv_heads, M, n_tokens, cfg->budget, cfg->mix_lambda, kept, Z,
+                          static_cast<uint32_t *>(workspace), s);
+    return cuda_status(e);
+}
+
+rkv_status rkv_compact_kv(const rkv_config *cfg, const rkv_bf16 *k_src, const rkv_bf16 *v_src,
+                          const int32_t *kept, rkv_bf16 *k_dst, rkv_bf16 *v_dst,
+                          int64_t head_stride, int32_t n_tokens, void *workspace,
+                          size_t ws_bytes, rkv_stream_t stream) {
+    rkv_status st = check_cfg(cfg);
+    if (st != RKV_OK) return st;
+    if (cfg->budget <= 0 || cfg->buffer <= 0) return RKV_STATUS_DISABLED;
+    if (!k_src || !v_src || !kept || !k_dst || !v_dst) return RKV_ERR_NULL;
+    if (!workspace) return RKV_ERR_WORKSPACE;
+    if (ws_bytes < kStatusBytes) return RKV_ERR_WORKSPACE;
+    if (!aligned16(k_src) || !aligned16(v_src) || !aligned16(k_dst) || !aligned16(v_dst))
+        return RKV_ERR_ALIGN;
+    if (head_stride % 8 != 0) return RKV_ERR_ALIGN;
+    if (cfg->budget > n_tokens || head_stride < static_cast<int64_t>(n_tokens) * kHeadDim)
+        return RKV_ERR_INVALID;
+    const size_t extent =
+        (static_cast<size_t>(cfg->n_kv_heads - 1) * head_stride + static_cast<size_t>(n_tokens) * kHeadDim) * 2;
+    const bool k_same = k_dst == k_src, v_same = v_dst == v_src;
+    if (k_same != v_same) return RKV_ERR_ALIAS;
+    if (overlap(k_dst, extent, v_dst, extent) || overlap(k_src, extent, v_src, extent))
+        return RKV_ERR_ALIAS;
+    int cs = 0;
+    if (k_same) {
+        cs = compact_in_place_cluster(cfg->budget);
+        if (cs == 0) return RKV_ERR_UNSUPPORTED;
+    } else if (overlap(k_dst, extent, k_src, extent) || overlap(k_dst, extent, v_src, extent) ||
+               overlap(v_dst, extent, k_src, extent) || overlap(v_dst, extent, v_src, extent)) {
+        return RKV_ERR_ALIAS;
+    }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytes, s);
+    if (e == cudaSuccess)
+        e = launch_compact(k_src, v_src, kept, k_dst, v_dst, head_stride, cfg->n_kv_heads,
+                           cfg->budget, n_tokens, k_same, cs, static_cast<uint32_t *>(workspace), s);
+    return cuda_status(e);
+}
+
+rkv_status rkv_compress_step(const rkv_config *cfg, int32_t n_layers, int32_t batch, int32_t cap,
+                             rkv_bf16 *const *k_layers, rkv_bf16 *const *v_layers,
+                             const rkv_bf16 *const *q_layers, const int32_t *budgets,
+                             const float *lambdas, int32_t *cur_len,
+                             const rkv_step_options *opts, void *workspace, size_t ws_bytes,
+                             rkv_stream_t stream) {
+    rkv_status st = check_cfg(cfg);
+    if (st != RKV_OK) return st;
+    if (cfg->buffer <= 0 || (!budgets && cfg->budget <= 0)) return RKV_STATUS_DISABLED;
+    if (!k_layers || !v_layers || !q_layers || !cur_len) return RKV_ERR_NULL;
+    if (!workspace) return RKV_ERR_WORKSPACE;
+    if (n_layers < 1 || batch < 1 || cap < 2) return RKV_ERR_INVALID;
+    if (!budgets && (cfg->budget < cfg->window || cfg->budget >= cap)) return RKV_ERR_INVALID;
+    if (static_cast<int64_t>(batch) * cfg->n_kv_heads * cap > INT32_MAX ||
+        static_cast<int64_t>(batch) * cfg->n_q_heads * cfg->window > INT32_MAX)
+        return RKV_ERR_UNSUPPORTED;
+    const size_t layer_bytes = static_cast<size_t>(batch) * cfg->n_kv_heads * cap * kHeadDim * 2;
+    for (int l = 0; l < n_layers; ++l) {
+        if (!k_layers[l] || !v_layers[l] || !q_layers[l]) return RKV_ERR_NULL;
+        if (!aligned16(k_layers[l]) || !aligned16(v_layers[l]) || !aligned16(q_layers[l]))
+            return RKV_ERR_ALIGN;
+        if (overlap(k_layers[l], layer_bytes, v_layers[l], layer_bytes)) return RKV_ERR_ALIAS;
+    }
+    if (!aligned16(workspace) || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return RKV_ERR_ALIGN;
+    if (ws_bytes < ws_bytes_for(cfg, n_layers, batch, cap)) return RKV_ERR_WORKSPACE;
+    if (cfg->redundancy_mode == RKV_RED_MAX) return RKV_ERR_UNSUPPORTED;
+    const int nqp = nqp_of((cfg->n_q_heads / cfg->n_kv_heads) * cfg->window);
+    const Shape s = choose_shape(cap, nqp, opts ? opts->cluster_size : 0);
+    if (s.cs == 0) return RKV_ERR_UNSUPPORTED;
+    if (opts && opts->cluster_size && opts->cluster_size != 2 && opts->cluster_size != 4 &&
+        opts->cluster_size != 8 && opts->cluster_size != 16)
+        return RKV_ERR_INVALID;
+
+    cudaStream_t strm = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    uint32_t *status = reinterpret_cast<uint32_t *>(ws);
+    int32_t *n_eff = reinterpret_cast<int32_t *>(ws + kStatusBytes);
+
+    StepParams *pp = new StepParams();
+    StepParams &p = *pp;
+    std::memset(&p, 0, sizeof(p));
+    fill_common(p, cfg, s, batch, cap);
+    p.budgets = budgets;
+    p.lambdas = lambdas;
+    p.n_eff = n_eff;
+    p.flags = kFlagImportance | kFlagSelect;
+    p.kept_out = opts ? opts->kept_out : nullptr;
+    p.scores_out = opts ? opts->scores_out : nullptr;
+    p.status = status;
+
+    cudaError_t e = cudaMemsetAsync(ws, 0, kStatusBytes, strm);
+    if (e == cudaSuccess)
+        e = launch_plan(batch, budgets, cfg->budget, cfg->buffer, cfg->window, cap, cur_len, n_eff,
+                        status, strm);
+    if (e == cudaSuccess && opts && opts->main_begin)
+        e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->main_begin), strm);
+    for (int l0 = 0; e == cudaSuccess && l0 < n_layers; l0 += kMaxLayersPerLaunch) {
+        const int nl = (n_layers - l0 < kMaxLayersPerLaunch) ? n_layers - l0 : kMaxLayersPerLaunch;
+        p.n_layers = nl;
+        p.layer_base = l0;
+        for (int i = 0; i < nl; ++i) {
+            const int l = l0 + i;
+            if (!encode_rows128(&p.tmap_k[i], k_layers[l],
+                                static_cast<uint64_t>(batch) * cfg->n_kv_heads * cap, 16) ||
+                !encode_rows128(&p.tmap_q[i], q_layers[l],
+                                static_cast<uint64_t>(batch) * cfg->n_q_heads * cfg->window,
+                                static_cast<uint32_t>(nqp))) {
+                e = cudaErrorInvalidValue;
+                break;
+            }
+            p.k[i] = k_layers[l];
+            p.v[i] = v_layers[l];
+        }
+        if (e == cudaSuccess) e = launch_step(p, nl * batch * cfg->n_kv_heads, nqp, s.smem, strm);
+    }
+    if (e == cudaSuccess && opts && opts->main_end)
+        e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->main_end), strm);
+    delete pp;
+    return cuda_status(e);
+}
+
+}  // extern "C"
