@@ -1,0 +1,395 @@
+"""Benchmark of the R-KV decode-time KV compression step on B200.
+
+One step = one rkv_compress_step call over every layer, sequence and KV head
+of the workload (plan kernel + fused per-unit kernel), on a cache that is due
+for compression.  The step compacts the cache in place, so every warm-up and
+timed step gets its own pristine replica of the inputs, materialised in HBM
+before timing; each replica (K+V, 151 MB for the Llama3-8B-shaped step) is
+larger than the 126 MB L2, and a 256 MB buffer is written after the replicas
+are made, so every step starts from a cold L2.
+
+Metric: cached tokens compressed per second (sum over compressed units of
+their cached length N), and microseconds per step.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl rkv|reference]
+                  [--workload NAME] [--redundancy mean|max]
+
+Under torchrun (N > 1) every rank compresses its own batch (weak scaling,
+no collective on the data path); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from rkv_synth import WORKLOADS, bf16_bits, make_inputs  # noqa: E402
+
+METRIC = "cached tokens compressed/sec (all layers×heads); µs per compress step"
+UNIT = "tokens/s"
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "rkv_step_kernel.llama3_8b_step.traffic.txt")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="rkv", choices=["rkv", "reference"])
+    ap.add_argument("--workload", default="llama3_8b_step", choices=sorted(WORKLOADS))
+    ap.add_argument("--redundancy", default="mean", choices=["mean", "max"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- helpers
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_digest():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "decode_kv_cache_head_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(units_per_launch):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    if not os.path.exists(PROFILE_TRAFFIC):
+        return None
+    kv = {}
+    with open(PROFILE_TRAFFIC) as f:
+        for line in f:
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                kv[k.strip()] = v.strip()
+    if kv.get("kernel_source_sha256_16") != kernel_source_digest():
+        return None
+    try:
+        per_unit = float(kv["dram_bytes_per_unit"])
+    except (KeyError, ValueError):
+        return None
+    return per_unit * units_per_launch
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons of this rank's GPU, sampled in the background."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,utilization.gpu,"
+              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.path = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            gid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            gid = str(device_index)
+        self.gid = gid
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="rkv_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gid, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[0]), float(parts[1]), float(parts[2]),
+                                 float(parts[3]), parts[4:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        busy = [r for r in rows if r[3] > 0] or rows
+        names = ["active", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        reasons = sorted({names[i] for r in busy for i in range(1, 5)
+                          if r[4][i].lower() in ("active", "1")})
+        return {"sm_mhz": statistics.median(r[0] for r in busy),
+                "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": max(r[2] for r in rows),
+                "samples": len(rows), "samples_busy": len([r for r in rows if r[3] > 0]),
+                "reasons": reasons}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ----------------------------------------------------------------------------- reference arm
+def oracle_sample(w, red_mode):
+    """Inputs for the oracle arm: the first layer of the workload (all its units)."""
+    x = make_inputs(w, layers=[0])
+    G = w.n_q_heads // w.n_kv_heads
+    qb, kb = bf16_bits(x["Q"]), bf16_bits(x["K"])
+    units = [(b, h) for b in range(w.batch) for h in range(w.n_kv_heads)]
+    q = np.stack([qb[0, b, h * G:(h + 1) * G] for (b, h) in units])
+    k = np.stack([kb[0, b, h] for (b, h) in units])
+    N = np.array([int(x["cur_len"][b]) for (b, _) in units], dtype=np.int32)
+    bud = np.array([w.budget_of(b) for (b, _) in units], dtype=np.int32)
+    lam = np.full(len(units), w.mix_lambda)
+    return q, k, N, bud, lam
+
+
+def time_oracle(w, red_mode, reps, threads):
+    import oracle
+    q, k, N, bud, lam = oracle_sample(w, red_mode)
+    oracle.build()
+    times = []
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        oracle.units(q, k, N, bud, lam, red_mode=red_mode, n_threads=threads)
+        times.append(time.perf_counter() - t0)
+    tokens = int(N.sum())
+    return tokens, times, len(N)
+
+
+def run_reference(args, w, red_mode):
+    world, rank, _ = dist_setup(args)
+    if rank != 0:
+        return
+    threads = os.cpu_count() or 1
+    tokens, wt, units = time_oracle(w, red_mode, args.warmup, threads) if args.warmup else (0, [], 0)
+    tokens, times, units = time_oracle(w, red_mode, args.steps, threads)
+    per = sum(times) / len(times)
+    value = tokens / per
+    sample = (f"layer 0 of {w.name} ({units} units, {tokens} cached tokens) per step; "
+              f"C oracle, fp64, OpenMP over units")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w, red_mode, args),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w, red_mode, args):
+    return {"workload": w.name, "n_layers": w.n_layers, "batch": w.batch,
+            "n_kv_heads": w.n_kv_heads, "n_q_heads": w.n_q_heads, "head_dim": w.head_dim,
+            "budget": list(w.budgets) if len(w.budgets) > 1 else w.budgets[0],
+            "buffer": w.buffer, "window": w.window, "mix_lambda": w.mix_lambda,
+            "redundancy": "max" if red_mode else "mean", "gqa_pool": "max",
+            "cached_len": w.n_tokens()[0] if len(set(w.n_tokens())) == 1 else "ragged",
+            "near_duplicate_frac": list(w.dup_frac) if len(w.dup_frac) > 1 else w.dup_frac[0],
+            "l2": "fresh in-HBM replica per step (K+V larger than L2) and a 256 MB L2 flush "
+                  "before the timed region",
+            "parallelism": f"dp{args.gpus} (independent sequences per rank)"}
+
+
+# ----------------------------------------------------------------------------- rkv arm
+def run_rkv(args, w, red_mode):
+    world, rank, local = dist_setup(args)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=dev)
+    from decode_kv_cache_head_b200 import build
+    build.build()
+    import decode_kv_cache_head_b200 as rkv
+    from decode_kv_cache_head_b200 import dist as rdist
+
+    seed = rdist.rank_seed(w.seed, rank)
+    x = make_inputs(w, device=str(dev), seed=seed)
+    K0, V0, Q, cur0 = x["K"], x["V"], x["Q"], x["cur_len"].to(dev)
+    L, B, H, cap, D = K0.shape
+    cfg = rkv.make_config(w.budget_of(0), w.buffer, w.window, 128, w.n_kv_heads, w.n_q_heads,
+                          w.mix_lambda, redundancy_mode=red_mode)
+    budgets = None
+    if len(w.budgets) > 1:
+        budgets = torch.tensor([w.budget_of(b) for b in range(B)], dtype=torch.int32, device=dev)
+    ws = torch.zeros(rkv.rkv_workspace_size(cfg, L, B, cap), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(Kr, Vr, cr, events=None, kept=None):
+        rkv.rkv_compress_step(cfg, Kr, Vr, Q, cr, ws, budgets=budgets, kept_out=kept,
+                              events=events, stream=stream)
+
+    # exact moved-row count (rows whose destination differs from their source)
+    kept = torch.full((L, B, H, cap), -1, dtype=torch.int32, device=dev)
+    Kt, Vt, ct = K0.clone(), V0.clone(), cur0.clone()
+    step(Kt, Vt, ct, kept=kept)
+    torch.cuda.synchronize()
+    assert rkv.rkv_workspace_status(ws) == 0
+    kept_h = kept.cpu().numpy()
+    n_tok = np.array([w.budget_of(b) + w.buffer for b in range(B)])
+    moved = 0
+    for b in range(B):
+        kb = kept_h[:, b, :, :w.budget_of(b)]
+        moved += int((kb != np.arange(w.budget_of(b))[None, None, :]).sum())
+    del Kt, Vt, ct, kept
+    units = L * B * H
+    token_heads = int(L * H * n_tok.sum())
+    G = w.n_q_heads // w.n_kv_heads
+    alg_bytes = 256 * (L * H * int(n_tok.sum()) + units * G * w.window + 3 * moved)
+
+    # replicas: one pristine copy per warm-up and timed step
+    n_rep = args.warmup + args.steps
+    reps = [(K0.clone(), V0.clone(), cur0.clone()) for _ in range(n_rep)]
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    for a, b in ev:        # materialise the events before handing them to the library
+        a.record(stream); b.record(stream)
+    sampler = ClockSampler(local)
+    sampler.start()
+    for i in range(args.warmup):
+        step(*reps[i])
+    flush.fill_(1.0)
+    torch.cuda.synchronize()
+    rdist.barrier(dev)
+    torch.cuda.synchronize()
+    t_start, t_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(*reps[args.warmup + i], events=ev[i])
+    t_stop.record(stream)
+    torch.cuda.synchronize()
+    rdist.barrier(dev)
+    clocks = sampler.stop()
+    assert rkv.rkv_workspace_status(ws) == 0
+    elapsed_ms = t_start.elapsed_time(t_stop)
+    kern_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    elapsed_ms, kern_ms = rdist.max_over_ranks([elapsed_ms, kern_ms], dev)
+    del reps
+    ms_per_step = elapsed_ms / args.steps
+    value = world * token_heads / (ms_per_step / 1e3)
+
+    # end to end through host buffers: H2D of the inputs, the step, D2H of the result
+    e2e = None
+    if args.e2e_steps > 0:
+        hK, hV, hQ = K0.cpu().pin_memory(), V0.cpu().pin_memory(), Q.cpu().pin_memory()
+        hc = cur0.cpu().pin_memory()
+        oK, oV, oc = torch.empty_like(hK).pin_memory(), torch.empty_like(hV).pin_memory(), \
+            torch.empty_like(hc).pin_memory()
+        dK, dV, dQ, dc = torch.empty_like(K0), torch.empty_like(V0), torch.empty_like(Q), \
+            torch.empty_like(cur0)
+
+        def e2e_step():
+            dK.copy_(hK, non_blocking=True); dV.copy_(hV, non_blocking=True)
+            dQ.copy_(hQ, non_blocking=True); dc.copy_(hc, non_blocking=True)
+            rkv.rkv_compress_step(cfg, dK, dV, dQ, dc, ws, budgets=budgets, stream=stream)
+            oK.copy_(dK, non_blocking=True); oV.copy_(dV, non_blocking=True)
+            oc.copy_(dc, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        rdist.barrier(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = rdist.max_over_ranks([a.elapsed_time(b) / args.e2e_steps], dev)[0]
+        h2d = sum(t.numel() * t.element_size() for t in (hK, hV, hQ, hc))
+        d2h = sum(t.numel() * t.element_size() for t in (oK, oV, oc))
+        e2e = {"value": world * token_heads / (e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+
+    peak, peak_kind = measured_peaks()
+    achieved = alg_bytes / (kern_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": profiled_traffic(units),
+                "kernel": "rkv_step_kernel", "kernel_us_per_launch": kern_ms * 1e3,
+                "algorithmic_bytes_per_launch": alg_bytes, "peak_source": peak_kind,
+                "kernel_source_sha256_16": kernel_source_digest()}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        threads = os.cpu_count() or 1
+        tokens, times, nu = time_oracle(w, red_mode, 3, threads)
+        per = sorted(times)[1]
+        cpu = {"value": tokens / per, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"layer 0 of {w.name}: {nu} units, {tokens} cached tokens per run, "
+                         f"median of 3 runs, C oracle fp64 with OpenMP over units"}
+
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return
+    n_main_launches = (L + 31) // 32
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "us_per_step": ms_per_step * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": workload_config(w, red_mode, args),
+        "e2e": e2e, "gpu_launches": args.steps * (1 + n_main_launches),
+        "roofline": roofline, "cpu_baseline": cpu, "clocks": clocks,
+        "token_heads_per_step_per_gpu": token_heads,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    w = WORKLOADS[args.workload]
+    red_mode = 1 if args.redundancy == "max" else 0
+    if args.impl == "reference":
+        run_reference(args, w, red_mode)
+    else:
+        run_rkv(args, w, red_mode)
+
+
+if __name__ == "__main__":
+    main()
