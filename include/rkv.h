@@ -217,6 +217,41 @@ RKV_API rkv_status rkv_compress_step(const rkv_config *cfg, int32_t n_layers, in
                              const rkv_step_options *opts, void *workspace, size_t ws_bytes,
                              rkv_stream_t stream);
 
+/*
+ * The whole step as rkv_compress_step, for callers that cannot allocate
+ * device memory, so cannot hand over a workspace.  Examples are a plugin
+ * inside a serving engine that owns all of the GPU's memory, or a decode loop
+ * where an allocation (which may synchronise the device) is not allowed.  The
+ * R-KV pages have no counterpart: this is a packaging variant, not part of
+ * the method.
+ *
+ * Instead of a workspace the call uses a fixed scratch array of
+ * RKV_NOALLOC_SCRATCH_BYTES in the library's own device memory.  It holds a
+ * status header and one int32 per sequence, so batch is limited to
+ * RKV_NOALLOC_MAX_BATCH; a larger batch returns RKV_ERR_UNSUPPORTED, and so
+ * does any config whose workspace would not fit.  Every GPU on which the
+ * library is used keeps this array until the process exits.
+ *
+ * The first call on each device looks up the array's device address with
+ * cudaGetSymbolAddress (that device must be current), so make that first call
+ * before any stream capture.  The call allocates nothing (no cudaMalloc, no
+ * cudaFree, no allocating library routine).  All calls share the one array
+ * and it keeps whatever the last call left in it; the call resets what must
+ * start at zero itself.  Calls whose work overlaps on the GPU (two streams,
+ * two host threads) race on the array: serialise them.  Other arguments,
+ * results and statuses are those of rkv_compress_step.
+ */
+#define RKV_NOALLOC_MAX_BATCH 4096
+#define RKV_NOALLOC_SCRATCH_BYTES (256 + 4 * RKV_NOALLOC_MAX_BATCH)
+RKV_API rkv_status rkv_compress_step_noalloc(const rkv_config *cfg, int32_t n_layers,
+                                             int32_t batch, int32_t cap,
+                                             rkv_bf16 *const *k_layers,
+                                             rkv_bf16 *const *v_layers,
+                                             const rkv_bf16 *const *q_layers,
+                                             const int32_t *budgets, const float *lambdas,
+                                             int32_t *cur_len, const rkv_step_options *opts,
+                                             rkv_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
