@@ -54,6 +54,10 @@ def parse_args():
     ap.add_argument("--redundancy", default="mean", choices=["mean", "max"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--loop", action="store_true",
+                    help="run the whole decode loop of the workload (append + compress steps)")
+    ap.add_argument("--generated", type=int, default=16384,
+                    help="tokens generated per sequence in --loop mode")
     return ap.parse_args()
 
 
@@ -259,6 +263,7 @@ def run_rkv(args, w, red_mode):
     if len(w.budgets) > 1:
         budgets = torch.tensor([w.budget_of(b) for b in range(B)], dtype=torch.int32, device=dev)
     ws = torch.zeros(rkv.rkv_workspace_size(cfg, L, B, cap), dtype=torch.uint8, device=dev)
+    shape = rkv.rkv_query_step_shape(cfg, cap)
     stream = torch.cuda.current_stream()
 
     def step(Kr, Vr, cr, events=None, kept=None):
@@ -353,7 +358,8 @@ def run_rkv(args, w, red_mode):
                 "frac": achieved / peak, "traffic": profiled_traffic(units),
                 "kernel": "rkv_step_kernel", "kernel_us_per_launch": kern_ms * 1e3,
                 "algorithmic_bytes_per_launch": alg_bytes, "peak_source": peak_kind,
-                "kernel_source_sha256_16": kernel_source_digest()}
+                "kernel_source_sha256_16": kernel_source_digest(),
+                "cluster_size": shape[0], "rows_per_cta": shape[1], "smem_per_cta": shape[2]}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -381,12 +387,110 @@ def run_rkv(args, w, red_mode):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- decode loop
+def run_loop(args, w, red_mode):
+    """Steady-state decode loop: fill the cache to budget + buffer, compress, then
+    append `buffer` tokens and compress again until `--generated` tokens.  Only the
+    compression steps are timed (CUDA events around each call); the same cycle is
+    also replayed as a captured CUDA graph of (append + compress)."""
+    from decode_kv_cache_head_b200 import build
+    build.build()
+    import decode_kv_cache_head_b200 as rkv
+    from rkv_synth import DecodeTrace
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    L, B, H, D = w.n_layers, w.batch, w.n_kv_heads, w.head_dim
+    bud, buf, cap = w.budget_of(0), w.buffer, w.cap
+    cfg = rkv.make_config(bud, buf, w.window, D, H, w.n_q_heads, w.mix_lambda,
+                          redundancy_mode=red_mode)
+    K = torch.zeros((L, B, H, cap, D), dtype=torch.bfloat16, device=dev)
+    V = torch.zeros_like(K)
+    cur = torch.zeros(B, dtype=torch.int32, device=dev)
+    ws = torch.zeros(rkv.rkv_workspace_size(cfg, L, B, cap), dtype=torch.uint8, device=dev)
+    trace = DecodeTrace(w, device=str(dev))
+    stream = torch.cuda.current_stream()
+    evs = []
+
+    def compress(Q):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        rkv.rkv_compress_step(cfg, K, V, Q, cur, ws, stream=stream)
+        b.record(stream)
+        evs.append((a, b))
+
+    k_new, v_new = trace.chunk(cap, K, V, [0] * B)
+    rkv.rkv_append_kv(cfg, K, V, k_new, v_new, cur, ws, stream=stream)
+    del k_new, v_new
+    compress(trace.queries())
+    t = cap
+    while t + buf <= args.generated:
+        k_new, v_new = trace.chunk(buf, K, V, [bud] * B)
+        rkv.rkv_append_kv(cfg, K, V, k_new, v_new, cur, ws, stream=stream)
+        t += buf
+        compress(trace.queries())
+    torch.cuda.synchronize()
+    assert rkv.rkv_workspace_status(ws) == 0
+    assert cur.tolist() == [bud] * B
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    total_ms = sum(step_ms)
+
+    # the same cycle as a CUDA graph (append + compress), replayed on fixed buffers
+    kb = torch.empty((L, B, H, buf, D), dtype=torch.bfloat16, device=dev)
+    vb = torch.empty_like(kb)
+    Qb = torch.empty((L, B, w.n_q_heads, w.window, D), dtype=torch.bfloat16, device=dev)
+    kb.copy_(k_new); vb.copy_(v_new); Qb.copy_(trace.queries())
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            rkv.rkv_append_kv(cfg, K, V, kb, vb, cur, ws, stream=side)
+            rkv.rkv_compress_step(cfg, K, V, Qb, cur, ws, stream=side)
+    stream.wait_stream(side)
+    reps = 20
+    g_ms = []
+    for _ in range(reps):
+        k_new, v_new = trace.chunk(buf, K, V, [bud] * B)
+        kb.copy_(k_new); vb.copy_(v_new); Qb.copy_(trace.queries())
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        graph.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        g_ms.append(a.elapsed_time(b))
+    assert rkv.rkv_workspace_status(ws) == 0
+    del graph
+
+    token_heads = L * B * H * cap
+    full = L * B * H * args.generated * D * 2 * 2
+    line = {
+        "metric": METRIC, "value": len(step_ms) * token_heads / (total_ms / 1e3), "unit": UNIT,
+        "n_gpus": 1, "steps": len(step_ms), "warmup": 0, "ms_per_step": total_ms / len(step_ms),
+        "us_per_step": 1e3 * total_ms / len(step_ms), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(workload_config(w, red_mode, args), mode="decode_loop",
+                       generated_tokens=args.generated),
+        "loop": {"compress_steps": len(step_ms), "total_compress_ms": total_ms,
+                 "step_us_median": 1e3 * statistics.median(step_ms),
+                 "graph_append_plus_compress_us_median": 1e3 * statistics.median(g_ms),
+                 "full_cache_bytes": full,
+                 "capacity_cache_bytes": L * B * H * cap * D * 2 * 2,
+                 "compacted_cache_bytes": L * B * H * bud * D * 2 * 2,
+                 "capacity_fraction": cap / args.generated,
+                 "compacted_fraction": bud / args.generated},
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     w = WORKLOADS[args.workload]
     red_mode = 1 if args.redundancy == "max" else 0
     if args.impl == "reference":
         run_reference(args, w, red_mode)
+    elif args.loop:
+        run_loop(args, w, red_mode)
     else:
         run_rkv(args, w, red_mode)
 

@@ -18,8 +18,9 @@ __all__ = [
     "RKV_OK", "RKV_STATUS_DISABLED", "RKV_RED_MEAN", "RKV_RED_MAX", "RKV_GQA_MAX", "RKV_GQA_MEAN",
     "RkvError", "rkv_config", "rkv_step_options", "make_config", "library_path",
     "rkv_status_string", "rkv_version", "rkv_workspace_size", "rkv_workspace_status",
+    "rkv_query_step_shape",
     "rkv_score_importance", "rkv_score_redundancy", "rkv_select_topk", "rkv_compact_kv",
-    "rkv_compress_step",
+    "rkv_compress_step", "rkv_append_kv",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -71,12 +72,15 @@ def _load() -> ctypes.CDLL:
         "rkv_version": (I32, []),
         "rkv_workspace_size": (SZ, [CFG, I32, I32, I32]),
         "rkv_workspace_status": (ctypes.c_int, [P, P]),
+        "rkv_query_step_shape": (ctypes.c_int, [CFG, I32, ctypes.POINTER(I32), ctypes.POINTER(I32),
+                                                ctypes.POINTER(SZ)]),
         "rkv_score_importance": (ctypes.c_int, [CFG, P, P, I64, I32, P, P, P, SZ, P]),
         "rkv_score_redundancy": (ctypes.c_int, [CFG, P, I64, I32, P, P, P, SZ, P]),
         "rkv_select_topk": (ctypes.c_int, [CFG, P, P, I32, P, P, P, SZ, P]),
         "rkv_compact_kv": (ctypes.c_int, [CFG, P, P, P, P, P, I64, I32, P, SZ, P]),
         "rkv_compress_step": (ctypes.c_int, [CFG, I32, I32, I32, P, P, P, P, P, P,
                                              ctypes.POINTER(rkv_step_options), P, SZ, P]),
+        "rkv_append_kv": (ctypes.c_int, [CFG, I32, I32, I32, P, P, P, P, I32, P, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -137,6 +141,15 @@ def _check(status: int, where: str, allow_disabled: bool = False) -> int:
 
 def rkv_workspace_size(cfg: rkv_config, n_layers: int, batch: int, cap: int) -> int:
     return int(_lib.rkv_workspace_size(ctypes.byref(cfg), n_layers, batch, cap))
+
+
+def rkv_query_step_shape(cfg: rkv_config, cap: int):
+    """(cluster_size, rows_per_cta, smem_bytes) that rkv_compress_step uses for `cap` rows."""
+    cs, rows, smem = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_size_t()
+    _check(_lib.rkv_query_step_shape(ctypes.byref(cfg), int(cap), ctypes.byref(cs),
+                                     ctypes.byref(rows), ctypes.byref(smem)),
+           "rkv_query_step_shape")
+    return cs.value, rows.value, smem.value
 
 
 def rkv_workspace_status(workspace: torch.Tensor, stream=None) -> int:
@@ -223,3 +236,21 @@ def rkv_compress_step(cfg, k_layers, v_layers, q_layers, cur_len, workspace, bud
                                          _ptr(cur_len), ctypes.byref(opts), _ptr(workspace), ws,
                                          _stream(stream)), "rkv_compress_step",
                   allow_disabled=True)
+
+
+def rkv_append_kv(cfg, k_layers, v_layers, k_new_layers, v_new_layers, cur_len, workspace,
+                  stream=None):
+    """Appends [batch, Hkv, n_new, 128] rows per layer at cur_len, then cur_len += n_new."""
+    k_layers, v_layers = list(k_layers), list(v_layers)
+    k_new_layers, v_new_layers = list(k_new_layers), list(v_new_layers)
+    batch, _, cap, _ = k_layers[0].shape
+    n_new = k_new_layers[0].shape[2]
+    for t in k_layers + v_layers + k_new_layers + v_new_layers:
+        _dtype(t, torch.bfloat16, "k/v")
+    _dtype(cur_len, torch.int32, "cur_len")
+    ws = workspace.numel() * workspace.element_size()
+    return _check(_lib.rkv_append_kv(ctypes.byref(cfg), len(k_layers), batch, cap,
+                                     _ptr_array(k_layers), _ptr_array(v_layers),
+                                     _ptr_array(k_new_layers), _ptr_array(v_new_layers), n_new,
+                                     _ptr(cur_len), _ptr(workspace), ws, _stream(stream)),
+                  "rkv_append_kv")

@@ -99,7 +99,7 @@ Shape shape_for(int cap, int nqp, int cs) {
     s.rp = s.rmax < 128 ? 128 : s.rmax;
     const int ntiles = (s.rmax + 127) / 128;
     s.tmem_cols = pow2_at_least(ntiles * nqp);
-    s.smem = step_smem_bytes(s.rp, s.rmax, cap, nqp);
+    s.smem = step_smem_bytes(s.rp, s.rmax, cap, nqp, cs);
     // TMEM holds 512 columns per SM: never let more CTAs share an SM than fit,
     // by asking for enough shared memory to cap residency.
     const int max_res = 512 / s.tmem_cols;
@@ -166,8 +166,7 @@ rkv_status run_per_head_scores(const rkv_config *cfg, const rkv_bf16 *q, const r
     const int nqp = nqp_of((cfg->n_q_heads / cfg->n_kv_heads) * cfg->window);
     const Shape s = choose_shape(cap, nqp, 0);
     if (s.cs == 0) return RKV_ERR_UNSUPPORTED;
-    if (cfg->redundancy_mode == RKV_RED_MAX && (flags & ~kFlagImportance) != 0 && (r || R))
-        return RKV_ERR_UNSUPPORTED;   // the MAX-mode similarity kernel is separate
+    const bool red_max = cfg->redundancy_mode == RKV_RED_MAX && (r || R);
     StepParams *pp = new StepParams();
     StepParams &p = *pp;
     std::memset(&p, 0, sizeof(p));
@@ -180,20 +179,38 @@ rkv_status run_per_head_scores(const rkv_config *cfg, const rkv_bf16 *q, const r
     p.out_r = r;
     p.out_R = R;
     p.status = static_cast<uint32_t *>(ws);
-    p.red_mode = RKV_RED_MEAN;
+    p.red_mode = red_max ? RKV_RED_MAX : RKV_RED_MEAN;
     bool ok = encode_rows128(&p.tmap_k[0], k, static_cast<uint64_t>(cfg->n_kv_heads) * cap, 16);
     if (flags & kFlagImportance)
         ok = ok && encode_rows128(&p.tmap_q[0], q,
                                   static_cast<uint64_t>(cfg->n_q_heads) * cfg->window,
                                   static_cast<uint32_t>(nqp));
+    GramParams *gp = nullptr;
+    if (ok && red_max) {
+        gp = new GramParams();
+        std::memset(gp, 0, sizeof(*gp));
+        ok = encode_rows128(&gp->tmap[0], k, static_cast<uint64_t>(cfg->n_kv_heads) * cap, 128);
+        gp->batch = 1;
+        gp->n_kv = cfg->n_kv_heads;
+        gp->window = cfg->window;
+        gp->cap = cap;
+        gp->nblk = (cap - cfg->window + 127) / 128;
+        gp->n_tokens_fixed = n_tokens;
+        gp->r_out = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + kStatusBytes + 256);
+        gp->status = static_cast<uint32_t *>(ws);
+        p.r_ext = gp->r_out;
+    }
     if (!ok) {
         delete pp;
+        delete gp;
         return RKV_ERR_CUDA;
     }
     p.k[0] = const_cast<uint16_t *>(k);
     cudaError_t e = cudaMemsetAsync(ws, 0, kStatusBytes, stream);
+    if (e == cudaSuccess && gp) e = launch_gram_max(*gp, cfg->n_kv_heads, stream);
     if (e == cudaSuccess) e = launch_step(p, cfg->n_kv_heads, nqp, s.smem, stream);
     delete pp;
+    delete gp;
     (void)ws_bytes;
     return cuda_status(e);
 }
@@ -224,6 +241,20 @@ int32_t rkv_version(void) { return kVersion; }
 size_t rkv_workspace_size(const rkv_config *cfg, int32_t n_layers, int32_t batch, int32_t cap) {
     if (check_cfg(cfg) != RKV_OK || n_layers < 1 || batch < 1 || cap < 2) return 0;
     return ws_bytes_for(cfg, n_layers, batch, cap);
+}
+
+rkv_status rkv_query_step_shape(const rkv_config *cfg, int32_t cap, int32_t *cluster_size,
+                                int32_t *rows_per_cta, size_t *smem_bytes) {
+    const rkv_status st = check_cfg(cfg);
+    if (st != RKV_OK) return st;
+    if (cap < 2) return RKV_ERR_INVALID;
+    const int nqp = nqp_of((cfg->n_q_heads / cfg->n_kv_heads) * cfg->window);
+    const Shape s = choose_shape(cap, nqp, 0);
+    if (s.cs == 0) return RKV_ERR_UNSUPPORTED;
+    if (cluster_size) *cluster_size = s.cs;
+    if (rows_per_cta) *rows_per_cta = s.rmax;
+    if (smem_bytes) *smem_bytes = s.smem;
+    return RKV_OK;
 }
 
 rkv_status rkv_workspace_status(const void *workspace, rkv_stream_t stream) {
@@ -364,7 +395,6 @@ rkv_status rkv_compress_step(const rkv_config *cfg, int32_t n_layers, int32_t ba
     }
     if (!aligned16(workspace) || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return RKV_ERR_ALIGN;
     if (ws_bytes < ws_bytes_for(cfg, n_layers, batch, cap)) return RKV_ERR_WORKSPACE;
-    if (cfg->redundancy_mode == RKV_RED_MAX) return RKV_ERR_UNSUPPORTED;
     const int nqp = nqp_of((cfg->n_q_heads / cfg->n_kv_heads) * cfg->window);
     const Shape s = choose_shape(cap, nqp, opts ? opts->cluster_size : 0);
     if (s.cs == 0) return RKV_ERR_UNSUPPORTED;
@@ -376,6 +406,8 @@ rkv_status rkv_compress_step(const rkv_config *cfg, int32_t n_layers, int32_t ba
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     uint32_t *status = reinterpret_cast<uint32_t *>(ws);
     int32_t *n_eff = reinterpret_cast<int32_t *>(ws + kStatusBytes);
+    float *r_ext = reinterpret_cast<float *>(ws + kStatusBytes + align256(static_cast<size_t>(batch) * 4));
+    const bool red_max = cfg->redundancy_mode == RKV_RED_MAX;
 
     StepParams *pp = new StepParams();
     StepParams &p = *pp;
@@ -388,11 +420,34 @@ rkv_status rkv_compress_step(const rkv_config *cfg, int32_t n_layers, int32_t ba
     p.kept_out = opts ? opts->kept_out : nullptr;
     p.scores_out = opts ? opts->scores_out : nullptr;
     p.status = status;
+    p.r_ext = red_max ? r_ext : nullptr;
 
     cudaError_t e = cudaMemsetAsync(ws, 0, kStatusBytes, strm);
     if (e == cudaSuccess)
         e = launch_plan(batch, budgets, cfg->budget, cfg->buffer, cfg->window, cap, cur_len, n_eff,
                         status, strm);
+    if (red_max) {   // raw r of every candidate: the tcgen05 similarity kernel
+        GramParams *gp = new GramParams();
+        std::memset(gp, 0, sizeof(*gp));
+        gp->batch = batch;
+        gp->n_kv = cfg->n_kv_heads;
+        gp->window = cfg->window;
+        gp->cap = cap;
+        gp->nblk = (cap - cfg->window + 127) / 128;
+        gp->n_eff = n_eff;
+        gp->r_out = r_ext;
+        gp->status = status;
+        for (int l0 = 0; e == cudaSuccess && l0 < n_layers; l0 += kMaxLayersPerLaunch) {
+            const int nl = (n_layers - l0 < kMaxLayersPerLaunch) ? n_layers - l0 : kMaxLayersPerLaunch;
+            gp->layer_base = l0;
+            for (int i = 0; i < nl && e == cudaSuccess; ++i)
+                if (!encode_rows128(&gp->tmap[i], k_layers[l0 + i],
+                                    static_cast<uint64_t>(batch) * cfg->n_kv_heads * cap, 128))
+                    e = cudaErrorInvalidValue;
+            if (e == cudaSuccess) e = launch_gram_max(*gp, nl * batch * cfg->n_kv_heads, strm);
+        }
+        delete gp;
+    }
     if (e == cudaSuccess && opts && opts->main_begin)
         e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->main_begin), strm);
     for (int l0 = 0; e == cudaSuccess && l0 < n_layers; l0 += kMaxLayersPerLaunch) {
@@ -417,6 +472,56 @@ rkv_status rkv_compress_step(const rkv_config *cfg, int32_t n_layers, int32_t ba
     if (e == cudaSuccess && opts && opts->main_end)
         e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->main_end), strm);
     delete pp;
+    return cuda_status(e);
+}
+
+rkv_status rkv_append_kv(const rkv_config *cfg, int32_t n_layers, int32_t batch, int32_t cap,
+                         rkv_bf16 *const *k_layers, rkv_bf16 *const *v_layers,
+                         const rkv_bf16 *const *k_new_layers, const rkv_bf16 *const *v_new_layers,
+                         int32_t n_new, int32_t *cur_len, void *workspace, size_t ws_bytes,
+                         rkv_stream_t stream) {
+    rkv_status st = check_cfg(cfg);
+    if (st != RKV_OK) return st;
+    if (!k_layers || !v_layers || !k_new_layers || !v_new_layers || !cur_len) return RKV_ERR_NULL;
+    if (!workspace) return RKV_ERR_WORKSPACE;
+    if (ws_bytes < kStatusBytes) return RKV_ERR_WORKSPACE;
+    if (n_layers < 1 || batch < 1 || cap < 2 || n_new < 1 || n_new > cap) return RKV_ERR_INVALID;
+    const size_t layer_bytes = static_cast<size_t>(batch) * cfg->n_kv_heads * cap * kHeadDim * 2;
+    const size_t new_bytes = static_cast<size_t>(batch) * cfg->n_kv_heads * n_new * kHeadDim * 2;
+    for (int l = 0; l < n_layers; ++l) {
+        if (!k_layers[l] || !v_layers[l] || !k_new_layers[l] || !v_new_layers[l]) return RKV_ERR_NULL;
+        if (!aligned16(k_layers[l]) || !aligned16(v_layers[l]) || !aligned16(k_new_layers[l]) ||
+            !aligned16(v_new_layers[l]))
+            return RKV_ERR_ALIGN;
+        if (overlap(k_layers[l], layer_bytes, v_layers[l], layer_bytes) ||
+            overlap(k_new_layers[l], new_bytes, k_layers[l], layer_bytes) ||
+            overlap(k_new_layers[l], new_bytes, v_layers[l], layer_bytes) ||
+            overlap(v_new_layers[l], new_bytes, k_layers[l], layer_bytes) ||
+            overlap(v_new_layers[l], new_bytes, v_layers[l], layer_bytes))
+            return RKV_ERR_ALIAS;
+    }
+    cudaStream_t strm = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t *status = static_cast<uint32_t *>(workspace);
+    cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytes, strm);
+    AppendParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.batch = batch;
+    p.n_kv = cfg->n_kv_heads;
+    p.cap = cap;
+    p.n_new = n_new;
+    p.cur_len = cur_len;
+    p.status = status;
+    for (int l0 = 0; e == cudaSuccess && l0 < n_layers; l0 += kMaxLayersPerLaunch) {
+        const int nl = (n_layers - l0 < kMaxLayersPerLaunch) ? n_layers - l0 : kMaxLayersPerLaunch;
+        for (int i = 0; i < nl; ++i) {
+            p.k[i] = k_layers[l0 + i];
+            p.v[i] = v_layers[l0 + i];
+            p.k_new[i] = k_new_layers[l0 + i];
+            p.v_new[i] = v_new_layers[l0 + i];
+        }
+        e = launch_append(p, nl, strm);
+    }
+    if (e == cudaSuccess) e = launch_bump(batch, n_new, cap, cur_len, strm);
     return cuda_status(e);
 }
 

@@ -1,17 +1,17 @@
-// rkv_block.cuh -- block-level building blocks for 128-thread CTAs:
-// deterministic reductions (fixed butterfly order, then warps 0..3 in order),
-// 0/1 exclusive scans, a warp "transpose-reduce" that folds 16 per-thread
-// columns across the 32 lanes, the order-preserving key of a float, and a
-// radix select of the k-th largest 32-bit key.
+// rkv_block.cuh -- block-level building blocks, templated on the CTA's thread
+// count NT (a multiple of 32): deterministic reductions (fixed butterfly order,
+// then the warps in warp order), a merged (sum, max, sum-of-exp) reduction,
+// packed exclusive scans, a warp "transpose-reduce" that folds 16 per-thread
+// columns across the 32 lanes, the order-preserving key of a float, the joint
+// score, and a radix select of the k-th largest 32-bit key.
 #pragma once
 
 #include <cstdint>
 
 namespace rkv {
 
-constexpr int kThreads = 128;
-constexpr int kWarps = kThreads / 32;
 constexpr unsigned kFull = 0xffffffffu;
+constexpr float kLog2e = 1.4426950408889634f;
 
 struct OpSum {
     __device__ __forceinline__ float operator()(float a, float b) const { return a + b; }
@@ -27,9 +27,8 @@ __device__ __forceinline__ float warp_allreduce(float x, Op op) {
     return x;
 }
 
-// Every thread gets the same value: butterfly inside each warp, then the four
-// warp results combined in warp order.  `red` needs kWarps floats.
-template <class Op>
+// Every thread gets the same value.  `red` needs NT/32 floats.
+template <int NT, class Op>
 __device__ __forceinline__ float block_allreduce(float x, Op op, float *red) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     x = warp_allreduce(x, op);
@@ -37,35 +36,98 @@ __device__ __forceinline__ float block_allreduce(float x, Op op, float *red) {
     __syncthreads();
     float r = red[0];
 #pragma unroll
-    for (int w = 1; w < kWarps; ++w) r = op(r, red[w]);
+    for (int w = 1; w < NT / 32; ++w) r = op(r, red[w]);
     __syncthreads();
     return r;
 }
 
-// Exclusive prefix count of a 0/1 flag across the block in thread order;
-// `total` receives the block-wide count.  `sw` needs kWarps ints.
-__device__ __forceinline__ int block_excl_scan_flag(bool f, int *sw, int &total) {
+template <int NT>
+__device__ __forceinline__ uint32_t block_sum_u32(uint32_t x, uint32_t *red) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const unsigned m = __ballot_sync(kFull, f);
-    const int lane_pre = __popc(m & ((1u << lane) - 1u));
-    if (lane == 0) sw[warp] = __popc(m);
+    x = __reduce_add_sync(kFull, x);
+    if (lane == 0) red[warp] = x;
     __syncthreads();
-    int pre = 0, tot = 0;
+    uint32_t r = 0;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-        const int c = sw[w];
-        pre += (w < warp) ? c : 0;
+    for (int w = 0; w < NT / 32; ++w) r += red[w];
+    __syncthreads();
+    return r;
+}
+
+// (s, m, l): a plain sum s, and a running max m with l = sum exp(x - m).
+struct SumMaxExp {
+    float s, m, l;
+};
+
+__device__ __forceinline__ SumMaxExp merge_sme(SumMaxExp a, SumMaxExp b) {
+    SumMaxExp r;
+    r.s = a.s + b.s;
+    r.m = fmaxf(a.m, b.m);
+    const float la = (a.m == -INFINITY) ? 0.f : a.l * exp2f((a.m - r.m) * kLog2e);
+    const float lb = (b.m == -INFINITY) ? 0.f : b.l * exp2f((b.m - r.m) * kLog2e);
+    r.l = la + lb;
+    return r;
+}
+
+__device__ __forceinline__ SumMaxExp sme_add(SumMaxExp a, float s, float x) {
+    a.s += s;
+    if (x > a.m) {
+        a.l = ((a.m == -INFINITY) ? 0.f : a.l * exp2f((a.m - x) * kLog2e)) + 1.0f;
+        a.m = x;
+    } else {
+        a.l += exp2f((x - a.m) * kLog2e);
+    }
+    return a;
+}
+
+// `red` needs 4 * NT/32 floats.  Every thread gets the same result.
+template <int NT>
+__device__ __forceinline__ SumMaxExp block_reduce_sme(SumMaxExp v, float *red) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+        SumMaxExp o;
+        o.s = __shfl_xor_sync(kFull, v.s, off);
+        o.m = __shfl_xor_sync(kFull, v.m, off);
+        o.l = __shfl_xor_sync(kFull, v.l, off);
+        v = merge_sme(v, o);
+    }
+    if (lane == 0) {
+        red[4 * warp + 0] = v.s;
+        red[4 * warp + 1] = v.m;
+        red[4 * warp + 2] = v.l;
+    }
+    __syncthreads();
+    SumMaxExp r = {red[0], red[1], red[2]};
+#pragma unroll
+    for (int w = 1; w < NT / 32; ++w) r = merge_sme(r, SumMaxExp{red[4 * w], red[4 * w + 1], red[4 * w + 2]});
+    __syncthreads();
+    return r;
+}
+
+// Exclusive prefix sum of small packed counters across the block in thread
+// order; `total` receives the block-wide sum.  `sw` needs NT/32 uint32.
+template <int NT>
+__device__ __forceinline__ uint32_t block_excl_scan_u32(uint32_t v, uint32_t *sw, uint32_t &total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t inc = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t o = __shfl_up_sync(kFull, inc, off);
+        if (lane >= off) inc += o;
+    }
+    if (lane == 31) sw[warp] = inc;
+    __syncthreads();
+    uint32_t pre = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < NT / 32; ++w) {
+        const uint32_t c = sw[w];
+        pre += (w < warp) ? c : 0u;
         tot += c;
     }
     __syncthreads();
     total = tot;
-    return pre + lane_pre;
-}
-
-__device__ __forceinline__ int block_count(bool f, int *sw) {
-    int total;
-    block_excl_scan_flag(f, sw, total);
-    return total;
+    return pre + inc - v;
 }
 
 // Folds v[0..15] (16 columns held by every lane) across the warp: afterwards
@@ -100,57 +162,299 @@ __device__ __forceinline__ float joint_score(float lambda, float I, float R) {
     return __fsub_rn(__fmul_rn(lambda, I), __fmul_rn(__fsub_rn(1.0f, lambda), R));
 }
 
-// Radix select over keys[0..n) in shared memory (all threads call): T = the
-// kk-th largest key (1 <= kk <= n) and n_gt = the number of keys > T.
-// hist: 256 uint32, sh: 2 ints of shared scratch.
+// Radix select over keys[0..n) in shared memory (all NT threads call): T =
+// the kk-th largest key (1 <= kk <= n) and n_gt = the number of keys > T.
+// Four rounds of 8-bit digits, most significant first.  Each warp counts into
+// its own 256-bin histogram (one atomic per warp when all its lanes share the
+// digit, which is the common case in the first rounds), the bins are summed
+// over the warps and a block-wide suffix scan finds the digit holding the
+// kk-th largest key.  Key j is keys[j * STRIDE].  hist: (NT/32) * 256 uint32;
+// scan: NT/32 + 4 uint32.
+template <int NT, int STRIDE = 1>
 __device__ __forceinline__ void block_select_kth(const uint32_t *keys, int n, int kk,
-                                                 uint32_t *hist, int *sh, uint32_t &T,
+                                                 uint32_t *hist, uint32_t *scan, uint32_t &T,
                                                  int &n_gt) {
+    constexpr int NW = NT / 32;
+    static_assert(NT == 256, "one thread per histogram bin");
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint32_t *my = hist + warp * 256;
     uint32_t prefix = 0, mask = 0;
     int remaining = kk, above_total = 0;
 #pragma unroll 1
-    for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int i = tid; i < 256; i += kThreads) hist[i] = 0;
-        __syncthreads();
-        for (int j = tid; j < n; j += kThreads) {
-            const uint32_t key = keys[j];
-            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    for (int round = 0; round < 4; ++round) {
+        const int shift = 24 - 8 * round;
+#pragma unroll
+        for (int i = lane; i < 256; i += 32) my[i] = 0;
+        __syncwarp();
+        for (int base = 0; base < n; base += NT) {
+            const int j = base + tid;
+            const uint32_t key = (j < n) ? keys[j * STRIDE] : 0u;
+            const bool part = (j < n) && ((key & mask) == prefix);
+            const uint32_t digit = (key >> shift) & 255u;
+            const unsigned act = __ballot_sync(kFull, part);
+            if (act == 0) continue;
+            const uint32_t d0 = __shfl_sync(kFull, digit, __ffs(act) - 1);
+            if (__all_sync(kFull, !part || digit == d0)) {
+                if (lane == 0) my[d0] += static_cast<uint32_t>(__popc(act));
+            } else if (part) {
+                atomicAdd(&my[digit], 1u);
+            }
+            __syncwarp();
         }
         __syncthreads();
-        if (warp == 0) {
-            uint32_t c[8];
-            uint32_t s = 0;
+        // thread t owns bin 255 - t, so a prefix over threads is a suffix over bins
+        const int bin = 255 - tid;
+        uint32_t cnt = 0;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                c[i] = hist[8 * lane + i];
-                s += c[i];
-            }
-            uint32_t suf = s;  // inclusive suffix sum over lanes (higher lanes = higher bins)
+        for (int w = 0; w < NW; ++w) cnt += hist[w * 256 + bin];
+        uint32_t inc = cnt;
 #pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const uint32_t o = __shfl_down_sync(kFull, suf, off);
-                if (lane + off < 32) suf += o;
-            }
-            uint32_t above = suf - s;
+        for (int off = 1; off < 32; off <<= 1) {
+            const uint32_t o = __shfl_up_sync(kFull, inc, off);
+            if (lane >= off) inc += o;
+        }
+        if (lane == 31) scan[warp] = inc;
+        __syncthreads();
+        uint32_t above = inc - cnt;
 #pragma unroll
-            for (int i = 7; i >= 0; --i) {
-                if (above < static_cast<uint32_t>(remaining) &&
-                    above + c[i] >= static_cast<uint32_t>(remaining)) {
-                    sh[0] = 8 * lane + i;
-                    sh[1] = static_cast<int>(above);
-                }
-                above += c[i];
-            }
+        for (int w = 0; w < NW; ++w) above += (w < warp) ? scan[w] : 0u;
+        if (above < static_cast<uint32_t>(remaining) && above + cnt >= static_cast<uint32_t>(remaining)) {
+            scan[NW + 0] = static_cast<uint32_t>(bin);
+            scan[NW + 1] = above;
         }
         __syncthreads();
-        const uint32_t d = static_cast<uint32_t>(sh[0]);
-        const int above = sh[1];
-        __syncthreads();
+        const uint32_t d = scan[NW + 0];
+        const int ab = static_cast<int>(scan[NW + 1]);
         prefix |= d << shift;
         mask |= 255u << shift;
-        remaining -= above;
-        above_total += above;
+        remaining -= ab;
+        above_total += ab;
+        __syncthreads();   // scan[] and the histograms are reused by the next round
+    }
+    T = prefix;
+    n_gt = above_total;
+}
+
+// The same select with each thread's keys held in registers across the four
+// rounds (key j = keys[j * STRIDE] for j = tid + k * NT, k < KPT); needs
+// n <= KPT * NT.  Three block barriers per round.
+template <int NT, int KPT, int STRIDE>
+__device__ __forceinline__ void block_select_kth_reg(const uint32_t *keys, int n, int kk,
+                                                     uint32_t *hist, uint32_t *scan, uint32_t &T,
+                                                     int &n_gt) {
+    constexpr int NW = NT / 32;
+    static_assert(NT == 256, "one thread per histogram bin");
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int kpt = (n + NT - 1) / NT;
+    uint32_t kr[KPT];
+#pragma unroll
+    for (int k = 0; k < KPT; ++k) {
+        const int j = tid + k * NT;
+        kr[k] = (k < kpt && j < n) ? keys[j * STRIDE] : 0u;
+    }
+    uint32_t *my = hist + warp * 256;
+    uint32_t prefix = 0, mask = 0;
+    int remaining = kk, above_total = 0;
+#pragma unroll 1
+    for (int round = 0; round < 4; ++round) {
+        const int shift = 24 - 8 * round;
+#pragma unroll
+        for (int i = lane; i < 256; i += 32) my[i] = 0;
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < KPT; ++k) {
+            if (k < kpt) {
+                const int j = tid + k * NT;
+                const bool part = (j < n) && ((kr[k] & mask) == prefix);
+                const uint32_t digit = (kr[k] >> shift) & 255u;
+                const unsigned act = __ballot_sync(kFull, part);
+                if (act != 0) {
+                    const uint32_t d0 = __shfl_sync(kFull, digit, __ffs(act) - 1);
+                    if (__all_sync(kFull, !part || digit == d0)) {
+                        if (lane == 0) atomicAdd(&my[d0], static_cast<uint32_t>(__popc(act)));
+                    } else if (part) {
+                        atomicAdd(&my[digit], 1u);
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        const int bin = 255 - tid;   // a prefix over threads is a suffix over bins
+        uint32_t cnt = 0;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) cnt += hist[w * 256 + bin];
+        uint32_t inc = cnt;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const uint32_t o = __shfl_up_sync(kFull, inc, off);
+            if (lane >= off) inc += o;
+        }
+        if (lane == 31) scan[warp] = inc;
+        __syncthreads();
+        uint32_t above = inc - cnt;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) above += (w < warp) ? scan[w] : 0u;
+        if (above < static_cast<uint32_t>(remaining) && above + cnt >= static_cast<uint32_t>(remaining)) {
+            scan[NW + 0] = static_cast<uint32_t>(bin);
+            scan[NW + 1] = above;
+        }
+        __syncthreads();
+        const uint32_t d = scan[NW + 0];
+        const int ab = static_cast<int>(scan[NW + 1]);
+        prefix |= d << shift;
+        mask |= 255u << shift;
+        remaining -= ab;
+        above_total += ab;
+    }
+    T = prefix;
+    n_gt = above_total;
+    __syncthreads();   // the scan slots and histograms may be reused by the caller
+}
+
+// Radix select with the keys already in registers (thread tid holds keys
+// tid + k * NT, k < KPT; kv[k] false where there is no key) and one block
+// barrier per round: every warp adds into the round's shared 256-bin histogram
+// (one atomic per warp when all its lanes share the digit), zeroes the next
+// round's histogram, and after the barrier every warp scans the whole
+// histogram itself, so that no result needs to be written back.
+// hist: 4 * 256 uint32, whose first 256 entries must be zero on entry; the
+// call ends with all threads synchronised.  T = the kk-th largest key
+// (1 <= kk <= number of keys); n_gt = the number of keys above T.
+template <int NT, int KPT>
+__device__ __forceinline__ void block_select_kth_fast(const uint32_t (&kr)[KPT],
+                                                      const bool (&kv)[KPT], int kk,
+                                                      uint32_t *hist, uint32_t &T, int &n_gt) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    uint32_t prefix = 0, mask = 0;
+    int remaining = kk, above_total = 0;
+#pragma unroll 1
+    for (int round = 0; round < 4; ++round) {
+        const int shift = 24 - 8 * round;
+        uint32_t *H = hist + 256 * round;
+#pragma unroll
+        for (int k = 0; k < KPT; ++k) {
+            const bool part = kv[k] && ((kr[k] & mask) == prefix);
+            const uint32_t digit = (kr[k] >> shift) & 255u;
+            const unsigned act = __ballot_sync(kFull, part);
+            if (act != 0) {
+                const uint32_t d0 = __shfl_sync(kFull, digit, __ffs(act) - 1);
+                if (__all_sync(kFull, !part || digit == d0)) {
+                    if (lane == 0) atomicAdd(&H[d0], static_cast<uint32_t>(__popc(act)));
+                } else if (part) {
+                    atomicAdd(&H[digit], 1u);
+                }
+            }
+        }
+        if (round < 3)
+            for (int i = tid; i < 256; i += NT) H[256 + i] = 0;
+        __syncthreads();
+        // every warp: lane l holds bins 8l .. 8l + 7; suffix sums from the top bin down
+        const uint4 a = *reinterpret_cast<const uint4 *>(H + 8 * lane);
+        const uint4 b = *reinterpret_cast<const uint4 *>(H + 8 * lane + 4);
+        const uint32_t c[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        uint32_t s = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s += c[i];
+        uint32_t suf = s;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const uint32_t o = __shfl_down_sync(kFull, suf, off);
+            if (lane + off < 32) suf += o;
+        }
+        uint32_t above = suf - s, found_bin = 0, found_above = 0;
+        bool found = false;
+#pragma unroll
+        for (int i = 7; i >= 0; --i) {
+            if (!found && above < static_cast<uint32_t>(remaining) &&
+                above + c[i] >= static_cast<uint32_t>(remaining)) {
+                found = true;
+                found_bin = 8 * lane + i;
+                found_above = above;
+            }
+            above += c[i];
+        }
+        const int src = __ffs(__ballot_sync(kFull, found)) - 1;
+        const uint32_t d = __shfl_sync(kFull, found_bin, src);
+        const int ab = static_cast<int>(__shfl_sync(kFull, found_above, src));
+        prefix |= d << shift;
+        mask |= 255u << shift;
+        remaining -= ab;
+        above_total += ab;
+    }
+    T = prefix;
+    n_gt = above_total;
+    __syncthreads();   // the histograms may be reused by the caller
+}
+
+// The same select for 128-thread CTAs (two bins per thread).
+template <int NT>
+__device__ __forceinline__ void block_select_kth_small(const uint32_t *keys, int n, int kk,
+                                                       uint32_t *hist, uint32_t *scan,
+                                                       uint32_t &T, int &n_gt) {
+    constexpr int NW = NT / 32;
+    static_assert(NT == 128, "two bins per thread");
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint32_t *my = hist + warp * 256;
+    uint32_t prefix = 0, mask = 0;
+    int remaining = kk, above_total = 0;
+#pragma unroll 1
+    for (int round = 0; round < 4; ++round) {
+        const int shift = 24 - 8 * round;
+#pragma unroll
+        for (int i = lane; i < 256; i += 32) my[i] = 0;
+        __syncwarp();
+        for (int base = 0; base < n; base += NT) {
+            const int j = base + tid;
+            const uint32_t key = (j < n) ? keys[j] : 0u;
+            const bool part = (j < n) && ((key & mask) == prefix);
+            const uint32_t digit = (key >> shift) & 255u;
+            const unsigned act = __ballot_sync(kFull, part);
+            if (act == 0) continue;
+            const uint32_t d0 = __shfl_sync(kFull, digit, __ffs(act) - 1);
+            if (__all_sync(kFull, !part || digit == d0)) {
+                if (lane == 0) my[d0] += static_cast<uint32_t>(__popc(act));
+            } else if (part) {
+                atomicAdd(&my[digit], 1u);
+            }
+            __syncwarp();
+        }
+        __syncthreads();
+        // thread t owns bins 255 - 2t and 254 - 2t (descending)
+        const int b0 = 255 - 2 * tid, b1 = 254 - 2 * tid;
+        uint32_t c0 = 0, c1 = 0;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+            c0 += hist[w * 256 + b0];
+            c1 += hist[w * 256 + b1];
+        }
+        const uint32_t cnt = c0 + c1;
+        uint32_t inc = cnt;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const uint32_t o = __shfl_up_sync(kFull, inc, off);
+            if (lane >= off) inc += o;
+        }
+        if (lane == 31) scan[warp] = inc;
+        __syncthreads();
+        uint32_t above = inc - cnt;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) above += (w < warp) ? scan[w] : 0u;
+        const uint32_t rem = static_cast<uint32_t>(remaining);
+        if (above < rem && above + c0 >= rem) {
+            scan[NW + 0] = static_cast<uint32_t>(b0);
+            scan[NW + 1] = above;
+        } else if (above + c0 < rem && above + cnt >= rem) {
+            scan[NW + 0] = static_cast<uint32_t>(b1);
+            scan[NW + 1] = above + c0;
+        }
+        __syncthreads();
+        const uint32_t d = scan[NW + 0];
+        const int ab = static_cast<int>(scan[NW + 1]);
+        prefix |= d << shift;
+        mask |= 255u << shift;
+        remaining -= ab;
+        above_total += ab;
+        __syncthreads();
     }
     T = prefix;
     n_gt = above_total;

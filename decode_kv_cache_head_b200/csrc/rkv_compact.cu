@@ -26,6 +26,7 @@ namespace cg = cooperative_groups;
 namespace rkv {
 
 constexpr int kCompactMaxStageBytes = 200 * 1024;
+constexpr int kThreads = 128;
 
 __global__ void __launch_bounds__(256) rkv_gather_kernel(
     const uint16_t *__restrict__ k_src, const uint16_t *__restrict__ v_src,
@@ -53,7 +54,7 @@ __global__ void __launch_bounds__(kThreads, 1) rkv_compact_inplace_kernel(
     uint8_t *stage = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~static_cast<uintptr_t>(127));
     __shared__ uint64_t bar;
-    __shared__ float s_red[kWarps];
+    __shared__ float s_red[kThreads / 32];
     cg::cluster_group cluster = cg::this_cluster();
     const int cs = static_cast<int>(cluster.num_blocks());
     const int rank = static_cast<int>(cluster.block_rank());
@@ -83,7 +84,7 @@ __global__ void __launch_bounds__(kThreads, 1) rkv_compact_inplace_kernel(
         bulk_g2s(stage + i * 512 + 256, vh + static_cast<int64_t>(s) * kHeadDim, 256u, &bar);
         ++moved;
     }
-    moved = static_cast<int>(block_allreduce(static_cast<float>(moved), OpSum(), s_red));
+    moved = static_cast<int>(block_allreduce<kThreads>(static_cast<float>(moved), OpSum(), s_red));
     if (tid == 0) mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(moved) * 512u);
     bool ok = mbar_wait(&bar, 0);
     if (!ok) record_flag(status, kDevFlagTimeout);
@@ -122,14 +123,15 @@ cudaError_t launch_compact(const uint16_t *k_src, const uint16_t *v_src, const i
     }
     const int rb = (budget + cs - 1) / cs;
     const size_t smem = static_cast<size_t>(rb) * 512u + 128u;
-    cudaError_t e = cudaFuncSetAttribute(rkv_compact_inplace_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    static std::atomic<int> granted{0};
+    static std::atomic<bool> nonportable{false};
+    cudaError_t e = ensure_smem_attr(rkv_compact_inplace_kernel, smem, granted);
     if (e != cudaSuccess) return e;
-    if (cs > 8) {
+    if (cs > 8 && !nonportable.load()) {
         e = cudaFuncSetAttribute(rkv_compact_inplace_kernel,
                                  cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         if (e != cudaSuccess) return e;
+        nonportable.store(true);
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(n_kv * cs), 1, 1);

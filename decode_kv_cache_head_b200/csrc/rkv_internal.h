@@ -4,6 +4,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 
@@ -48,9 +49,11 @@ struct alignas(64) StepParams {
     uint32_t *status;
 };
 
+constexpr int kStepThreads = 256;     // threads per CTA of the fused kernel
+
 struct SmemLayout {
-    uint32_t k, q, v, inv, ss, ihat, rr, dst, keys, spart, gs, reds, statm, statl, gm, glinv,
-        red, hist, misc, bars, total;
+    uint32_t k, xstatm, xstatl, xs, hist, v, x, q, scratch, inv, ss, ihat, rr, dst, xp, gs, spart,
+        gm, glinv, vis, red, misc, bars, total;
 };
 
 __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) {
@@ -58,32 +61,65 @@ __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) {
 }
 
 // Offsets from a 1024-byte-aligned base; `total` includes 1024 bytes of slack
-// for aligning the dynamic shared-memory pointer.
-__host__ __device__ inline SmemLayout make_layout(int rp, int rmax, int cap, int nqp) {
+// for aligning the dynamic shared-memory pointer.  Regions whose names start
+// with x are written by the other CTAs of the cluster (one slot per CTA).
+// Lifetimes let regions share bytes:
+//  * the select histograms (after barrier 2) reuse the barrier-1 exchange slots;
+//  * region `x` first holds the query tile and the reduction scratch (both dead
+//    before this CTA reaches barrier 1), then the (Ihat, r) pairs that the
+//    cluster pushes after barrier 1, then, in place, the select keys.
+__host__ __device__ inline SmemLayout make_layout(int rp, int rmax, int cap, int nqp, int cs) {
     SmemLayout L;
     uint32_t o = 0;
-    L.k = o;      o += 2u * rp * 128u;
-    L.q = o;      o += 2u * nqp * 128u;
-    L.v = o;      o += static_cast<uint32_t>(rmax) * 256u;
+    L.k = o;      o += 2u * rp * 128u;                 // K rows, two 64-column swizzled halves
+    const uint32_t u0 = o;
+    L.xstatm = o; o += cs * nqp * 4u;                  // column max of every CTA
+    L.xstatl = o; o += cs * nqp * 4u;                  // column sum of exp of every CTA
+    L.xs = o;     o += cs * 128u * 4u;                 // S partial of every CTA
+    L.hist = u0;                                       // 8 warps x 256 bins
+    if (o - u0 < 8u * 256u * 4u) o = u0 + 8u * 256u * 4u;
+    o = align_up(o, 1024);
+    L.v = o;      o += static_cast<uint32_t>(rmax) * 256u;   // V rows, plain row-major
+    o = align_up(o, 1024);
+    L.x = o;
+    L.q = o;                                           // window queries (swizzled, 1024-aligned)
+    L.scratch = o + 2u * nqp * 128u;                   // 8 x 128 + 8 x nqp floats
+    const uint32_t xbytes = cap * 8u;
+    const uint32_t early = 2u * nqp * 128u + 8u * 128u * 4u + 8u * nqp * 4u;
+    o += align_up(xbytes > early ? xbytes : early, 16);
     L.inv = o;    o += align_up(rmax * 4u, 16);
     L.ss = o;     o += align_up(rmax * 4u, 16);
     L.ihat = o;   o += align_up(rmax * 4u, 16);
     L.rr = o;     o += align_up(rmax * 4u, 16);
     L.dst = o;    o += align_up(rmax * 4u, 16);
-    L.keys = o;   o += align_up(cap * 4u, 16);
-    L.spart = o;  o += 128u * 4u;
+    L.xp = o;     o += cs * 16u;                       // (sum Ihat, max r, sum exp r) of every CTA
     L.gs = o;     o += 128u * 4u;
-    L.reds = o;   o += 4u * 128u * 4u;
-    L.statm = o;  o += nqp * 4u;
-    L.statl = o;  o += nqp * 4u;
+    L.spart = o;  o += 128u * 4u;
     L.gm = o;     o += nqp * 4u;
     L.glinv = o;  o += nqp * 4u;
-    L.red = o;    o += 4u * nqp * 4u;
-    L.hist = o;   o += 256u * 4u;
+    L.vis = o;    o += 64u * 8u;
+    L.red = o;    o += 64u * 4u;
     L.misc = o;   o += 64u * 4u;
     L.bars = o;   o += 64u;
     L.total = o + 1024u;
     return L;
+}
+
+// Raises a kernel's dynamic shared-memory limit only when a launch needs more
+// than any earlier one (so repeated and graph-captured launches make no
+// attribute calls).  Per process; the value only grows.
+template <class K>
+inline cudaError_t ensure_smem_attr(K kernel, size_t bytes, std::atomic<int> &granted) {
+    if (static_cast<int>(bytes) <= granted.load(std::memory_order_relaxed)) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(bytes));
+    if (e == cudaSuccess) {
+        int cur = granted.load(std::memory_order_relaxed);
+        while (cur < static_cast<int>(bytes) &&
+               !granted.compare_exchange_weak(cur, static_cast<int>(bytes))) {
+        }
+    }
+    return e;
 }
 
 // Launchers (defined in the .cu files); all return cudaSuccess or the launch error.
@@ -92,7 +128,7 @@ cudaError_t launch_plan(int batch, const int32_t *budgets, int32_t budget_cfg, i
                         uint32_t *status, cudaStream_t stream);
 cudaError_t launch_step(const StepParams &p, int n_units, int nqp, size_t smem,
                         cudaStream_t stream);
-size_t step_smem_bytes(int rp, int rmax, int cap, int nqp);
+size_t step_smem_bytes(int rp, int rmax, int cap, int nqp, int cs);
 cudaError_t launch_select(const float *I, const float *R, int n_kv, int M, int N, int budget,
                           float lambda, int32_t *kept, float *Z, uint32_t *status,
                           cudaStream_t stream);
@@ -101,5 +137,29 @@ cudaError_t launch_compact(const uint16_t *k_src, const uint16_t *v_src, const i
                            int budget, int n_tokens, bool in_place, int cs, uint32_t *status,
                            cudaStream_t stream);
 int compact_in_place_cluster(int budget);   // 0: too large for the staged in-place path
+
+// MAX-mode similarity kernel: raw r of every candidate of every due unit.
+struct alignas(64) GramParams {
+    CUtensorMap tmap[kMaxLayersPerLaunch];   // [B*Hkv*cap rows, 128] bf16, box 64 x 128, SW128
+    int32_t layer_base, batch, n_kv, window, cap, nblk;
+    int32_t n_tokens_fixed;  // > 0: per-head entry point, N fixed
+    const int32_t *n_eff;
+    float *r_out;            // [units][cap]
+    uint32_t *status;
+};
+cudaError_t launch_gram_max(const GramParams &p, int n_units, cudaStream_t stream);
+
+struct AppendParams {
+    uint16_t *k[kMaxLayersPerLaunch];
+    uint16_t *v[kMaxLayersPerLaunch];
+    const uint16_t *k_new[kMaxLayersPerLaunch];
+    const uint16_t *v_new[kMaxLayersPerLaunch];
+    int32_t batch, n_kv, cap, n_new;
+    const int32_t *cur_len;
+    uint32_t *status;
+};
+cudaError_t launch_append(const AppendParams &p, int n_layers, cudaStream_t stream);
+cudaError_t launch_bump(int batch, int n_new, int cap, int32_t *cur_len, cudaStream_t stream);
+size_t gram_smem_bytes();
 
 }  // namespace rkv

@@ -13,28 +13,31 @@
 // importance from attention weights, cosine similarity for near-duplicates,
 // top-k within the budget).
 //
-// Work decomposition.  One cluster of `cs` CTAs (128 threads each) handles one
+// Work decomposition.  One cluster of `cs` CTAs (256 threads each) handles one
 // unit of N cached rows; CTA c owns rows [c*R, c*R + R) with R = ceil16(N/cs).
 //   1. TMA loads the CTA's K rows and the unit's G*w query rows into shared
-//      memory (128-byte swizzle), once; K is never read from HBM again.
+//      memory (128-byte swizzle); one bulk copy brings the CTA's V rows.  These
+//      are the only reads of K and V, and they finish before barrier 1.
 //   2. One thread issues tcgen05 UMMAs: logits[rows, G*w] = K_rows . Q^T into
 //      TMEM (M = 128 key rows per tile, N = G*w padded to 16, K = 128).
 //   3. Meanwhile all threads compute ||k_i||^2, 1/max(||k_i||, 1e-12) and the
 //      CTA's part of S = sum_i khat_i (for the mean-redundancy row sum).
 //   4. TMEM epilogue: per-query-column max and sum of exp over the CTA's
-//      visible keys; exchanged over DSMEM (cluster barrier 1).
+//      visible keys.  Every exchange is a push: each CTA stores its partials
+//      straight into its slot in every peer's shared memory, so that after a
+//      cluster barrier all reads are local (barrier 1).
 //   5. Per row: p = softmax probabilities, mean over the window, max over the
 //      group -> Ihat_i; r_i = (khat_i . S - khat_i . khat_i) / (N - 1) (MEAN)
-//      or r from the similarity kernel (MAX).  Partial sum Ihat, max r and
-//      sum exp(r - max) exchanged (cluster barrier 2).
-//   6. Every CTA pulls all candidates' Ihat and r over DSMEM, forms
-//      Z = lambda Ihat/sum - (1-lambda) exp(r - rmax)/rsum, and runs the same
-//      deterministic radix select (the k-th largest key, ties to the lower
-//      index), so all CTAs agree on the kept set without another exchange.
-//   7. Each CTA stages the V rows of its kept rows that move (bulk copies),
-//      cluster barrier 3 (all K and V reads of the unit are done), then writes
-//      its kept K rows (from shared memory) and V rows to their destinations.
-//      Reading everything before any write makes the in-place gather safe.
+//      or r from the similarity kernel (MAX).  (Ihat_i, r_i) and the partial
+//      sum Ihat / max r / sum exp(r - max) are pushed to every CTA (barrier 2).
+//   6. Every CTA forms Z = lambda Ihat/sum - (1-lambda) exp(r - rmax)/rsum for
+//      all candidates and runs the same deterministic radix select (the k-th
+//      largest key, ties to the lower index), so all CTAs agree on the kept
+//      set without another exchange.
+//   7. Each CTA writes its kept rows that move: K from its swizzled tile, V
+//      from its staging copy.  Since every read of the unit's K and V finished
+//      before barrier 1, these in-place writes cannot clobber a row that some
+//      CTA still has to read.
 #include <cooperative_groups.h>
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -85,15 +88,89 @@ cudaError_t launch_plan(int batch, const int32_t *budgets, int32_t budget_cfg, i
 // ----------------------------------------------------------------------------
 // The fused per-unit kernel.
 // ----------------------------------------------------------------------------
-template <int NQP>
-__global__ void __launch_bounds__(kThreads, 1) rkv_step_kernel(const __grid_constant__ StepParams p) {
+// After barrier 2: (sum Ihat, max r) and sum exp(r - max r) over all M
+// candidates from the local copies in xIR (thread tid holds candidates
+// tid + k * NT in registers), then, if `select`, each candidate's key
+// (also stored at sKeys[2j], in place over xIR) and the radix select.
+template <int NT, int KPT>
+__device__ __forceinline__ void post_exchange(const float2 *xIR, uint32_t *sKeys, uint32_t *sHist,
+                                              float *sRed, int M, int kk, float lam, bool select,
+                                              float &inv_sumI, float &rmax_g, float &inv_rsum,
+                                              uint32_t &T, int &n_gt) {
+    constexpr int NW = NT / 32;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    float ih[KPT], rr[KPT];
+    bool kv[KPT];
+    float sI = 0.f, mx = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < KPT; ++k) {
+        const int j = tid + k * NT;
+        kv[k] = j < M;
+        const float2 v = kv[k] ? xIR[j] : make_float2(0.f, -INFINITY);
+        ih[k] = v.x;
+        rr[k] = v.y;
+        sI += v.x;
+        mx = fmaxf(mx, v.y);
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+        sI += __shfl_xor_sync(kFull, sI, off);
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, off));
+    }
+    if (lane == 0) {
+        sRed[2 * warp] = sI;
+        sRed[2 * warp + 1] = mx;
+    }
+    for (int i = tid; i < 256; i += NT) sHist[i] = 0;   // first histogram of the select
+    __syncthreads();
+    sI = sRed[0];
+    mx = sRed[1];
+#pragma unroll
+    for (int w = 1; w < NW; ++w) {
+        sI += sRed[2 * w];
+        mx = fmaxf(mx, sRed[2 * w + 1]);
+    }
+    float e[KPT];
+    float rs = 0.f;
+#pragma unroll
+    for (int k = 0; k < KPT; ++k) {
+        e[k] = kv[k] ? ex2_approx((rr[k] - mx) * kLog2e) : 0.f;
+        rs += e[k];
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) rs += __shfl_xor_sync(kFull, rs, off);
+    if (lane == 0) sRed[2 * NW + warp] = rs;
+    __syncthreads();
+    rs = sRed[2 * NW];
+#pragma unroll
+    for (int w = 1; w < NW; ++w) rs += sRed[2 * NW + w];
+    inv_sumI = 1.0f / sI;
+    rmax_g = mx;
+    inv_rsum = 1.0f / rs;
+    if (!select) return;
+    uint32_t kr[KPT];
+#pragma unroll
+    for (int k = 0; k < KPT; ++k) {
+        kr[k] = ordered_key(joint_score(lam, ih[k] * inv_sumI, e[k] * inv_rsum));
+        if (kv[k]) sKeys[2 * (tid + k * NT)] = kr[k];
+    }
+    if (kk > 0) block_select_kth_fast<NT, KPT>(kr, kv, kk, sHist, T, n_gt);
+    else __syncthreads();
+}
+
+// NQP: query columns G*w rounded up to 16.  WC: the window size when it is
+// known at compile time (the common w = 8), 0 for a runtime window.
+template <int NQP, int WC>
+__global__ void __launch_bounds__(kStepThreads, 2) rkv_step_kernel(const __grid_constant__ StepParams p) {
+    constexpr int NT = kStepThreads;
+    constexpr int NW = NT / 32;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
 
     cg::cluster_group cluster = cg::this_cluster();
     const int cs = p.cs;
-    const uint32_t rank = cluster.block_rank();
+    const int rank = static_cast<int>(cluster.block_rank());
     const int unit = blockIdx.x / cs;
     const int h = unit % p.n_kv;
     const int b = (unit / p.n_kv) % p.batch;
@@ -103,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1) rkv_step_kernel(const __grid_cons
     const int N = p.n_tokens_fixed > 0 ? p.n_tokens_fixed : p.n_eff[b];
     if (N <= 0) return;  // not due: the whole cluster leaves before any exchange
 
-    const int w = p.window;
+    const int w = WC > 0 ? WC : p.window;
     const int G = p.group;
     const int NQ = G * w;
     const int M = N - w;
@@ -113,9 +190,10 @@ __global__ void __launch_bounds__(kThreads, 1) rkv_step_kernel(const __grid_cons
     const bool do_imp = (p.flags & kFlagImportance) != 0;
     const bool do_sel = (p.flags & kFlagSelect) != 0;
     const bool red_max = p.red_mode == RKV_RED_MAX;
+    const bool pool_max = p.gqa_pool == RKV_GQA_MAX;
 
     const int R = ((N + cs - 1) / cs + 15) / 16 * 16;
-    const int row0 = static_cast<int>(rank) * R;
+    const int row0 = rank * R;
     const int nrows = max(0, min(R, N - row0));
     const int nbox = (nrows + 15) / 16;
     const int nrows_pad = nbox * 16;
@@ -123,54 +201,70 @@ __global__ void __launch_bounds__(kThreads, 1) rkv_step_kernel(const __grid_cons
     const int64_t krow0 = (static_cast<int64_t>(b) * p.n_kv + h) * p.cap;   // row in the layer's 2D view
     const int64_t unit_g = (static_cast<int64_t>(p.layer_base + l) * p.batch + b) * p.n_kv + h;
 
-    const SmemLayout L = make_layout(p.rp, p.rmax, p.cap, NQP);
+    const SmemLayout L = make_layout(p.rp, p.rmax, p.cap, NQP, cs);
     uint8_t *sK = base + L.k;
-    uint8_t *sQ = base + L.q;
+    uint8_t *sQ = base + L.q;                                     // until the UMMAs complete
     uint8_t *sV = base + L.v;
+    float2 *xIR = reinterpret_cast<float2 *>(base + L.x);         // after barrier 1
+    uint32_t *sKeys = reinterpret_cast<uint32_t *>(base + L.x);   // key of candidate j at [2j]
+    float *sScratch = reinterpret_cast<float *>(base + L.scratch);  // before barrier 1 only
     float *sInv = reinterpret_cast<float *>(base + L.inv);
     float *sSS = reinterpret_cast<float *>(base + L.ss);
     float *sIhat = reinterpret_cast<float *>(base + L.ihat);
     float *sRr = reinterpret_cast<float *>(base + L.rr);
     int32_t *sDst = reinterpret_cast<int32_t *>(base + L.dst);
-    uint32_t *sKeys = reinterpret_cast<uint32_t *>(base + L.keys);
-    float *sSpart = reinterpret_cast<float *>(base + L.spart);
+    float *xStatM = reinterpret_cast<float *>(base + L.xstatm);
+    float *xStatL = reinterpret_cast<float *>(base + L.xstatl);
+    float4 *xS = reinterpret_cast<float4 *>(base + L.xs);
     float *sGS = reinterpret_cast<float *>(base + L.gs);
-    float *sRedS = reinterpret_cast<float *>(base + L.reds);
-    float *sStatM = reinterpret_cast<float *>(base + L.statm);
-    float *sStatL = reinterpret_cast<float *>(base + L.statl);
+    float *sSpart = reinterpret_cast<float *>(base + L.spart);
     float *sGM = reinterpret_cast<float *>(base + L.gm);
     float *sGLinv = reinterpret_cast<float *>(base + L.glinv);
-    float *sRed = reinterpret_cast<float *>(base + L.red);
+    uint64_t *sVis = reinterpret_cast<uint64_t *>(base + L.vis);
     uint32_t *sHist = reinterpret_cast<uint32_t *>(base + L.hist);
-    float *sMisc = reinterpret_cast<float *>(base + L.misc);   // [0..2]: published partials
-    float *sRed4 = sMisc + 8;                                   // block reduction scratch
-    int *sInt = reinterpret_cast<int *>(sMisc + 16);            // scan / select scratch
-    float *sGlob = sMisc + 32;                                  // cluster-wide scalars
+    float *sRed = reinterpret_cast<float *>(base + L.red);
+    uint32_t *sRedU = reinterpret_cast<uint32_t *>(base + L.red);
     uint64_t *bars = reinterpret_cast<uint64_t *>(base + L.bars);
-    uint64_t *bar_tma = bars + 0, *bar_mma = bars + 1, *bar_v = bars + 2;
+    uint64_t *bar_tma = bars + 0, *bar_mma = bars + 1;
     uint32_t *sTmem = reinterpret_cast<uint32_t *>(bars + 4);
+
+    // Query columns q = g * w + j.  colmask: columns that exist; lastmask: the
+    // last window query of each head (where the window mean is complete).
+    uint64_t colmask, lastmask;
+    {
+        const int j0 = lane % w, j1 = (lane + 32) % w;
+        colmask = static_cast<uint64_t>(__ballot_sync(kFull, lane < NQ)) |
+                  (static_cast<uint64_t>(__ballot_sync(kFull, lane + 32 < NQ)) << 32);
+        lastmask = static_cast<uint64_t>(__ballot_sync(kFull, lane < NQ && j0 == w - 1)) |
+                   (static_cast<uint64_t>(__ballot_sync(kFull, lane + 32 < NQ && j1 == w - 1)) << 32);
+        // key M + d (a window key) is seen by query j only when j >= d (causal)
+        if (warp == 0) {
+            for (int d = 0; d < w; ++d) {
+                const uint64_t m = static_cast<uint64_t>(__ballot_sync(kFull, lane < NQ && j0 >= d)) |
+                                   (static_cast<uint64_t>(__ballot_sync(kFull, lane + 32 < NQ && j1 >= d)) << 32);
+                if (lane == 0) sVis[d] = m;
+            }
+        }
+    }
 
     bool ok = true;  // false after a timed-out wait: keep joining barriers, skip the writes
 
-    // ---- set-up: TMEM, barriers, loads
+    // ---- set-up: TMEM, barriers, loads (K and Q by TMA, this CTA's V rows by one bulk copy)
     if (do_imp && warp == 0) {
         tmem_alloc(sTmem, static_cast<uint32_t>(p.tmem_cols));
         tmem_relinquish();
     }
-    if (tid == 0) {
+    // warp 1 starts the loads while warp 0 allocates TMEM
+    if (tid == 32) {
         mbar_init(bar_tma, 1);
         mbar_init(bar_mma, 1);
-        mbar_init(bar_v, 1);
         fence_mbar_init();
     }
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem_base = do_imp ? *sTmem : 0u;
-
-    if (tid == 0 && nrows > 0) {
+    if (tid == 32 && nrows > 0) {
         const CUtensorMap *mk = &p.tmap_k[l];
         const uint32_t bytes = static_cast<uint32_t>(nbox) * 4096u +
-                               (do_imp ? static_cast<uint32_t>(NQP) * 256u : 0u);
+                               (do_imp ? static_cast<uint32_t>(NQP) * 256u : 0u) +
+                               (do_sel ? static_cast<uint32_t>(nrows) * 256u : 0u);
         mbar_arrive_expect_tx(bar_tma, bytes);
         for (int bx = 0; bx < nbox; ++bx) {
             const int32_t y = static_cast<int32_t>(krow0 + row0 + bx * 16);
@@ -183,17 +277,22 @@ __global__ void __launch_bounds__(kThreads, 1) rkv_step_kernel(const __grid_cons
             tma_load_2d(sQ, mq, bar_tma, 0, yq);
             tma_load_2d(sQ + NQP * 128, mq, bar_tma, 64, yq);
         }
+        if (do_sel)
+            bulk_g2s(sV, p.v[l] + (krow0 + row0) * kHeadDim, static_cast<uint32_t>(nrows) * 256u,
+                     bar_tma);
     }
-    if (nrows > 0) {
-        if (!mbar_wait(bar_tma, 0)) {
-            ok = false;
-            record_flag(p.status, kDevFlagTimeout);
-        }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = do_imp ? *sTmem : 0u;
+
+    if (nrows > 0 && !mbar_wait(bar_tma, 0)) {
+        ok = false;
+        record_flag(p.status, kDevFlagTimeout);
     }
 
     // ---- UMMA: logits of every row against the G*w window queries
     auto tile_start = [&](int t) { return t < ntiles - 1 ? t * 128 : max(0, nrows_pad - 128); };
-    if (do_imp && nrows > 0 && tid == 0) {
+    if (do_imp && nrows > 0 && tid == kStepThreads - 32) {
         tc_fence_after();
         constexpr uint32_t idesc = idesc_bf16_f32(128, NQP);
         const uint32_t k_base = smem_u32(sK), q_base = smem_u32(sQ);
@@ -210,52 +309,62 @@ __global__ void __launch_bounds__(kThreads, 1) rkv_step_kernel(const __grid_cons
         umma_commit(bar_mma);
     }
 
-    // ---- norms (thread per row) while the tensor cores work
-    for (int t = 0; t < ntiles; ++t) {
-        const int row = tile_start(t) + tid;
+    // Rows: thread tid takes tiles t = tid/128, tid/128 + 2, ..., row tile_start(t) + tid%128,
+    // which is also the TMEM lane its warp reads.
+    const int t_first = tid >> 7, lane_row = tid & 127;
+    const uint32_t tmem_warp = tmem_base + ((32u * static_cast<uint32_t>(warp & 3)) << 16);
+
+    // ---- norms while the tensor cores work
+    for (int t = t_first; t < ntiles; t += 2) {
+        const int row = tile_start(t) + lane_row;
         if (row < t * 128 || row >= nrows) continue;
-        float ss = 0.f;
+        float2 ss2 = make_float2(0.f, 0.f);
 #pragma unroll 4
         for (int c = 0; c < 16; ++c) {
-            const uint8_t *src = sK + (c >> 3) * p.rp * 128 + sw128_offset(row, c & 7);
-            const uint4 raw = *reinterpret_cast<const uint4 *>(src);
+            const uint4 raw = *reinterpret_cast<const uint4 *>(sK + (c >> 3) * p.rp * 128 +
+                                                               sw128_offset(row, c & 7));
             const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const float2 f = __bfloat1622float2(h2[e]);
-                ss = fmaf(f.x, f.x, ss);
-                ss = fmaf(f.y, f.y, ss);
+                ss2 = __ffma2_rn(f, f, ss2);
             }
         }
+        const float ss = ss2.x + ss2.y;
         sSS[row] = ss;
         sInv[row] = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
     }
     __syncthreads();
 
-    // ---- this CTA's part of S = sum_i khat_i (warp w takes rows w, w+4, ...; lane: 4 columns)
+    // ---- this CTA's part of S = sum_i khat_i, pushed into every CTA's slot `rank`
     if (!red_max) {
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
         const int half = lane >> 4, cc = (lane & 15) >> 1, sub = lane & 1;
-        for (int row = warp; row < nrows; row += kWarps) {
-            const uint8_t *src = sK + half * p.rp * 128 + sw128_offset(row, cc) + sub * 8;
-            const uint2 raw = *reinterpret_cast<const uint2 *>(src);
+        for (int row = warp; row < nrows; row += NW) {
+            const uint2 raw = *reinterpret_cast<const uint2 *>(sK + half * p.rp * 128 +
+                                                               sw128_offset(row, cc) + sub * 8);
             const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
             const float iv = sInv[row];
-            const float2 f0 = __bfloat1622float2(h2[0]);
-            const float2 f1 = __bfloat1622float2(h2[1]);
-            acc[0] = fmaf(f0.x, iv, acc[0]);
-            acc[1] = fmaf(f0.y, iv, acc[1]);
-            acc[2] = fmaf(f1.x, iv, acc[2]);
-            acc[3] = fmaf(f1.y, iv, acc[3]);
+            const float2 iv2 = make_float2(iv, iv);
+            acc0 = __ffma2_rn(__bfloat1622float2(h2[0]), iv2, acc0);
+            acc1 = __ffma2_rn(__bfloat1622float2(h2[1]), iv2, acc1);
         }
         const int col = half * 64 + (lane & 15) * 4;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sRedS[warp * 128 + col + e] = acc[e];
+        *reinterpret_cast<float4 *>(sScratch + warp * 128 + col) = make_float4(acc0.x, acc0.y, acc1.x, acc1.y);
         __syncthreads();
-        sSpart[tid] = ((sRedS[tid] + sRedS[128 + tid]) + sRedS[256 + tid]) + sRedS[384 + tid];
+        if (tid < 128) {
+            float s = sScratch[tid];
+#pragma unroll
+            for (int w2 = 1; w2 < NW; ++w2) s += sScratch[w2 * 128 + tid];
+            sSpart[tid] = s;
+        }
+        __syncthreads();
+        const float4 *sp4 = reinterpret_cast<const float4 *>(sSpart);
+        for (int i = tid; i < cs * 32; i += NT)
+            cluster.map_shared_rank(xS, i >> 5)[rank * 32 + (i & 31)] = sp4[i & 31];
     }
 
-    // ---- softmax statistics of the CTA's rows for every query column
+    // ---- softmax statistics of the CTA's visible keys for every query column
     const float sc = p.logit_scale_log2;
     if (do_imp) {
         if (nrows > 0) {
@@ -265,274 +374,300 @@ __global__ void __launch_bounds__(kThreads, 1) rkv_step_kernel(const __grid_cons
             }
             tc_fence_after();
         }
+        float *sRedQ = sScratch + NW * 128;   // [NW][NQP]
+        const bool nopad = (NQ == NQP);
         // pass 1: column max (log2 domain)
-        float cm[NQP];
+        {
+            float cm[NQP];
 #pragma unroll
-        for (int q = 0; q < NQP; ++q) cm[q] = -INFINITY;
-        if (nrows > 0) {
-            for (int t = 0; t < ntiles; ++t) {
-                const int row = tile_start(t) + tid;
-                const bool valid = row >= t * 128 && row < nrows;
+            for (int q = 0; q < NQP; ++q) cm[q] = -INFINITY;
+            for (int t = t_first; t < ntiles; t += 2) {
+                const int row = tile_start(t) + lane_row;
                 const int gi = row0 + row;
+                const bool valid = row >= t * 128 && row < nrows;
+                // warp-uniform fast path: every row a candidate, every column real
+                const bool fast = nopad && __all_sync(kFull, valid && gi < M);
+                const uint64_t rm = !valid ? 0ull : (gi < M ? colmask : sVis[gi - M]);
 #pragma unroll
                 for (int c0 = 0; c0 < NQP; c0 += 16) {
                     float v[16];
-                    tmem_ld16(tmem_base + ((32u * warp) << 16) + t * NQP + c0, v);
+                    tmem_ld16(tmem_warp + t * NQP + c0, v);
+                    if (fast) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int q = c0 + i;
-                        const bool vis = valid && q < NQ && gi <= M + (q % w);
-                        cm[q] = fmaxf(cm[q], vis ? v[i] * sc : -INFINITY);
+                        for (int i = 0; i < 16; ++i) cm[c0 + i] = fmaxf(cm[c0 + i], v[i] * sc);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            cm[c0 + i] = fmaxf(cm[c0 + i], ((rm >> (c0 + i)) & 1ull) ? v[i] * sc : -INFINITY);
                     }
                 }
             }
-        }
 #pragma unroll
-        for (int c0 = 0; c0 < NQP; c0 += 16) {
-            float v[16];
+            for (int c0 = 0; c0 < NQP; c0 += 16) {
+                float v[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] = cm[c0 + i];
-            warp_transpose_reduce16(v, OpMax());
-            if (lane < 16) sRed[warp * NQP + c0 + lane] = v[0];
+                for (int i = 0; i < 16; ++i) v[i] = cm[c0 + i];
+                warp_transpose_reduce16(v, OpMax());
+                if (lane < 16) sRedQ[warp * NQP + c0 + lane] = v[0];
+            }
         }
         __syncthreads();
-        if (tid < NQP)
-            sStatM[tid] = fmaxf(fmaxf(sRed[tid], sRed[NQP + tid]),
-                                fmaxf(sRed[2 * NQP + tid], sRed[3 * NQP + tid]));
-        __syncthreads();
-        // pass 2: column sum of exp2(s - max) over the visible rows
-        float cl[NQP];
+        if (tid < NQP) {
+            float m = sRedQ[tid];
 #pragma unroll
-        for (int q = 0; q < NQP; ++q) cl[q] = 0.f;
-        if (nrows > 0) {
-            for (int t = 0; t < ntiles; ++t) {
-                const int row = tile_start(t) + tid;
-                const bool valid = row >= t * 128 && row < nrows;
+            for (int w2 = 1; w2 < NW; ++w2) m = fmaxf(m, sRedQ[w2 * NQP + tid]);
+            sGM[tid] = m;    // local column max (pushed to the cluster below)
+        }
+        __syncthreads();
+        // pass 2: exp2(s - local max), written back to TMEM (zero where not visible),
+        // and its column sums
+        {
+            float cl[NQP];
+#pragma unroll
+            for (int q = 0; q < NQP; ++q) cl[q] = 0.f;
+            for (int t = t_first; t < ntiles; t += 2) {
+                const int row = tile_start(t) + lane_row;
                 const int gi = row0 + row;
+                const bool valid = row >= t * 128 && row < nrows;
+                const bool fast = nopad && __all_sync(kFull, valid && gi < M);
+                const uint64_t rm = !valid ? 0ull : (gi < M ? colmask : sVis[gi - M]);
 #pragma unroll
                 for (int c0 = 0; c0 < NQP; c0 += 16) {
-                    float v[16];
-                    tmem_ld16(tmem_base + ((32u * warp) << 16) + t * NQP + c0, v);
+                    float v[16], mq[16];
+                    tmem_ld16(tmem_warp + t * NQP + c0, v);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int q = c0 + i;
-                        const bool vis = valid && q < NQ && gi <= M + (q % w);
-                        if (vis) cl[q] += exp2f(v[i] * sc - sStatM[q]);
+                    for (int i = 0; i < 16; ++i) mq[i] = sGM[c0 + i];
+                    if (fast) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            v[i] = ex2_approx(fmaf(v[i], sc, -mq[i]));
+                            cl[c0 + i] += v[i];
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const float e = ex2_approx(fmaf(v[i], sc, -mq[i]));
+                            v[i] = ((rm >> (c0 + i)) & 1ull) ? e : 0.f;
+                            cl[c0 + i] += v[i];
+                        }
                     }
+                    tmem_st16(tmem_warp + t * NQP + c0, v);
                 }
             }
-        }
 #pragma unroll
-        for (int c0 = 0; c0 < NQP; c0 += 16) {
-            float v[16];
+            for (int c0 = 0; c0 < NQP; c0 += 16) {
+                float v[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] = cl[c0 + i];
-            warp_transpose_reduce16(v, OpSum());
-            if (lane < 16) sRed[warp * NQP + c0 + lane] = v[0];
+                for (int i = 0; i < 16; ++i) v[i] = cl[c0 + i];
+                warp_transpose_reduce16(v, OpSum());
+                if (lane < 16) sRedQ[warp * NQP + c0 + lane] = v[0];
+            }
+            tmem_wait_st();
         }
         __syncthreads();
-        if (tid < NQP)
-            sStatL[tid] = ((sRed[tid] + sRed[NQP + tid]) + sRed[2 * NQP + tid]) + sRed[3 * NQP + tid];
+        for (int i = tid; i < cs * NQP; i += NT) {
+            const int q = i % NQP;
+            float s = sRedQ[q];
+#pragma unroll
+            for (int w2 = 1; w2 < NW; ++w2) s += sRedQ[w2 * NQP + q];
+            const int peer = i / NQP;
+            cluster.map_shared_rank(xStatM, peer)[rank * NQP + q] = sGM[q];
+            cluster.map_shared_rank(xStatL, peer)[rank * NQP + q] = s;
+        }
     }
-    __syncthreads();
 
-    // ================= cluster barrier 1: column statistics and S partials published
+    // ================= cluster barrier 1: column statistics and S partials delivered
     cluster.sync();
 
-    if (do_imp && tid < NQP) {
-        float m = -INFINITY;
-        for (int c = 0; c < cs; ++c) m = fmaxf(m, cluster.map_shared_rank(sStatM, c)[tid]);
-        float lsum = 0.f;
-        for (int c = 0; c < cs; ++c) {
-            const float mc = cluster.map_shared_rank(sStatM, c)[tid];
-            const float lc = cluster.map_shared_rank(sStatL, c)[tid];
-            if (mc != -INFINITY) lsum += lc * exp2f(mc - m);
+    // Cluster-wide column statistics and S: thread t takes CTA slot t % cs of
+    // column t / cs and the cs slots are folded with shuffles inside groups of
+    // cs lanes (same order in every CTA, so every CTA gets the same bits).
+    {
+        const int per = NT / cs;   // columns per pass
+        const int c = tid % cs, col = tid / cs;
+        if (do_imp) {
+            for (int q0 = 0; q0 < NQP; q0 += per) {
+                const int q = q0 + col;
+                const float mc = (q < NQP) ? xStatM[c * NQP + q] : -INFINITY;
+                float m = mc;
+                for (int off = 1; off < cs; off <<= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
+                float lsum = (mc != -INFINITY && q < NQP) ? xStatL[c * NQP + q] * ex2_approx(mc - m) : 0.f;
+                for (int off = 1; off < cs; off <<= 1) lsum += __shfl_xor_sync(kFull, lsum, off);
+                if (c == 0 && q < NQP) {
+                    // probabilities = (stored exp relative to this CTA's max) * factor
+                    const float mloc = xStatM[rank * NQP + q];
+                    sGLinv[q] = (lsum > 0.f && mloc != -INFINITY) ? ex2_approx(mloc - m) / lsum : 0.f;
+                }
+            }
         }
-        sGM[tid] = m;
-        sGLinv[tid] = (lsum > 0.f) ? 1.0f / lsum : 0.f;
-    }
-    if (!red_max) {
-        float s = 0.f;
-        for (int c = 0; c < cs; ++c) s += cluster.map_shared_rank(sSpart, c)[tid];
-        sGS[tid] = s;
+        if (!red_max) {
+            for (int d0 = 0; d0 < 32; d0 += per) {
+                const int d4 = d0 + col;
+                float4 v = (d4 < 32) ? xS[c * 32 + d4] : make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int off = 1; off < cs; off <<= 1) {
+                    v.x += __shfl_xor_sync(kFull, v.x, off);
+                    v.y += __shfl_xor_sync(kFull, v.y, off);
+                    v.z += __shfl_xor_sync(kFull, v.z, off);
+                    v.w += __shfl_xor_sync(kFull, v.w, off);
+                }
+                if (c == 0 && d4 < 32) reinterpret_cast<float4 *>(sGS)[d4] = v;
+            }
+        }
     }
     __syncthreads();
 
-    // ---- per row: importance Ihat_i, redundancy r_i
+    // ---- per row: importance Ihat_i, redundancy r_i; pushed to every CTA
     const float inv_w = 1.0f / static_cast<float>(w);
     const float inv_nm1 = 1.0f / static_cast<float>(N - 1);
-    float sumI = 0.f, rmax_loc = -INFINITY;
-    for (int t = 0; t < ntiles; ++t) {
-        const int row = tile_start(t) + tid;
+    for (int t = t_first; t < ntiles; t += 2) {
+        const int row = tile_start(t) + lane_row;
         const bool valid = row >= t * 128 && row < nrows;
         const int gi = row0 + row;
         float ihat = 0.f;
         if (do_imp) {
-            // loads are warp-collective: every lane takes part, valid or not
-            float run = 0.f, best = (p.gqa_pool == RKV_GQA_MAX) ? -INFINITY : 0.f;
+            // warp-collective loads: every lane takes part, valid or not
+            // TMEM now holds exp2(s - local max), zero where the key is not visible;
+            // probability = that value * per-column factor
+            float run = 0.f, best = pool_max ? -INFINITY : 0.f;
 #pragma unroll
             for (int c0 = 0; c0 < NQP; c0 += 16) {
-                float v[16];
-                tmem_ld16(tmem_base + ((32u * warp) << 16) + t * NQP + c0, v);
+                float v[16], fq[16];
+                tmem_ld16(tmem_warp + t * NQP + c0, v);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) fq[i] = sGLinv[c0 + i];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int q = c0 + i;
-                    if (q < NQ) {
-                        const int j = q % w;
-                        const float pr = (gi <= M + j) ? exp2f(v[i] * sc - sGM[q]) * sGLinv[q] : 0.f;
-                        run += pr;
-                        if (j == w - 1) {
+                    run = fmaf(v[i], fq[i], run);
+                    if (WC > 0) {
+                        if (q % (WC > 0 ? WC : 1) == WC - 1) {   // compile time: end of a head
                             const float a = run * inv_w;
-                            best = (p.gqa_pool == RKV_GQA_MAX) ? fmaxf(best, a) : best + a;
+                            best = pool_max ? fmaxf(best, a) : best + a;
                             run = 0.f;
                         }
+                    } else {
+                        const bool last = (lastmask >> q) & 1ull;
+                        const float a = run * inv_w;
+                        best = last ? (pool_max ? fmaxf(best, a) : best + a) : best;
+                        run = last ? 0.f : run;
                     }
                 }
             }
-            ihat = (p.gqa_pool == RKV_GQA_MAX) ? best : best / static_cast<float>(G);
+            ihat = pool_max ? best : best / static_cast<float>(G);
         }
         if (!valid || gi >= M) continue;
         float r;
         if (red_max) {
             r = p.r_ext[unit_g * p.cap + gi];
         } else {
-            float dot = 0.f;
+            float2 dot2 = make_float2(0.f, 0.f);
 #pragma unroll 4
             for (int c = 0; c < 16; ++c) {
-                const uint8_t *src = sK + (c >> 3) * p.rp * 128 + sw128_offset(row, c & 7);
-                const uint4 raw = *reinterpret_cast<const uint4 *>(src);
+                const uint4 raw = *reinterpret_cast<const uint4 *>(sK + (c >> 3) * p.rp * 128 +
+                                                                   sw128_offset(row, c & 7));
                 const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
                 const float4 s0 = *reinterpret_cast<const float4 *>(sGS + c * 8);
                 const float4 s1 = *reinterpret_cast<const float4 *>(sGS + c * 8 + 4);
-                const float2 f0 = __bfloat1622float2(h2[0]), f1 = __bfloat1622float2(h2[1]);
-                const float2 f2 = __bfloat1622float2(h2[2]), f3 = __bfloat1622float2(h2[3]);
-                dot = fmaf(f0.x, s0.x, dot); dot = fmaf(f0.y, s0.y, dot);
-                dot = fmaf(f1.x, s0.z, dot); dot = fmaf(f1.y, s0.w, dot);
-                dot = fmaf(f2.x, s1.x, dot); dot = fmaf(f2.y, s1.y, dot);
-                dot = fmaf(f3.x, s1.z, dot); dot = fmaf(f3.y, s1.w, dot);
+                dot2 = __ffma2_rn(__bfloat1622float2(h2[0]), make_float2(s0.x, s0.y), dot2);
+                dot2 = __ffma2_rn(__bfloat1622float2(h2[1]), make_float2(s0.z, s0.w), dot2);
+                dot2 = __ffma2_rn(__bfloat1622float2(h2[2]), make_float2(s1.x, s1.y), dot2);
+                dot2 = __ffma2_rn(__bfloat1622float2(h2[3]), make_float2(s1.z, s1.w), dot2);
             }
+            const float dot = dot2.x + dot2.y;
             const float iv = sInv[row];
             r = (iv * dot - iv * iv * sSS[row]) * inv_nm1;
         }
         sIhat[row] = ihat;
         sRr[row] = r;
-        sumI += ihat;
-        rmax_loc = fmaxf(rmax_loc, r);
+        const float2 ir = make_float2(ihat, r);
+        for (int c = 0; c < cs; ++c) cluster.map_shared_rank(xIR, c)[gi] = ir;
     }
-    sumI = block_allreduce(sumI, OpSum(), sRed4);
-    rmax_loc = block_allreduce(rmax_loc, OpMax(), sRed4);
-    float rsum = 0.f;
-    for (int t = 0; t < ntiles; ++t) {
-        const int row = tile_start(t) + tid;
-        const int gi = row0 + row;
-        if (row < t * 128 || row >= nrows || gi >= M) continue;
-        rsum += exp2f((sRr[row] - rmax_loc) * 1.4426950408889634f);
-    }
-    rsum = block_allreduce(rsum, OpSum(), sRed4);
-    if (tid == 0) {
-        sMisc[0] = sumI;
-        sMisc[1] = rmax_loc;
-        sMisc[2] = rsum;
-    }
-    __syncthreads();
-
-    // ================= cluster barrier 2: per-row scores and partial normalisers published
+    // ================= cluster barrier 2: every candidate's (Ihat, r) delivered.
+    // No CTA reads another's shared memory after this point, and every read of
+    // this unit's K and V in global memory finished before barrier 1.
     cluster.sync();
 
-    if (tid == 0) {
-        float si = 0.f, rm = -INFINITY;
-        for (int c = 0; c < cs; ++c) {
-            const float *pm = cluster.map_shared_rank(sMisc, c);
-            si += pm[0];
-            rm = fmaxf(rm, pm[1]);
-        }
-        float rs = 0.f;
-        for (int c = 0; c < cs; ++c) {
-            const float *pm = cluster.map_shared_rank(sMisc, c);
-            if (pm[1] != -INFINITY) rs += pm[2] * exp2f((pm[1] - rm) * 1.4426950408889634f);
-        }
-        sGlob[0] = si;
-        sGlob[1] = rm;
-        sGlob[2] = rs;
+    // Normalisers and keys from the local copies of every candidate's (Ihat, r):
+    // identical data and order in every CTA, hence identical bits everywhere.
+    float inv_sumI, rmax_g, inv_rsum;
+    uint32_t T = 0xffffffffu;
+    int n_gt = 0;
+    {
+        const bool sel = do_sel && nrows > 0;
+        if (M <= 5 * NT)
+            post_exchange<NT, 5>(xIR, sKeys, sHist, sRed, M, kk, lam, sel, inv_sumI, rmax_g, inv_rsum, T, n_gt);
+        else if (M <= 7 * NT)
+            post_exchange<NT, 7>(xIR, sKeys, sHist, sRed, M, kk, lam, sel, inv_sumI, rmax_g, inv_rsum, T, n_gt);
+        else if (M <= 9 * NT)
+            post_exchange<NT, 9>(xIR, sKeys, sHist, sRed, M, kk, lam, sel, inv_sumI, rmax_g, inv_rsum, T, n_gt);
+        else if (M <= 16 * NT)
+            post_exchange<NT, 16>(xIR, sKeys, sHist, sRed, M, kk, lam, sel, inv_sumI, rmax_g, inv_rsum, T, n_gt);
+        else
+            post_exchange<NT, 32>(xIR, sKeys, sHist, sRed, M, kk, lam, sel, inv_sumI, rmax_g, inv_rsum, T, n_gt);
     }
-    __syncthreads();
-    const float sumI_g = sGlob[0], rmax_g = sGlob[1], rsum_g = sGlob[2];
-    const float inv_rsum = 1.0f / rsum_g;
 
     if (p.flags & kFlagOutScores) {
-        // per-head entry points: write this CTA's rows and stop
-        for (int t = 0; t < ntiles; ++t) {
-            const int row = tile_start(t) + tid;
+        // per-head entry points: write this CTA's rows
+        for (int t = t_first; t < ntiles; t += 2) {
+            const int row = tile_start(t) + lane_row;
             const int gi = row0 + row;
             if (row < t * 128 || row >= nrows) continue;
             if (p.out_inv) p.out_inv[static_cast<int64_t>(h) * N + gi] = sInv[row];
             if (gi < M) {
                 const int64_t o = static_cast<int64_t>(h) * M + gi;
-                if (p.out_I) p.out_I[o] = sIhat[row] / sumI_g;
+                if (p.out_I) p.out_I[o] = sIhat[row] * inv_sumI;
                 if (p.out_r) p.out_r[o] = sRr[row];
-                if (p.out_R)
-                    p.out_R[o] = exp2f((sRr[row] - rmax_g) * 1.4426950408889634f) * inv_rsum;
+                if (p.out_R) p.out_R[o] = ex2_approx((sRr[row] - rmax_g) * kLog2e) * inv_rsum;
             }
         }
     }
 
-    if (do_sel) {
-        // ---- every CTA: keys of all M candidates (pulled over DSMEM), then the same select
-        for (int j = tid; j < M; j += kThreads) {
-            const int c = j / R, lr = j - c * R;
-            const float ih = cluster.map_shared_rank(sIhat, c)[lr];
-            const float rr = cluster.map_shared_rank(sRr, c)[lr];
-            const float I = ih / sumI_g;
-            const float Rv = exp2f((rr - rmax_g) * 1.4426950408889634f) * inv_rsum;
-            sKeys[j] = ordered_key(joint_score(lam, I, Rv));
-        }
-        __syncthreads();
-        uint32_t T = 0xffffffffu;
-        int n_gt = 0;
-        if (kk > 0) block_select_kth(sKeys, M, kk, sHist, sInt, T, n_gt);
+    if (do_sel && nrows > 0) {
         const int need_eq = (kk > 0) ? kk - n_gt : 0;
 
-        // kept rows before this CTA's range
+        // counts of candidates above / tied with the threshold before this CTA's rows
         const int lim = min(row0, M);
-        int c_gt = 0, c_eq = 0;
-        for (int j = tid; j < lim; j += kThreads) {
-            const uint32_t key = sKeys[j];
-            c_gt += (kk > 0 && key > T) ? 1 : 0;
-            c_eq += (kk > 0 && key == T) ? 1 : 0;
-        }
-        const int gt_before = static_cast<int>(block_allreduce(static_cast<float>(c_gt), OpSum(), sRed4));
-        const int eq_before = static_cast<int>(block_allreduce(static_cast<float>(c_eq), OpSum(), sRed4));
-        const int kept_before = gt_before + min(eq_before, need_eq) + max(0, row0 - M);
+        uint32_t packed = 0;
+        if (kk > 0)
+            for (int j = tid; j < lim; j += NT) {
+                const uint32_t key = sKeys[2 * j];
+                packed += (key > T ? 1u : 0u) + (key == T ? 65536u : 0u);
+            }
+        packed = block_sum_u32<NT>(packed, sRedU);
+        uint32_t g_run = (packed & 0xffffu) + static_cast<uint32_t>(max(0, row0 - M));
+        uint32_t e_run = packed >> 16;
 
-        int eq_run = 0, kept_run = 0;
-        for (int c0 = 0; c0 < nrows; c0 += kThreads) {
+        // kept flag and destination of each row: G_i = rows above the threshold or
+        // in the window before i, E_i = tied candidates before i;
+        // kept = above || window || (tied && E_i < need_eq), dst = G_i + min(E_i, need_eq)
+        for (int c0 = 0; c0 < nrows; c0 += NT) {
             const int row = c0 + tid;
             const int gi = row0 + row;
             const bool in = row < nrows;
             const bool cand = in && gi < M;
-            const uint32_t key = cand ? sKeys[gi] : 0u;
+            const uint32_t key = cand ? sKeys[2 * gi] : 0u;
             const bool eq = cand && kk > 0 && key == T;
-            int eq_tot;
-            const int eq_rank = eq_before + eq_run + block_excl_scan_flag(eq, sInt + 4, eq_tot);
-            const bool kept = in && (!cand || (kk > 0 && (key > T || (eq && eq_rank < need_eq))));
-            int kept_tot;
-            const int dst = kept_before + kept_run + block_excl_scan_flag(kept, sInt + 4, kept_tot);
-            if (in) sDst[row] = kept ? dst : -1;
-            eq_run += eq_tot;
-            kept_run += kept_tot;
+            const bool gw = in && (!cand || (kk > 0 && key > T));
+            uint32_t tot2;
+            const uint32_t ex = block_excl_scan_u32<NT>((eq ? 65536u : 0u) + (gw ? 1u : 0u), sRedU, tot2);
+            const uint32_t Ei = e_run + (ex >> 16), Gi = g_run + (ex & 0xffffu);
+            const bool kept = gw || (eq && Ei < static_cast<uint32_t>(need_eq));
+            if (in) sDst[row] = kept ? static_cast<int32_t>(Gi + min(Ei, static_cast<uint32_t>(need_eq))) : -1;
+            e_run += tot2 >> 16;
+            g_run += tot2 & 0xffffu;
         }
         __syncthreads();
 
         // optional outputs
         if (p.kept_out || p.scores_out) {
-            for (int row = tid; row < nrows; row += kThreads) {
+            for (int row = tid; row < nrows; row += NT) {
                 const int gi = row0 + row;
                 const int d = sDst[row];
                 if (p.kept_out && d >= 0) p.kept_out[unit_g * p.cap + d] = gi;
                 if (p.scores_out && gi < M) {
                     float *so = p.scores_out + unit_g * 4 * p.cap;
-                    const float I = sIhat[row] / sumI_g;
-                    const float Rv = exp2f((sRr[row] - rmax_g) * 1.4426950408889634f) * inv_rsum;
+                    const float I = sIhat[row] * inv_sumI;
+                    const float Rv = ex2_approx((sRr[row] - rmax_g) * kLog2e) * inv_rsum;
                     so[gi] = I;
                     so[p.cap + gi] = sRr[row];
                     so[2 * p.cap + gi] = Rv;
@@ -541,41 +676,21 @@ __global__ void __launch_bounds__(kThreads, 1) rkv_step_kernel(const __grid_cons
             }
         }
 
-        // ---- stage the V rows that move, then wait until the whole unit has read
-        const uint16_t *vsrc = p.v[l] + krow0 * kHeadDim;
-        int moved = 0;
-        for (int row = tid; row < nrows; row += kThreads) {
-            const int d = sDst[row];
-            if (d >= 0 && d != row0 + row) {
-                bulk_g2s(sV + row * 256, vsrc + static_cast<int64_t>(row0 + row) * kHeadDim, 256u,
-                         bar_v);
-                ++moved;
-            }
-        }
-        moved = static_cast<int>(block_allreduce(static_cast<float>(moved), OpSum(), sRed4));
-        if (tid == 0) mbar_arrive_expect_tx(bar_v, static_cast<uint32_t>(moved) * 256u);
-        if (!mbar_wait(bar_v, 0)) {
-            ok = false;
-            record_flag(p.status, kDevFlagTimeout);
-        }
+        // ---- compaction: kept rows that move, K from its swizzled tile, V from its staging
         ok = __syncthreads_and(ok);
-    }
-
-    // ================= cluster barrier 3: every read of this unit's K and V is done
-    cluster.sync();
-
-    if (do_sel && ok) {
-        uint16_t *kdst = p.k[l] + krow0 * kHeadDim;
-        uint16_t *vdst = p.v[l] + krow0 * kHeadDim;
-        for (int idx = tid; idx < nrows * 16; idx += kThreads) {
-            const int row = idx >> 4, c = idx & 15;
-            const int d = sDst[row];
-            if (d < 0 || d == row0 + row) continue;
-            const uint4 kx = *reinterpret_cast<const uint4 *>(sK + (c >> 3) * p.rp * 128 +
-                                                              sw128_offset(row, c & 7));
-            const uint4 vx = *reinterpret_cast<const uint4 *>(sV + row * 256 + c * 16);
-            *reinterpret_cast<uint4 *>(kdst + static_cast<int64_t>(d) * kHeadDim + c * 8) = kx;
-            *reinterpret_cast<uint4 *>(vdst + static_cast<int64_t>(d) * kHeadDim + c * 8) = vx;
+        if (ok) {
+            uint16_t *kdst = p.k[l] + krow0 * kHeadDim;
+            uint16_t *vdst = p.v[l] + krow0 * kHeadDim;
+            for (int idx = tid; idx < nrows * 16; idx += NT) {
+                const int row = idx >> 4, c = idx & 15;
+                const int d = sDst[row];
+                if (d < 0 || d == row0 + row) continue;
+                const uint4 kx = *reinterpret_cast<const uint4 *>(sK + (c >> 3) * p.rp * 128 +
+                                                                  sw128_offset(row, c & 7));
+                const uint4 vx = *reinterpret_cast<const uint4 *>(sV + row * 256 + c * 16);
+                *reinterpret_cast<uint4 *>(kdst + static_cast<int64_t>(d) * kHeadDim + c * 8) = kx;
+                *reinterpret_cast<uint4 *>(vdst + static_cast<int64_t>(d) * kHeadDim + c * 8) = vx;
+            }
         }
     }
 
@@ -586,24 +701,26 @@ __global__ void __launch_bounds__(kThreads, 1) rkv_step_kernel(const __grid_cons
     }
 }
 
-size_t step_smem_bytes(int rp, int rmax, int cap, int nqp) {
-    return make_layout(rp, rmax, cap, nqp).total;
+size_t step_smem_bytes(int rp, int rmax, int cap, int nqp, int cs) {
+    return make_layout(rp, rmax, cap, nqp, cs).total;
 }
 
-template <int NQP>
+template <int NQP, int WC>
 static cudaError_t launch_step_t(const StepParams &p, int n_units, size_t smem,
                                  cudaStream_t stream) {
-    auto kern = rkv_step_kernel<NQP>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    auto kern = rkv_step_kernel<NQP, WC>;
+    static std::atomic<int> granted{0};
+    static std::atomic<bool> nonportable{false};
+    cudaError_t e = ensure_smem_attr(kern, smem, granted);
     if (e != cudaSuccess) return e;
-    if (p.cs > 8) {
+    if (p.cs > 8 && !nonportable.load()) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         if (e != cudaSuccess) return e;
+        nonportable.store(true);
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(n_units * p.cs), 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.blockDim = dim3(kStepThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -618,11 +735,20 @@ static cudaError_t launch_step_t(const StepParams &p, int n_units, size_t smem,
 
 cudaError_t launch_step(const StepParams &p, int n_units, int nqp, size_t smem,
                         cudaStream_t stream) {
+    if (p.window == 8) {   // the window of every R-KV configuration on the pages
+        switch (nqp) {
+            case 16: return launch_step_t<16, 8>(p, n_units, smem, stream);
+            case 32: return launch_step_t<32, 8>(p, n_units, smem, stream);
+            case 48: return launch_step_t<48, 8>(p, n_units, smem, stream);
+            case 64: return launch_step_t<64, 8>(p, n_units, smem, stream);
+            default: return cudaErrorInvalidValue;
+        }
+    }
     switch (nqp) {
-        case 16: return launch_step_t<16>(p, n_units, smem, stream);
-        case 32: return launch_step_t<32>(p, n_units, smem, stream);
-        case 48: return launch_step_t<48>(p, n_units, smem, stream);
-        case 64: return launch_step_t<64>(p, n_units, smem, stream);
+        case 16: return launch_step_t<16, 0>(p, n_units, smem, stream);
+        case 32: return launch_step_t<32, 0>(p, n_units, smem, stream);
+        case 48: return launch_step_t<48, 0>(p, n_units, smem, stream);
+        case 64: return launch_step_t<64, 0>(p, n_units, smem, stream);
         default: return cudaErrorInvalidValue;
     }
 }

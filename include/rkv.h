@@ -132,6 +132,16 @@ RKV_API size_t rkv_workspace_size(const rkv_config *cfg, int32_t n_layers, int32
 RKV_API rkv_status rkv_workspace_status(const void *workspace, rkv_stream_t stream);
 
 /*
+ * The launch shape rkv_compress_step picks for caches of `cap` rows: CTAs per
+ * (sequence, layer, KV head) cluster, rows each CTA owns, and dynamic shared
+ * memory per CTA.  Host-only (no CUDA call).  RKV_ERR_UNSUPPORTED when no
+ * shape fits; any output pointer may be NULL.
+ */
+RKV_API rkv_status rkv_query_step_shape(const rkv_config *cfg, int32_t cap,
+                                        int32_t *cluster_size, int32_t *rows_per_cta,
+                                        size_t *smem_bytes);
+
+/*
  * Importance I for one (sequence, layer): step 1 of R-KV ("importance
  * (derived from attention weights)", [sourcepulse] How It Works; max pooling
  * over the GQA group, [atlas] Measured effects table).
@@ -216,6 +226,26 @@ RKV_API rkv_status rkv_compress_step(const rkv_config *cfg, int32_t n_layers, in
                              const float *lambdas, int32_t *cur_len,
                              const rkv_step_options *opts, void *workspace, size_t ws_bytes,
                              rkv_stream_t stream);
+
+/*
+ * The decode side of the loop: appends n_new tokens' keys and values to every
+ * sequence's cache at its current length, then cur_len[b] += n_new.  Together
+ * with rkv_compress_step this is the decode-time cycle of R-KV: tokens
+ * accumulate in the buffer until it holds divide_length = buffer new tokens,
+ * then the step compresses back to the budget ("applied periodically during
+ * decoding with a fixed buffer", [atlas] Approach).
+ * k_new_layers / v_new_layers: host arrays [n_layers] of device pointers to
+ * [batch][Hkv][n_new][128] bf16; k_layers / v_layers, cap and cur_len as in
+ * rkv_compress_step.  A sequence without room for n_new more rows is left
+ * untouched and reported through the workspace status (RKV_ERR_DEVICE_INPUT).
+ */
+RKV_API rkv_status rkv_append_kv(const rkv_config *cfg, int32_t n_layers, int32_t batch,
+                                 int32_t cap, rkv_bf16 *const *k_layers,
+                                 rkv_bf16 *const *v_layers,
+                                 const rkv_bf16 *const *k_new_layers,
+                                 const rkv_bf16 *const *v_new_layers, int32_t n_new,
+                                 int32_t *cur_len, void *workspace, size_t ws_bytes,
+                                 rkv_stream_t stream);
 
 /*
  * The whole step as rkv_compress_step, for callers that cannot allocate

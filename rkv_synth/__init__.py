@@ -169,6 +169,28 @@ def _ar1(eps: torch.Tensor, rho: float, chunk: int = 64) -> torch.Tensor:
     return out
 
 
+def _ar1_from_zero(drive: torch.Tensor, rho: float, chunk: int = 64) -> torch.Tensor:
+    """x_t = rho x_{t-1} + drive_t with x_{-1} = 0, along dim -2 (chunked matmuls)."""
+    n = drive.shape[-2]
+    t = torch.arange(chunk, device=drive.device, dtype=torch.float64)
+    diff = t[:, None] - t[None, :]
+    r = torch.tensor(rho, dtype=torch.float64, device=drive.device)
+    toep = torch.where(diff >= 0, torch.pow(r, diff.clamp(min=0)),
+                       torch.zeros((), dtype=torch.float64, device=drive.device)).to(torch.float32)
+    carry_w = torch.pow(r, t + 1).to(torch.float32)
+    out = torch.empty_like(drive)
+    prev = None
+    for c0 in range(0, n, chunk):
+        c1 = min(n, c0 + chunk)
+        m = c1 - c0
+        blk = torch.matmul(toep[:m, :m], drive[..., c0:c1, :])
+        if prev is not None:
+            blk = blk + carry_w[:m, None] * prev[..., None, :]
+        out[..., c0:c1, :] = blk
+        prev = blk[..., m - 1, :]
+    return out
+
+
 def _apply_runs(x: torch.Tensor, runs, noise_gen: torch.Generator, sigma: float) -> None:
     """In place on fp32 rows ``x[..., n, D]``: copy each run's source rows plus noise."""
     for (p, s, L) in runs:
@@ -220,3 +242,63 @@ def bf16_bits(t: torch.Tensor) -> np.ndarray:
     """Raw bf16 bit patterns of a tensor as a uint16 numpy array (host copy)."""
     assert t.dtype == torch.bfloat16
     return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+class DecodeTrace:
+    """New tokens of a steady-state decode loop, one chunk at a time, on the device.
+
+    Keys continue a stationary AR(1) process per (layer, sequence, KV head,
+    dimension); about ``dup_frac`` of each chunk's tokens are near-duplicate
+    runs (4..16 tokens) copied from rows currently in the cache, plus
+    N(0, 0.01^2) noise: a reasoning trace repeating context it still holds.
+    Values are N(0, 1) except in the copied runs.  Queries of the window are
+    fresh N(0, 1) every step.
+    """
+
+    def __init__(self, w: Workload, device: str = "cuda", seed: Optional[int] = None):
+        self.w = w
+        self.dev = device
+        s = w.seed if seed is None else seed
+        self.gen = torch.Generator(device=device)
+        self.gen.manual_seed(s * 7919 + 17)
+        self.rng = np.random.default_rng(s * 31 + 7)
+        L, B, H, D = w.n_layers, w.batch, w.n_kv_heads, w.head_dim
+        self.state = torch.randn((L, B, H, D), generator=self.gen, device=device)
+
+    def chunk(self, n: int, K: torch.Tensor, V: torch.Tensor, cur_len: Sequence[int]):
+        """n new tokens [L, B, H, n, D] (bf16) for K and V; copies read the cache K, V."""
+        w = self.w
+        L, B, H, D = w.n_layers, w.batch, w.n_kv_heads, w.head_dim
+        rho = w.ar_rho
+        eps = torch.randn((L, B, H, n, D), generator=self.gen, device=self.dev)
+        if rho > 0.0:
+            pw = torch.pow(torch.tensor(rho, device=self.dev), torch.arange(1, n + 1, device=self.dev,
+                                                                             dtype=torch.float32))
+            # AR(1) driven by eps from a zero start, plus the decayed previous state
+            drive = eps * float(np.sqrt(1.0 - rho * rho))
+            k = _ar1_from_zero(drive, rho) + pw[:, None] * self.state[..., None, :]
+        else:
+            k = eps
+        v = torch.randn((L, B, H, n, D), generator=self.gen, device=self.dev)
+        for b in range(B):
+            avail = int(cur_len[b])
+            target = int(round(self.w.dup_of(b) * n))
+            t = 0
+            covered = 0
+            while covered < target and t < n - 4 and avail > 16:
+                Lr = int(self.rng.integers(4, 17))
+                Lr = min(Lr, n - t, avail)
+                src = int(self.rng.integers(0, avail - Lr + 1))
+                k[:, b, :, t:t + Lr] = K[:, b, :, src:src + Lr].float() + 0.01 * torch.randn(
+                    (L, H, Lr, D), generator=self.gen, device=self.dev)
+                v[:, b, :, t:t + Lr] = V[:, b, :, src:src + Lr].float() + 0.01 * torch.randn(
+                    (L, H, Lr, D), generator=self.gen, device=self.dev)
+                covered += Lr
+                t += Lr + int(self.rng.integers(1, max(2, (n - covered) // 3)))
+        self.state = k[..., -1, :].clone()
+        return k.to(torch.bfloat16).contiguous(), v.to(torch.bfloat16).contiguous()
+
+    def queries(self):
+        w = self.w
+        return torch.randn((w.n_layers, w.batch, w.n_q_heads, w.window, w.head_dim),
+                           generator=self.gen, device=self.dev).to(torch.bfloat16)

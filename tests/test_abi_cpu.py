@@ -119,3 +119,13 @@ def test_per_head_entry_points_host_validation():
                             1152, A + (1 << 35), 4096, None) == -4
     assert L.rkv_compact_kv(cfgp, A + 2, A + (1 << 32), A + (1 << 34), A + 2, A + (1 << 32), hs,
                             1152, A + (1 << 35), 4096, None) == -3
+
+
+def test_step_shape_query():
+    """Two CTAs of the fused kernel must share an SM at the benchmark shapes."""
+    cs, rows, smem = rkv.rkv_query_step_shape(rkv.make_config(), 1152)
+    assert (cs, rows) == (8, 144) and smem <= 233472 // 2 - 1024
+    cs, rows, smem = rkv.rkv_query_step_shape(rkv.make_config(2048, n_q_heads=40), 2176)
+    assert rows * cs >= 2176 and smem <= 233472 // 2 - 1024
+    with pytest.raises(rkv.RkvError):
+        rkv.rkv_query_step_shape(rkv.make_config(head_dim=64), 1152)

@@ -163,3 +163,45 @@ def test_compaction_flags_out_of_range_index(rkv):
     Kd, Vd = torch.zeros_like(K), torch.zeros_like(V)
     rkv.rkv_compact_kv(cfg, K, V, kept, Kd, Vd, 48, ws)
     assert rkv.rkv_workspace_status(ws) == -9
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+def test_redundancy_max_on_the_tensor_cores(rkv, shape):
+    """MAX mode: r_i = max over the other keys of the cosine similarity (tcgen05 Gram)."""
+    n_kv, n_q, budget, buffer, window = shape
+    w, x = _case(n_kv, n_q, budget, buffer, window, seed=71 + budget)
+    N = budget + buffer
+    M = N - window
+    cfg = rkv.make_config(budget, buffer, window, 128, n_kv, n_q, 0.1,
+                          redundancy_mode=rkv.RKV_RED_MAX)
+    dev = torch.device("cuda")
+    k = x["K"][0, 0].to(dev)
+    r = torch.empty((n_kv, M), dtype=torch.float32, device=dev)
+    R = torch.empty((n_kv, M), dtype=torch.float32, device=dev)
+    ws = torch.zeros(rkv.rkv_workspace_size(cfg, 1, 1, w.cap), dtype=torch.uint8, device=dev)
+    rkv.rkv_score_redundancy(cfg, k, N, r, R, ws)
+    assert rkv.rkv_workspace_status(ws) == 0
+    kb = bf16_bits(x["K"][0, 0])
+    for h in range(n_kv):
+        rr = oracle.redundancy(kb[h], N, window, oracle.RED_MAX)
+        gc.check_scores(f"r head {h}", r[h].cpu().numpy(), rr)
+        gc.check_scores(f"M*R head {h}", R[h].cpu().numpy(), oracle.softmax(rr), scale=M)
+
+
+def test_redundancy_max_exact_copies_score_one(rkv):
+    dev = torch.device("cuda")
+    N, window = 300, 8
+    g = torch.Generator(device="cpu").manual_seed(5)
+    k = torch.randn((1, N, 128), generator=g).to(torch.bfloat16)
+    k[0, 200] = k[0, 17]
+    k[0, 250] = k[0, 17] * 4          # same direction, four times longer
+    cfg = rkv.make_config(200, 100, window, 128, 1, 4, 0.1, redundancy_mode=rkv.RKV_RED_MAX)
+    r = torch.empty((1, N - window), dtype=torch.float32, device=dev)
+    ws = torch.zeros(rkv.rkv_workspace_size(cfg, 1, 1, N), dtype=torch.uint8, device=dev)
+    rkv.rkv_score_redundancy(cfg, k.to(dev), N, r, None, ws)
+    rr = r[0].cpu()
+    for i in (17, 200, 250):
+        assert abs(float(rr[i]) - 1.0) < 1e-5
+    others = torch.ones(N - window, dtype=torch.bool)
+    others[[17, 200, 250]] = False
+    assert float(rr[others].max()) < 0.5

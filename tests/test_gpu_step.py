@@ -20,7 +20,7 @@ def rkv(cuda_device):
 
 
 def run_step(rkv, w, x, lam=None, budgets=None, lambdas=None, cur_len=None, cluster_size=0,
-             pool=0):
+             pool=0, red_mode=0):
     """Runs the fused step on copies of x's tensors; returns everything to compare."""
     dev = torch.device("cuda")
     K = x["K"].to(dev).clone()
@@ -29,7 +29,8 @@ def run_step(rkv, w, x, lam=None, budgets=None, lambdas=None, cur_len=None, clus
     L, B, H, cap, D = K.shape
     cur = (x["cur_len"] if cur_len is None else cur_len).to(dev).clone()
     cfg = rkv.make_config(w.budget_of(0), w.buffer, w.window, 128, w.n_kv_heads, w.n_q_heads,
-                          w.mix_lambda if lam is None else lam, gqa_pool=pool)
+                          w.mix_lambda if lam is None else lam, gqa_pool=pool,
+                          redundancy_mode=red_mode)
     ws = torch.zeros(rkv.rkv_workspace_size(cfg, L, B, cap), dtype=torch.uint8, device=dev)
     kept = torch.full((L, B, H, cap), -1, dtype=torch.int32, device=dev)
     scores = torch.full((L, B, H, 4, cap), float("nan"), dtype=torch.float32, device=dev)
@@ -41,12 +42,13 @@ def run_step(rkv, w, x, lam=None, budgets=None, lambdas=None, cur_len=None, clus
             "scores": scores.cpu().numpy()}
 
 
-def verify(w, x, out, units, budget_of, lam_of, pool=0, due=None):
+def verify(w, x, out, units, budget_of, lam_of, pool=0, due=None, red_mode=0):
     G = w.n_q_heads // w.n_kv_heads
     N_of = lambda b: int(x["cur_len"][b])
     due = due or (lambda b: True)
     units = [u for u in units if due(u[1])]
-    orc = gc.oracle_for_units(x["K"], x["Q"], units, N_of, budget_of, lam_of, G, pool=pool)
+    orc = gc.oracle_for_units(x["K"], x["Q"], units, N_of, budget_of, lam_of, G, pool=pool,
+                              red_mode=red_mode)
     und = []
     for i, (l, b, h) in enumerate(units):
         N, bud = N_of(b), budget_of(b)
@@ -174,3 +176,15 @@ def test_second_call_is_a_no_op(rkv):
     again = run_step(rkv, w, {"K": out["K"].cpu(), "V": out["V"].cpu(), "Q": x["Q"],
                               "cur_len": out["cur_len"].cpu()})
     assert torch.equal(again["K"], out["K"]) and torch.equal(again["V"], out["V"])
+
+
+@pytest.mark.parametrize("lam", [0.1, 0.0, 1.0])
+def test_max_redundancy_step(rkv, lam):
+    """The step in MAX mode: tcgen05 similarity kernel, then the fused kernel.  Near
+    duplicates make genuine near-ties under MAX; only decided tokens must agree."""
+    w = Workload("mx", 2, 2, 2, 8, 128, (1024, 700), seed=69)
+    x = make_inputs(w)
+    budgets = torch.tensor([1024, 700], dtype=torch.int32, device="cuda")
+    out = run_step(rkv, w, x, lam=lam, budgets=budgets, red_mode=1)
+    und = verify(w, x, out, all_units(w), w.budget_of, lambda b: lam, red_mode=1)
+    print(f"MAX mode lambda={lam}: undecided fraction {und:.4f}")
