@@ -41,7 +41,8 @@ from rkv_synth import WORKLOADS, bf16_bits, make_inputs  # noqa: E402
 
 METRIC = "cached tokens compressed/sec (all layers×heads); µs per compress step"
 UNIT = "tokens/s"
-PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "rkv_step_kernel.llama3_8b_step.traffic.txt")
+def profile_traffic_path(kernel, workload):
+    return os.path.join(ROOT, "profiles", f"{kernel}.{workload}.traffic.txt")
 
 
 def parse_args():
@@ -54,6 +55,9 @@ def parse_args():
     ap.add_argument("--redundancy", default="mean", choices=["mean", "max"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cluster-size", type=int, default=0,
+                    help="CTAs per unit: 0 = the library's choice, 1 = one CTA per unit, "
+                         "2/4/8/16 = a cluster per unit")
     ap.add_argument("--loop", action="store_true",
                     help="run the whole decode loop of the workload (append + compress steps)")
     ap.add_argument("--generated", type=int, default=16384,
@@ -81,13 +85,14 @@ def kernel_source_digest():
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(units_per_launch):
+def profiled_traffic(kernel, workload, units_per_launch):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
     the current kernel sources (else None)."""
-    if not os.path.exists(PROFILE_TRAFFIC):
+    path = profile_traffic_path(kernel, workload)
+    if not os.path.exists(path):
         return None
     kv = {}
-    with open(PROFILE_TRAFFIC) as f:
+    with open(path) as f:
         for line in f:
             if ":" in line and not line.startswith("#"):
                 k, v = line.split(":", 1)
@@ -263,11 +268,15 @@ def run_rkv(args, w, red_mode):
     if len(w.budgets) > 1:
         budgets = torch.tensor([w.budget_of(b) for b in range(B)], dtype=torch.int32, device=dev)
     ws = torch.zeros(rkv.rkv_workspace_size(cfg, L, B, cap), dtype=torch.uint8, device=dev)
-    shape = rkv.rkv_query_step_shape(cfg, cap)
+    shape = rkv.rkv_query_step_shape(cfg, L * B * H, cap)
+    if args.cluster_size:
+        shape = (args.cluster_size, cap if args.cluster_size == 1 else shape[1], shape[2])
+    kernel_name = "rkv_unit_kernel" if shape[0] == 1 else "rkv_step_kernel"
     stream = torch.cuda.current_stream()
 
     def step(Kr, Vr, cr, events=None, kept=None):
         rkv.rkv_compress_step(cfg, Kr, Vr, Q, cr, ws, budgets=budgets, kept_out=kept,
+                              cluster_size=args.cluster_size,
                               events=events, stream=stream)
 
     # exact moved-row count (rows whose destination differs from their source)
@@ -333,7 +342,8 @@ def run_rkv(args, w, red_mode):
         def e2e_step():
             dK.copy_(hK, non_blocking=True); dV.copy_(hV, non_blocking=True)
             dQ.copy_(hQ, non_blocking=True); dc.copy_(hc, non_blocking=True)
-            rkv.rkv_compress_step(cfg, dK, dV, dQ, dc, ws, budgets=budgets, stream=stream)
+            rkv.rkv_compress_step(cfg, dK, dV, dQ, dc, ws, budgets=budgets,
+                                  cluster_size=args.cluster_size, stream=stream)
             oK.copy_(dK, non_blocking=True); oV.copy_(dV, non_blocking=True)
             oc.copy_(dc, non_blocking=True)
 
@@ -355,8 +365,8 @@ def run_rkv(args, w, red_mode):
     peak, peak_kind = measured_peaks()
     achieved = alg_bytes / (kern_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": profiled_traffic(units),
-                "kernel": "rkv_step_kernel", "kernel_us_per_launch": kern_ms * 1e3,
+                "frac": achieved / peak, "traffic": profiled_traffic(kernel_name, w.name, units),
+                "kernel": kernel_name, "kernel_us_per_launch": kern_ms * 1e3,
                 "algorithmic_bytes_per_launch": alg_bytes, "peak_source": peak_kind,
                 "kernel_source_sha256_16": kernel_source_digest(),
                 "cluster_size": shape[0], "rows_per_cta": shape[1], "smem_per_cta": shape[2]}
@@ -415,7 +425,7 @@ def run_loop(args, w, red_mode):
     def compress(Q):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        rkv.rkv_compress_step(cfg, K, V, Q, cur, ws, stream=stream)
+        rkv.rkv_compress_step(cfg, K, V, Q, cur, ws, cluster_size=args.cluster_size, stream=stream)
         b.record(stream)
         evs.append((a, b))
 
@@ -446,7 +456,8 @@ def run_loop(args, w, red_mode):
     with torch.cuda.stream(side):
         with torch.cuda.graph(graph, stream=side):
             rkv.rkv_append_kv(cfg, K, V, kb, vb, cur, ws, stream=side)
-            rkv.rkv_compress_step(cfg, K, V, Qb, cur, ws, stream=side)
+            rkv.rkv_compress_step(cfg, K, V, Qb, cur, ws, cluster_size=args.cluster_size,
+                                  stream=side)
     stream.wait_stream(side)
     reps = 20
     g_ms = []

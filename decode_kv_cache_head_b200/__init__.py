@@ -72,8 +72,8 @@ def _load() -> ctypes.CDLL:
         "rkv_version": (I32, []),
         "rkv_workspace_size": (SZ, [CFG, I32, I32, I32]),
         "rkv_workspace_status": (ctypes.c_int, [P, P]),
-        "rkv_query_step_shape": (ctypes.c_int, [CFG, I32, ctypes.POINTER(I32), ctypes.POINTER(I32),
-                                                ctypes.POINTER(SZ)]),
+        "rkv_query_step_shape": (ctypes.c_int, [CFG, I64, I32, ctypes.POINTER(I32),
+                                                ctypes.POINTER(I32), ctypes.POINTER(SZ)]),
         "rkv_score_importance": (ctypes.c_int, [CFG, P, P, I64, I32, P, P, P, SZ, P]),
         "rkv_score_redundancy": (ctypes.c_int, [CFG, P, I64, I32, P, P, P, SZ, P]),
         "rkv_select_topk": (ctypes.c_int, [CFG, P, P, I32, P, P, P, SZ, P]),
@@ -143,10 +143,11 @@ def rkv_workspace_size(cfg: rkv_config, n_layers: int, batch: int, cap: int) -> 
     return int(_lib.rkv_workspace_size(ctypes.byref(cfg), n_layers, batch, cap))
 
 
-def rkv_query_step_shape(cfg: rkv_config, cap: int):
-    """(cluster_size, rows_per_cta, smem_bytes) that rkv_compress_step uses for `cap` rows."""
+def rkv_query_step_shape(cfg: rkv_config, n_units: int, cap: int):
+    """(cluster_size, rows_per_cta, smem_bytes) that rkv_compress_step uses for n_units
+    units (layers x batch x KV heads) of `cap` rows; cluster_size 1 = one CTA per unit."""
     cs, rows, smem = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_size_t()
-    _check(_lib.rkv_query_step_shape(ctypes.byref(cfg), int(cap), ctypes.byref(cs),
+    _check(_lib.rkv_query_step_shape(ctypes.byref(cfg), int(n_units), int(cap), ctypes.byref(cs),
                                      ctypes.byref(rows), ctypes.byref(smem)),
            "rkv_query_step_shape")
     return cs.value, rows.value, smem.value

@@ -20,6 +20,8 @@ constexpr int32_t kVersion = 1 * 10000 + 0 * 100 + 0;
 constexpr int kSmemPerSM = 233472;            // 228 KB of shared memory per SM
 constexpr int kSmemPerCtaMax = 232448;        // 227 KB opt-in limit per CTA
 constexpr int kSmemTwoPerSM = kSmemPerSM / 2 - 1024;
+constexpr int kB200SMs = 148;                 // launches with at least this many units use
+                                              // the one-CTA-per-unit kernel
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
@@ -127,6 +129,33 @@ Shape choose_shape(int cap, int nqp, int cs_req) {
     }
     Shape none = {};
     return none;
+}
+
+// The one-CTA-per-unit kernel: dynamic shared memory and TMEM columns for
+// caches of `cap` rows; ok = false when the unit does not fit one CTA.
+struct UnitShape {
+    bool ok;
+    int tmem_cols;
+    size_t smem;
+};
+
+UnitShape unit_shape(int cap, int nqp) {
+    UnitShape u = {};
+    if (cap > kUnitMaxRows) return u;
+    u.tmem_cols = pow2_at_least(2 * (nqp + 16));
+    u.smem = make_unit_layout(cap, nqp).total;
+    const int max_res = 512 / u.tmem_cols;   // CTAs whose TMEM fits one SM
+    const size_t floor_smem = static_cast<size_t>(kSmemPerSM / (max_res + 1) - 1024 + 16);
+    if (u.smem < floor_smem) u.smem = floor_smem;
+    u.ok = u.smem <= static_cast<size_t>(kSmemPerCtaMax);
+    return u;
+}
+
+// cs_req: 0 = automatic, 1 = one CTA per unit, else the cluster size.
+bool use_unit_kernel(int64_t n_units, int cap, int nqp, int cs_req) {
+    if (cs_req == 1) return true;
+    if (cs_req > 1) return false;
+    return n_units >= kB200SMs && unit_shape(cap, nqp).ok;
 }
 
 size_t ws_bytes_for(const rkv_config *cfg, int32_t n_layers, int32_t batch, int32_t cap) {
@@ -243,12 +272,19 @@ size_t rkv_workspace_size(const rkv_config *cfg, int32_t n_layers, int32_t batch
     return ws_bytes_for(cfg, n_layers, batch, cap);
 }
 
-rkv_status rkv_query_step_shape(const rkv_config *cfg, int32_t cap, int32_t *cluster_size,
-                                int32_t *rows_per_cta, size_t *smem_bytes) {
+rkv_status rkv_query_step_shape(const rkv_config *cfg, int64_t n_units, int32_t cap,
+                                int32_t *cluster_size, int32_t *rows_per_cta, size_t *smem_bytes) {
     const rkv_status st = check_cfg(cfg);
     if (st != RKV_OK) return st;
-    if (cap < 2) return RKV_ERR_INVALID;
+    if (cap < 2 || n_units < 1) return RKV_ERR_INVALID;
     const int nqp = nqp_of((cfg->n_q_heads / cfg->n_kv_heads) * cfg->window);
+    if (use_unit_kernel(n_units, cap, nqp, 0)) {
+        const UnitShape u = unit_shape(cap, nqp);
+        if (cluster_size) *cluster_size = 1;
+        if (rows_per_cta) *rows_per_cta = cap;
+        if (smem_bytes) *smem_bytes = u.smem;
+        return RKV_OK;
+    }
     const Shape s = choose_shape(cap, nqp, 0);
     if (s.cs == 0) return RKV_ERR_UNSUPPORTED;
     if (cluster_size) *cluster_size = s.cs;
@@ -396,11 +432,15 @@ rkv_status rkv_compress_step(const rkv_config *cfg, int32_t n_layers, int32_t ba
     if (!aligned16(workspace) || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return RKV_ERR_ALIGN;
     if (ws_bytes < ws_bytes_for(cfg, n_layers, batch, cap)) return RKV_ERR_WORKSPACE;
     const int nqp = nqp_of((cfg->n_q_heads / cfg->n_kv_heads) * cfg->window);
-    const Shape s = choose_shape(cap, nqp, opts ? opts->cluster_size : 0);
-    if (s.cs == 0) return RKV_ERR_UNSUPPORTED;
-    if (opts && opts->cluster_size && opts->cluster_size != 2 && opts->cluster_size != 4 &&
-        opts->cluster_size != 8 && opts->cluster_size != 16)
+    const int cs_req = opts ? opts->cluster_size : 0;
+    if (cs_req != 0 && cs_req != 1 && cs_req != 2 && cs_req != 4 && cs_req != 8 && cs_req != 16)
         return RKV_ERR_INVALID;
+    const bool unit_path =
+        use_unit_kernel(static_cast<int64_t>(n_layers) * batch * cfg->n_kv_heads, cap, nqp, cs_req);
+    const UnitShape us = unit_path ? unit_shape(cap, nqp) : UnitShape{};
+    if (unit_path && !us.ok) return RKV_ERR_UNSUPPORTED;
+    const Shape s = unit_path ? Shape{} : choose_shape(cap, nqp, cs_req);
+    if (!unit_path && s.cs == 0) return RKV_ERR_UNSUPPORTED;
 
     cudaStream_t strm = reinterpret_cast<cudaStream_t>(stream);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -450,7 +490,49 @@ rkv_status rkv_compress_step(const rkv_config *cfg, int32_t n_layers, int32_t ba
     }
     if (e == cudaSuccess && opts && opts->main_begin)
         e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->main_begin), strm);
-    for (int l0 = 0; e == cudaSuccess && l0 < n_layers; l0 += kMaxLayersPerLaunch) {
+    if (unit_path) {
+        UnitParams *up = new UnitParams();
+        std::memset(up, 0, sizeof(*up));
+        up->batch = batch;
+        up->n_kv = cfg->n_kv_heads;
+        up->group = cfg->n_q_heads / cfg->n_kv_heads;
+        up->window = cfg->window;
+        up->cap = cap;
+        up->nmax = cap;
+        up->tmem_cols = us.tmem_cols;
+        up->budget_cfg = cfg->budget;
+        up->lambda_cfg = cfg->mix_lambda;
+        up->logit_scale_log2 = p.logit_scale_log2;
+        up->red_mode = cfg->redundancy_mode;
+        up->gqa_pool = cfg->gqa_pool;
+        up->budgets = budgets;
+        up->lambdas = lambdas;
+        up->n_eff = n_eff;
+        up->r_ext = p.r_ext;
+        up->kept_out = p.kept_out;
+        up->scores_out = p.scores_out;
+        up->status = status;
+        for (int l0 = 0; e == cudaSuccess && l0 < n_layers; l0 += kMaxLayersPerLaunch) {
+            const int nl = (n_layers - l0 < kMaxLayersPerLaunch) ? n_layers - l0 : kMaxLayersPerLaunch;
+            up->layer_base = l0;
+            for (int i = 0; i < nl; ++i) {
+                const int l = l0 + i;
+                if (!encode_rows128(&up->tmap_k[i], k_layers[l],
+                                    static_cast<uint64_t>(batch) * cfg->n_kv_heads * cap, 128) ||
+                    !encode_rows128(&up->tmap_q[i], q_layers[l],
+                                    static_cast<uint64_t>(batch) * cfg->n_q_heads * cfg->window,
+                                    static_cast<uint32_t>(nqp))) {
+                    e = cudaErrorInvalidValue;
+                    break;
+                }
+                up->k[i] = k_layers[l];
+                up->v[i] = v_layers[l];
+            }
+            if (e == cudaSuccess) e = launch_unit(*up, nl * batch * cfg->n_kv_heads, nqp, us.smem, strm);
+        }
+        delete up;
+    }
+    for (int l0 = 0; !unit_path && e == cudaSuccess && l0 < n_layers; l0 += kMaxLayersPerLaunch) {
         const int nl = (n_layers - l0 < kMaxLayersPerLaunch) ? n_layers - l0 : kMaxLayersPerLaunch;
         p.n_layers = nl;
         p.layer_base = l0;

@@ -138,6 +138,63 @@ cudaError_t launch_compact(const uint16_t *k_src, const uint16_t *v_src, const i
                            cudaStream_t stream);
 int compact_in_place_cluster(int budget);   // 0: too large for the staged in-place path
 
+// One-CTA-per-unit kernel (rkv_unit.cu): the whole (sequence, layer, KV head)
+// in one CTA, K streamed through a two-stage TMA ring twice (HBM, then L2).
+struct alignas(64) UnitParams {
+    CUtensorMap tmap_k[kMaxLayersPerLaunch];   // [B*Hkv*cap rows, 128] bf16, box 64 x 128, SW128
+    CUtensorMap tmap_q[kMaxLayersPerLaunch];   // [B*Hq*w rows, 128] bf16, box 64 x NQP, SW128
+    uint16_t *k[kMaxLayersPerLaunch];
+    uint16_t *v[kMaxLayersPerLaunch];
+    int32_t layer_base, batch, n_kv, group, window, cap;
+    int32_t nmax;          // rows the per-row arrays hold (= cap)
+    int32_t tmem_cols;
+    int32_t budget_cfg;
+    float lambda_cfg;
+    float logit_scale_log2;
+    int32_t red_mode, gqa_pool;
+    const int32_t *budgets;
+    const float *lambdas;
+    const int32_t *n_eff;
+    const float *r_ext;
+    int32_t *kept_out;
+    float *scores_out;
+    uint32_t *status;
+};
+
+constexpr int kUnitThreads = 256;
+constexpr int kUnitMaxRows = 7680;     // keys + destinations + histograms fit the 64 KB ring
+
+struct UnitLayout {
+    uint32_t stage, b, inv, self, ia, ib, r, scr, s, colm, colf, vis, red, bars, total;
+};
+
+// Offsets from a 1024-byte-aligned base.  The two 32 KB ring stages are reused
+// after the last tile for the select keys, the destinations and the histograms.
+__host__ __device__ inline UnitLayout make_unit_layout(int nmax, int nqp) {
+    UnitLayout L;
+    uint32_t o = 0;
+    L.stage = o;  o += 2u * 32768u;
+    L.b = o;      o += 2u * (nqp + 16u) * 128u;        // queries + split S, two swizzled halves
+    const uint32_t arr = align_up(static_cast<uint32_t>(nmax) * 4u, 16);
+    L.inv = o;    o += arr;
+    L.self = o;   o += arr;
+    L.ia = o;     o += arr;
+    L.ib = o;     o += arr;
+    L.r = o;      o += arr;
+    L.scr = o;    o += 8192u;
+    L.s = o;      o += 512u;
+    L.colm = o;   o += 256u;
+    L.colf = o;   o += 256u;
+    L.vis = o;    o += 512u;
+    L.red = o;    o += 256u;
+    L.bars = o;   o += 64u;
+    L.total = o + 1024u;
+    return L;
+}
+
+cudaError_t launch_unit(const UnitParams &p, int n_units, int nqp, size_t smem,
+                        cudaStream_t stream);
+
 // MAX-mode similarity kernel: raw r of every candidate of every due unit.
 struct alignas(64) GramParams {
     CUtensorMap tmap[kMaxLayersPerLaunch];   // [B*Hkv*cap rows, 128] bf16, box 64 x 128, SW128

@@ -48,6 +48,7 @@
 
 #include "rkv_block.cuh"
 #include "rkv_internal.h"
+#include "rkv_post.cuh"
 #include "rkv_ptx.cuh"
 
 namespace cg = cooperative_groups;
@@ -88,76 +89,6 @@ cudaError_t launch_plan(int batch, const int32_t *budgets, int32_t budget_cfg, i
 // ----------------------------------------------------------------------------
 // The fused per-unit kernel.
 // ----------------------------------------------------------------------------
-// After barrier 2: (sum Ihat, max r) and sum exp(r - max r) over all M
-// candidates from the local copies in xIR (thread tid holds candidates
-// tid + k * NT in registers), then, if `select`, each candidate's key
-// (also stored at sKeys[2j], in place over xIR) and the radix select.
-template <int NT, int KPT>
-__device__ __forceinline__ void post_exchange(const float2 *xIR, uint32_t *sKeys, uint32_t *sHist,
-                                              float *sRed, int M, int kk, float lam, bool select,
-                                              float &inv_sumI, float &rmax_g, float &inv_rsum,
-                                              uint32_t &T, int &n_gt) {
-    constexpr int NW = NT / 32;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    float ih[KPT], rr[KPT];
-    bool kv[KPT];
-    float sI = 0.f, mx = -INFINITY;
-#pragma unroll
-    for (int k = 0; k < KPT; ++k) {
-        const int j = tid + k * NT;
-        kv[k] = j < M;
-        const float2 v = kv[k] ? xIR[j] : make_float2(0.f, -INFINITY);
-        ih[k] = v.x;
-        rr[k] = v.y;
-        sI += v.x;
-        mx = fmaxf(mx, v.y);
-    }
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-        sI += __shfl_xor_sync(kFull, sI, off);
-        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, off));
-    }
-    if (lane == 0) {
-        sRed[2 * warp] = sI;
-        sRed[2 * warp + 1] = mx;
-    }
-    for (int i = tid; i < 256; i += NT) sHist[i] = 0;   // first histogram of the select
-    __syncthreads();
-    sI = sRed[0];
-    mx = sRed[1];
-#pragma unroll
-    for (int w = 1; w < NW; ++w) {
-        sI += sRed[2 * w];
-        mx = fmaxf(mx, sRed[2 * w + 1]);
-    }
-    float e[KPT];
-    float rs = 0.f;
-#pragma unroll
-    for (int k = 0; k < KPT; ++k) {
-        e[k] = kv[k] ? ex2_approx((rr[k] - mx) * kLog2e) : 0.f;
-        rs += e[k];
-    }
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) rs += __shfl_xor_sync(kFull, rs, off);
-    if (lane == 0) sRed[2 * NW + warp] = rs;
-    __syncthreads();
-    rs = sRed[2 * NW];
-#pragma unroll
-    for (int w = 1; w < NW; ++w) rs += sRed[2 * NW + w];
-    inv_sumI = 1.0f / sI;
-    rmax_g = mx;
-    inv_rsum = 1.0f / rs;
-    if (!select) return;
-    uint32_t kr[KPT];
-#pragma unroll
-    for (int k = 0; k < KPT; ++k) {
-        kr[k] = ordered_key(joint_score(lam, ih[k] * inv_sumI, e[k] * inv_rsum));
-        if (kv[k]) sKeys[2 * (tid + k * NT)] = kr[k];
-    }
-    if (kk > 0) block_select_kth_fast<NT, KPT>(kr, kv, kk, sHist, T, n_gt);
-    else __syncthreads();
-}
-
 // NQP: query columns G*w rounded up to 16.  WC: the window size when it is
 // known at compile time (the common w = 8), 0 for a runtime window.
 template <int NQP, int WC>
@@ -594,16 +525,8 @@ __global__ void __launch_bounds__(kStepThreads, 2) rkv_step_kernel(const __grid_
     int n_gt = 0;
     {
         const bool sel = do_sel && nrows > 0;
-        if (M <= 5 * NT)
-            post_exchange<NT, 5>(xIR, sKeys, sHist, sRed, M, kk, lam, sel, inv_sumI, rmax_g, inv_rsum, T, n_gt);
-        else if (M <= 7 * NT)
-            post_exchange<NT, 7>(xIR, sKeys, sHist, sRed, M, kk, lam, sel, inv_sumI, rmax_g, inv_rsum, T, n_gt);
-        else if (M <= 9 * NT)
-            post_exchange<NT, 9>(xIR, sKeys, sHist, sRed, M, kk, lam, sel, inv_sumI, rmax_g, inv_rsum, T, n_gt);
-        else if (M <= 16 * NT)
-            post_exchange<NT, 16>(xIR, sKeys, sHist, sRed, M, kk, lam, sel, inv_sumI, rmax_g, inv_rsum, T, n_gt);
-        else
-            post_exchange<NT, 32>(xIR, sKeys, sHist, sRed, M, kk, lam, sel, inv_sumI, rmax_g, inv_rsum, T, n_gt);
+        post_scores_any<NT, 2>([&](int j) { return xIR[j]; }, sKeys, sHist, sRed, M, kk, lam, sel,
+                               inv_sumI, rmax_g, inv_rsum, T, n_gt);
     }
 
     if (p.flags & kFlagOutScores) {

@@ -1,0 +1,630 @@
+// rkv_unit.cu -- the R-KV compression step with one CTA per unit (sequence,
+// layer, KV head), for launches with at least as many units as the GPU has
+// SMs: no cluster, no exchange, one select per unit.
+//
+// Method: "R-KV: Redundancy-aware KV Cache Compression for Reasoning Models"
+// (atlas.scime.ai summary, "Approach": Z = lambda I - (1 - lambda) R, applied
+// periodically during decoding; "Measured effects": max pooling over the GQA
+// group), the hysenlabs write-up (decode-time scoring: budget, window_size,
+// mix_lambda; the protected recent window) and the sourcepulse summary ("How
+// It Works": attention-weight importance, cosine-similarity redundancy, top-k
+// within the budget).
+//
+// A unit's K (N rows x 256 bytes) is larger than shared memory, so it is
+// streamed twice through a two-stage ring of 128-row tiles loaded by TMA:
+//   pass 1 (from HBM): one thread issues tcgen05 UMMAs, logits[128 rows, G*w]
+//     = K_tile . Q^T into TMEM; meanwhile the CTA computes ||k_i||^2 and
+//     1/max(||k_i||, 1e-12) and its running part of S = sum_i khat_i; then
+//     every thread folds its row's logits into per-column running (max, sum
+//     of exp) pairs (online softmax, rescaling only when a logit exceeds the
+//     running reference by more than 2^8).
+//   between the passes: the column pairs are merged over the CTA; S is split
+//     into three bf16 terms (hi + mid + lo carries its fp32 value) and written
+//     as three extra rows of the UMMA B operand.
+//   pass 2 (the same tiles, now from L2): the UMMA gives the logits again and,
+//     in three more columns, k_i . S; per row p = exp(s - max) / sum, the mean
+//     over the window queries and the max over the group (Ihat_i), and
+//     r_i = (khat_i . S - khat_i . khat_i) / (N - 1) (MEAN) or r_i from the
+//     similarity kernel (MAX).
+//   then the normalisers, the joint scores, the radix select and the
+//   destinations of the kept rows, and the in-place compaction in ascending
+//   chunks of 128 rows (every source row of a chunk is read before any row of
+//   it is written; later chunks only read rows above the current chunk).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cfloat>
+#include <cstdint>
+
+#include "rkv_block.cuh"
+#include "rkv_internal.h"
+#include "rkv_post.cuh"
+#include "rkv_ptx.cuh"
+
+namespace rkv {
+
+namespace {
+
+constexpr int kTileRows = 128;
+constexpr uint32_t kStageBytes = 32768u;
+constexpr uint32_t kHalfBytes = 16384u;
+constexpr int kChunkRows = 128;          // compaction chunk
+constexpr float kRescaleLog2 = 8.0f;     // online softmax: rescale past 2^8
+
+// Merges (m2, s2) into (m, s): s = sum of 2^(x - m) over the values seen.
+__device__ __forceinline__ void ms_merge(float &m, float &s, float m2, float s2) {
+    const float mn = fmaxf(m, m2);
+    const float a = (m == -INFINITY) ? 0.f : s * ex2_approx(m - mn);
+    const float b = (m2 == -INFINITY) ? 0.f : s2 * ex2_approx(m2 - mn);
+    m = mn;
+    s = a + b;
+}
+
+// Folds 8 per-lane columns of (m, s) pairs across the warp: afterwards lane L
+// holds the merge over all 32 lanes of column (L & 7) in m[0], s[0].
+__device__ __forceinline__ void warp_fold8_ms(float (&m)[8], float (&s)[8]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int off = 4; off >= 1; off >>= 1) {
+        const bool up = (lane & off) != 0;
+#pragma unroll
+        for (int i = 0; i < off; ++i) {
+            const float send_m = up ? m[i] : m[i + off];
+            const float send_s = up ? s[i] : s[i + off];
+            float km = up ? m[i + off] : m[i];
+            float ks = up ? s[i + off] : s[i];
+            const float rm = __shfl_xor_sync(kFull, send_m, off);
+            const float rs = __shfl_xor_sync(kFull, send_s, off);
+            ms_merge(km, ks, rm, rs);
+            m[i] = km;
+            s[i] = ks;
+        }
+    }
+#pragma unroll
+    for (int off = 8; off <= 16; off <<= 1) {
+        const float rm = __shfl_xor_sync(kFull, m[0], off);
+        const float rs = __shfl_xor_sync(kFull, s[0], off);
+        ms_merge(m[0], s[0], rm, rs);
+    }
+}
+
+__device__ __forceinline__ uint16_t bf16_rn_bits(float x) {
+    return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
+    return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+}  // namespace
+
+// NQP: query columns G*w rounded up to 16.  WC: the window when it is 8 (the
+// pages' value), 0 for a runtime window.
+template <int NQP, int WC>
+__global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_constant__ UnitParams p) {
+    constexpr int NT = kUnitThreads;
+    constexpr int NW = NT / 32;
+    constexpr int SLOT = NQP + 16;          // TMEM columns per tile slot
+    constexpr int HC = NQP / 2;             // pass-1 columns per warpgroup
+    constexpr uint32_t kBRows = NQP + 16;   // B operand rows: queries, then the split S
+    constexpr int MAXH = NQP / 16;          // heads per warpgroup in pass 2 (WC == 8)
+    static_assert(WC == 0 || WC == 8, "window template");
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+
+    const int unit = blockIdx.x;
+    const int h = unit % p.n_kv;
+    const int b = (unit / p.n_kv) % p.batch;
+    const int l = unit / (p.n_kv * p.batch);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wg = warp >> 2;
+
+    const int N = p.n_eff[b];
+    if (N <= 0) return;   // not due
+
+    const int w = WC > 0 ? WC : p.window;
+    const int G = p.group;
+    const int NQ = G * w;
+    const int M = N - w;
+    const int budget = p.budgets ? p.budgets[b] : p.budget_cfg;
+    const float lam = p.lambdas ? p.lambdas[b] : p.lambda_cfg;
+    const int kk = budget - w;
+    const bool red_max = p.red_mode == RKV_RED_MAX;
+    const bool pool_max = p.gqa_pool == RKV_GQA_MAX;
+    const int T = (N + kTileRows - 1) / kTileRows;
+    const int64_t krow0 = (static_cast<int64_t>(b) * p.n_kv + h) * p.cap;
+    const int64_t unit_g = (static_cast<int64_t>(p.layer_base + l) * p.batch + b) * p.n_kv + h;
+
+    const UnitLayout L = make_unit_layout(p.nmax, NQP);
+    uint8_t *sStage = base + L.stage;
+    uint8_t *sB = base + L.b;
+    float *sInv = reinterpret_cast<float *>(base + L.inv);
+    float *sSelf = reinterpret_cast<float *>(base + L.self);
+    float *sIa = reinterpret_cast<float *>(base + L.ia);
+    float *sIb = reinterpret_cast<float *>(base + L.ib);
+    float *sR = reinterpret_cast<float *>(base + L.r);
+    float *sScr = reinterpret_cast<float *>(base + L.scr);
+    float *sColM = reinterpret_cast<float *>(base + L.colm);
+    float *sColF = reinterpret_cast<float *>(base + L.colf);
+    uint64_t *sVis = reinterpret_cast<uint64_t *>(base + L.vis);
+    float *sRed = reinterpret_cast<float *>(base + L.red);
+    uint32_t *sRedU = reinterpret_cast<uint32_t *>(base + L.red);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(base + L.bars);   // full[2], mma[2]
+    uint32_t *sTmem = reinterpret_cast<uint32_t *>(bars + 4);
+    // after the last tile the ring holds the keys, the destinations and the histograms
+    const uint32_t arr = align_up(static_cast<uint32_t>(p.nmax) * 4u, 16);
+    uint32_t *sKeys = reinterpret_cast<uint32_t *>(sStage);
+    int32_t *sDst = reinterpret_cast<int32_t *>(sStage + arr);
+    uint32_t *sHist = reinterpret_cast<uint32_t *>(sStage + 2u * arr);
+
+    const uint64_t colmask = NQ >= 64 ? ~0ull : ((1ull << NQ) - 1ull);
+    const uint64_t lastmask = [&] {
+        uint64_t m = 0;
+        for (int g = 0; g < G; ++g) m |= 1ull << (g * w + w - 1);
+        return m;
+    }();
+
+    // ---- set-up
+    if (warp == 0) {
+        tmem_alloc(sTmem, static_cast<uint32_t>(p.tmem_cols));
+        tmem_relinquish();
+    }
+    if (tid == 32) {
+        for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+        fence_mbar_init();
+    }
+    // B operand rows past the queries start as zeros (the split S lands in three of them)
+    for (int i = tid; i < 2 * 16 * 8; i += NT) {
+        const int half = i >> 7, row = NQP + ((i & 127) >> 3), ch = i & 7;
+        *reinterpret_cast<uint4 *>(sB + half * kBRows * 128u + row * 128u + ch * 16u) =
+            make_uint4(0u, 0u, 0u, 0u);
+    }
+    // window key M + d is seen by query column g*w + j only when j >= d (causal)
+    if (warp == 0) {
+        const int j0 = lane % w, j1 = (lane + 32) % w;
+        for (int d = 0; d < w; ++d) {
+            const uint64_t m =
+                static_cast<uint64_t>(__ballot_sync(kFull, lane < NQ && j0 >= d)) |
+                (static_cast<uint64_t>(__ballot_sync(kFull, lane + 32 < NQ && j1 >= d)) << 32);
+            if (lane == 0) sVis[d] = m;
+        }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *sTmem;
+
+    const CUtensorMap *mk = &p.tmap_k[l];
+    auto issue_tile = [&](int g) {   // global tile g: pass 1 for g < T, pass 2 after
+        const int tt = g < T ? g : g - T;
+        uint8_t *stg = sStage + (g & 1) * kStageBytes;
+        const int32_t y = static_cast<int32_t>(krow0 + tt * kTileRows);
+        tma_load_2d(stg, mk, &bars[g & 1], 0, y);
+        tma_load_2d(stg + kHalfBytes, mk, &bars[g & 1], 64, y);
+    };
+    if (tid == 32) {
+        const CUtensorMap *mq = &p.tmap_q[l];
+        const int32_t yq = (b * p.n_kv + h) * NQ;   // the KV head's query rows
+        mbar_arrive_expect_tx(&bars[0], kStageBytes + static_cast<uint32_t>(NQP) * 256u);
+        tma_load_2d(sB, mq, &bars[0], 0, yq);
+        tma_load_2d(sB + kBRows * 128u, mq, &bars[0], 64, yq);
+        issue_tile(0);
+        mbar_arrive_expect_tx(&bars[1], kStageBytes);
+        issue_tile(1);
+    }
+
+    // ---- the two passes
+    const float sc = p.logit_scale_log2;
+    const float inv_nm1 = 1.0f / static_cast<float>(N - 1);
+    const float inv_w = 1.0f / static_cast<float>(w);
+    const uint32_t tmem_lane = tmem_base + ((32u * static_cast<uint32_t>(warp & 3)) << 16);
+    const int lrow = (warp & 3) * 32 + lane;   // TMEM lane = tile row
+    // norms: lanes 0-7 / 16-23 take the first 64 columns of rows (l & 7) + 8 (l >> 4)
+    const int nrow = (lane & 7) + 8 * (lane >> 4), nhalf = (lane >> 3) & 1;
+    // S partial: lane owns columns shalf * 64 + (lane & 15) * 4 .. + 3
+    const int shalf = lane >> 4, schunk = (lane & 15) >> 1, ssub = lane & 1;
+
+    float cm[HC], cs[HC];
+#pragma unroll
+    for (int c = 0; c < HC; ++c) {
+        cm[c] = -INFINITY;
+        cs[c] = 0.f;
+    }
+    float2 sacc0 = make_float2(0.f, 0.f), sacc1 = make_float2(0.f, 0.f);
+    bool ok = true;
+    int g = 0;
+    for (; g < 2 * T; ++g) {
+        const bool pass2 = g >= T;
+        const int tt = pass2 ? g - T : g;
+        const int s = g & 1;
+        const uint32_t par = static_cast<uint32_t>((g >> 1) & 1);
+        const uint8_t *stg = sStage + s * kStageBytes;
+        const uint32_t tslot = static_cast<uint32_t>(s * SLOT);
+
+        if (g == T) {
+            // ---- between the passes: column (max, sum) over the CTA; S split into B
+            float *xm = sScr + 1024;   // [8 warps][HC] (m, s) pairs
+#pragma unroll
+            for (int c0 = 0; c0 < HC; c0 += 8) {
+                float m8[8], s8[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    m8[j] = cm[c0 + j];
+                    s8[j] = cs[c0 + j];
+                }
+                warp_fold8_ms(m8, s8);
+                if (lane < 8) {
+                    xm[(warp * HC + c0 + lane) * 2] = m8[0];
+                    xm[(warp * HC + c0 + lane) * 2 + 1] = s8[0];
+                }
+            }
+            if (!red_max) {
+                const int col = shalf * 64 + (lane & 15) * 4;
+                *reinterpret_cast<float4 *>(sScr + warp * 128 + col) =
+                    make_float4(sacc0.x, sacc0.y, sacc1.x, sacc1.y);
+            }
+            __syncthreads();
+            if (tid < NQP) {
+                const int q = tid, gq = q / HC, c = q % HC;
+                float m = xm[((gq * 4) * HC + c) * 2], sm = xm[((gq * 4) * HC + c) * 2 + 1];
+#pragma unroll
+                for (int k = 1; k < 4; ++k)
+                    ms_merge(m, sm, xm[((gq * 4 + k) * HC + c) * 2], xm[((gq * 4 + k) * HC + c) * 2 + 1]);
+                sColM[q] = m;
+                sColF[q] = sm > 0.f ? 1.0f / sm : 0.f;
+            }
+            if (!red_max && tid >= 128) {
+                const int d = tid - 128;
+                float S = sScr[d];
+#pragma unroll
+                for (int k = 1; k < NW; ++k) S += sScr[k * 128 + d];
+                const uint16_t hi = bf16_rn_bits(S);
+                const float r1 = S - bf16_bits_to_float(hi);
+                const uint16_t mid = bf16_rn_bits(r1);
+                const uint16_t lo = bf16_rn_bits(r1 - bf16_bits_to_float(mid));
+                uint8_t *hb = sB + (d >> 6) * kBRows * 128u;
+                const uint32_t c = (d & 63) >> 3, e = (d & 7) * 2u;
+                *reinterpret_cast<uint16_t *>(hb + sw128_offset(NQP + 0, c) + e) = hi;
+                *reinterpret_cast<uint16_t *>(hb + sw128_offset(NQP + 1, c) + e) = mid;
+                *reinterpret_cast<uint16_t *>(hb + sw128_offset(NQP + 2, c) + e) = lo;
+            }
+            fence_proxy_async_smem();
+            __syncthreads();
+        }
+
+        bool wait_ok = mbar_wait(&bars[s], par);
+        if (tid == 0 && wait_ok) {
+            tc_fence_after();
+            const uint32_t idesc = (pass2 && !red_max) ? idesc_bf16_f32(128, NQP + 16)
+                                                       : idesc_bf16_f32(128, NQP);
+            const uint32_t a_base = smem_u32(stg), b_base = smem_u32(sB);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t half = ks >> 2, koff = (ks & 3) * 32u;
+                const uint64_t ad = desc_kmajor_sw128(a_base + half * kHalfBytes + koff);
+                const uint64_t bd = desc_kmajor_sw128(b_base + half * kBRows * 128u + koff);
+                umma_bf16(tmem_base + tslot, ad, bd, idesc, ks > 0 ? 1u : 0u);
+            }
+            umma_commit(&bars[2 + s]);
+        }
+
+        if (!pass2 && !red_max && wait_ok) {
+            // ||k_i||^2 and 1 / max(||k_i||, 1e-12): two lanes per row, 64 columns each
+            const int row_t = 16 * warp + nrow;
+            const int i = tt * kTileRows + row_t;
+            const uint8_t *hp = stg + nhalf * kHalfBytes;
+            float2 ss2 = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const uint4 raw = *reinterpret_cast<const uint4 *>(hp + sw128_offset(row_t, c));
+                const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(h2[e]);
+                    ss2 = __ffma2_rn(f, f, ss2);
+                }
+            }
+            float ssh = ss2.x + ss2.y;
+            const float ss = ssh + __shfl_xor_sync(kFull, ssh, 8);
+            const float inv = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
+            if (nhalf == 0 && i < N) {
+                sInv[i] = inv;
+                sSelf[i] = inv * inv * ss;
+            }
+            // this warp's 16 rows into the S partial (each lane 4 columns)
+            const uint8_t *sp = stg + shalf * kHalfBytes;
+#pragma unroll 4
+            for (int r = 0; r < 16; ++r) {
+                const float iv = __shfl_sync(kFull, inv, (r & 7) + 16 * (r >> 3));
+                if (tt * kTileRows + 16 * warp + r < N) {
+                    const uint2 raw = *reinterpret_cast<const uint2 *>(
+                        sp + sw128_offset(16 * warp + r, schunk) + ssub * 8);
+                    const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+                    const float2 iv2 = make_float2(iv, iv);
+                    sacc0 = __ffma2_rn(__bfloat1622float2(h2[0]), iv2, sacc0);
+                    sacc1 = __ffma2_rn(__bfloat1622float2(h2[1]), iv2, sacc1);
+                }
+            }
+        }
+
+        wait_ok = wait_ok && mbar_wait(&bars[2 + s], par);
+        tc_fence_after();
+        const int i = tt * kTileRows + lrow;
+        if (wait_ok && !pass2) {
+            // ---- pass 1: fold this row's logits into the running column pairs
+            const uint64_t rmask = i < M ? colmask : (i < N ? sVis[i - M] : 0ull);
+            const bool all_cand = __all_sync(kFull, i < M);
+            uint32_t raw[HC / 8][8];
+#pragma unroll
+            for (int c0 = 0; c0 < HC; c0 += 8)
+                tmem_ld8_nowait(tmem_lane + tslot + static_cast<uint32_t>(wg * HC + c0), raw[c0 / 8]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c0 = 0; c0 < HC; c0 += 8) reg_tie8(raw[c0 / 8]);
+#pragma unroll
+            for (int c0 = 0; c0 < HC; c0 += 8) {
+                const int q0 = wg * HC + c0;
+                float x[8];
+                bool vis[8];
+                bool big = false;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    x[j] = __uint_as_float(raw[c0 / 8][j]) * sc;
+                    vis[j] = (all_cand && q0 + 8 <= NQ) ? true : (((rmask >> (q0 + j)) & 1ull) != 0);
+                    big |= vis[j] && (x[j] > cm[c0 + j] + kRescaleLog2);
+                }
+                if (__any_sync(kFull, big)) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        if (vis[j]) {
+                            const float mn = fmaxf(cm[c0 + j], x[j]);
+                            cs[c0 + j] = cs[c0 + j] * ex2_approx(cm[c0 + j] - mn) + ex2_approx(x[j] - mn);
+                            cm[c0 + j] = mn;
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const float e = ex2_approx(x[j] - cm[c0 + j]);
+                        cs[c0 + j] += vis[j] ? e : 0.f;
+                    }
+                }
+            }
+        } else if (wait_ok) {
+            // ---- pass 2: Ihat partial (this warpgroup's heads) and r
+            const bool cand = i < M;
+            if (__any_sync(kFull, cand)) {
+                float pool = 0.f;   // Ihat >= 0: 0 is neutral for both pools
+                if (WC > 0) {
+                    const int Ga = (G + 1) >> 1;
+                    const int h0 = wg == 0 ? 0 : Ga, nh = wg == 0 ? Ga : G - Ga;
+                    uint32_t raw[MAXH][8];
+#pragma unroll
+                    for (int k = 0; k < MAXH; ++k)
+                        if (k < nh)
+                            tmem_ld8_nowait(tmem_lane + tslot + static_cast<uint32_t>((h0 + k) * 8), raw[k]);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int k = 0; k < MAXH; ++k)
+                        if (k < nh) reg_tie8(raw[k]);
+#pragma unroll
+                    for (int k = 0; k < MAXH; ++k) {
+                        if (k < nh) {
+                            const int q0 = (h0 + k) * 8;
+                            float run = 0.f;
+#pragma unroll
+                            for (int j = 0; j < 8; ++j)
+                                run = fmaf(ex2_approx(fmaf(__uint_as_float(raw[k][j]), sc, -sColM[q0 + j])),
+                                           sColF[q0 + j], run);
+                            const float a = run * inv_w;
+                            pool = pool_max ? fmaxf(pool, a) : pool + a;
+                        }
+                    }
+                } else if (wg == 0) {
+                    uint32_t raw[NQP / 8][8];
+#pragma unroll
+                    for (int c0 = 0; c0 < NQP; c0 += 8)
+                        tmem_ld8_nowait(tmem_lane + tslot + static_cast<uint32_t>(c0), raw[c0 / 8]);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c0 = 0; c0 < NQP; c0 += 8) reg_tie8(raw[c0 / 8]);
+                    float run = 0.f;
+#pragma unroll
+                    for (int q = 0; q < NQP; ++q) {
+                        if (q < NQ) {
+                            run = fmaf(ex2_approx(fmaf(__uint_as_float(raw[q / 8][q % 8]), sc, -sColM[q])),
+                                       sColF[q], run);
+                            if ((lastmask >> q) & 1ull) {
+                                const float a = run * inv_w;
+                                pool = pool_max ? fmaxf(pool, a) : pool + a;
+                                run = 0.f;
+                            }
+                        }
+                    }
+                }
+                float r = 0.f;
+                if (wg == 1) {
+                    if (red_max) {
+                        r = cand ? p.r_ext[unit_g * p.cap + i] : 0.f;
+                    } else {
+                        uint32_t d[4];
+                        tmem_ld4_nowait(tmem_lane + tslot + static_cast<uint32_t>(NQP), d);
+                        tmem_wait_ld();
+                        reg_tie4(d);
+                        const float dot = (__uint_as_float(d[0]) + __uint_as_float(d[1])) + __uint_as_float(d[2]);
+                        if (cand) r = (sInv[i] * dot - sSelf[i]) * inv_nm1;
+                    }
+                }
+                if (cand) {
+                    if (wg == 0) {
+                        sIa[i] = pool;
+                    } else {
+                        sIb[i] = pool;
+                        sR[i] = r;
+                    }
+                }
+            }
+        }
+        tc_fence_before();
+        if (__syncthreads_or(!wait_ok)) {
+            ok = false;
+            break;
+        }
+        if (tid == 32 && g + 2 < 2 * T) {
+            mbar_arrive_expect_tx(&bars[s], kStageBytes);
+            issue_tile(g + 2);
+        }
+    }
+
+    if (!ok) {
+        // A wait ran out: record it, wait (bounded) for this CTA's copies and
+        // UMMAs still in flight, free TMEM and leave without writing anything.
+        if (tid == 32) {
+            record_flag(p.status, kDevFlagTimeout);
+            for (int gg = g; gg < g + 2 && gg < 2 * T; ++gg)
+                (void)mbar_wait(&bars[gg & 1], static_cast<uint32_t>((gg >> 1) & 1));
+            (void)mbar_wait(&bars[2 + (g & 1)], static_cast<uint32_t>((g >> 1) & 1));
+        }
+        __syncthreads();
+        if (warp == 0) {
+            tc_fence_after();
+            tmem_dealloc(tmem_base, static_cast<uint32_t>(p.tmem_cols));
+        }
+        return;
+    }
+
+    // ---- normalisers, keys and the select (one per unit)
+    float inv_sumI, rmax_g, inv_rsum;
+    uint32_t Tk = 0xffffffffu;
+    int n_gt = 0;
+    const float invG = 1.0f / static_cast<float>(G);
+    post_scores_any<NT, 1>(
+        [&](int j) {
+            const float a = sIa[j], c = sIb[j];
+            return make_float2(pool_max ? fmaxf(a, c) : (a + c) * invG, sR[j]);
+        },
+        sKeys, sHist, sRed, M, kk, lam, true, inv_sumI, rmax_g, inv_rsum, Tk, n_gt);
+
+    // ---- destination of every row: G_i = rows above the threshold or in the
+    // window before i, E_i = tied candidates before i;
+    // kept = above || window || (tied && E_i < need_eq), dst = G_i + min(E_i, need_eq)
+    const int need_eq = (kk > 0) ? kk - n_gt : 0;
+    {
+        uint32_t g_run = 0, e_run = 0;
+        for (int c0 = 0; c0 < N; c0 += NT) {
+            const int row = c0 + tid;
+            const bool in = row < N;
+            const bool cand = row < M;
+            const uint32_t key = cand ? sKeys[row] : 0u;
+            const bool eq = cand && kk > 0 && key == Tk;
+            const bool gw = in && (!cand || (kk > 0 && key > Tk));
+            uint32_t tot2;
+            const uint32_t ex = block_excl_scan_u32<NT>((eq ? 65536u : 0u) + (gw ? 1u : 0u), sRedU, tot2);
+            const uint32_t Ei = e_run + (ex >> 16), Gi = g_run + (ex & 0xffffu);
+            const bool kept = gw || (eq && Ei < static_cast<uint32_t>(need_eq));
+            if (in) sDst[row] = kept ? static_cast<int32_t>(Gi + min(Ei, static_cast<uint32_t>(need_eq))) : -1;
+            e_run += tot2 >> 16;
+            g_run += tot2 & 0xffffu;
+        }
+    }
+    __syncthreads();
+
+    if (p.kept_out || p.scores_out) {
+        for (int row = tid; row < N; row += NT) {
+            const int d = sDst[row];
+            if (p.kept_out && d >= 0) p.kept_out[unit_g * p.cap + d] = row;
+            if (p.scores_out && row < M) {
+                float *so = p.scores_out + unit_g * 4 * p.cap;
+                const float a = sIa[row], c = sIb[row];
+                const float I = (pool_max ? fmaxf(a, c) : (a + c) * invG) * inv_sumI;
+                const float Rv = ex2_approx((sR[row] - rmax_g) * kLog2e) * inv_rsum;
+                so[row] = I;
+                so[p.cap + row] = sR[row];
+                so[2 * p.cap + row] = Rv;
+                so[3 * p.cap + row] = joint_score(lam, I, Rv);
+            }
+        }
+    }
+
+    // ---- compaction, in place, ascending chunks from the first row that moves
+    {
+        uint32_t first = static_cast<uint32_t>(N);
+        for (int row = tid; row < N; row += NT)
+            if (sDst[row] != row) {
+                first = static_cast<uint32_t>(row);
+                break;
+            }
+        first = __reduce_min_sync(kFull, first);
+        if (lane == 0) sRedU[warp] = first;
+        __syncthreads();
+        first = sRedU[0];
+#pragma unroll
+        for (int k = 1; k < NW; ++k) first = min(first, sRedU[k]);
+        uint16_t *kb = p.k[l] + krow0 * kHeadDim;
+        uint16_t *vb = p.v[l] + krow0 * kHeadDim;
+        constexpr int PER = kChunkRows * 16 / NT;   // 16-byte pieces per thread per chunk
+        for (int c0 = static_cast<int>(first); c0 < N; c0 += kChunkRows) {
+            uint4 kx[PER], vx[PER];
+            int dd[PER];
+#pragma unroll
+            for (int k = 0; k < PER; ++k) {
+                const int idx = tid + k * NT;
+                const int row = c0 + (idx >> 4), pc = idx & 15;
+                const int d = row < N ? sDst[row] : -1;
+                dd[k] = (d >= 0 && d != row) ? d : -1;
+                if (dd[k] >= 0) {
+                    kx[k] = __ldcg(reinterpret_cast<const uint4 *>(kb + static_cast<int64_t>(row) * kHeadDim) + pc);
+                    vx[k] = __ldcg(reinterpret_cast<const uint4 *>(vb + static_cast<int64_t>(row) * kHeadDim) + pc);
+                }
+            }
+            __syncthreads();
+#pragma unroll
+            for (int k = 0; k < PER; ++k) {
+                if (dd[k] >= 0) {
+                    const int pc = (tid + k * NT) & 15;
+                    reinterpret_cast<uint4 *>(kb + static_cast<int64_t>(dd[k]) * kHeadDim)[pc] = kx[k];
+                    reinterpret_cast<uint4 *>(vb + static_cast<int64_t>(dd[k]) * kHeadDim)[pc] = vx[k];
+                }
+            }
+        }
+    }
+
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, static_cast<uint32_t>(p.tmem_cols));
+    }
+}
+
+template <int NQP, int WC>
+static cudaError_t launch_unit_t(const UnitParams &p, int n_units, size_t smem, cudaStream_t stream) {
+    auto kern = rkv_unit_kernel<NQP, WC>;
+    static std::atomic<int> granted{0};
+    const cudaError_t e = ensure_smem_attr(kern, smem, granted);
+    if (e != cudaSuccess) return e;
+    kern<<<static_cast<unsigned>(n_units), kUnitThreads, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_unit(const UnitParams &p, int n_units, int nqp, size_t smem, cudaStream_t stream) {
+    if (p.window == 8) {
+        switch (nqp) {
+            case 16: return launch_unit_t<16, 8>(p, n_units, smem, stream);
+            case 32: return launch_unit_t<32, 8>(p, n_units, smem, stream);
+            case 48: return launch_unit_t<48, 8>(p, n_units, smem, stream);
+            case 64: return launch_unit_t<64, 8>(p, n_units, smem, stream);
+            default: return cudaErrorInvalidValue;
+        }
+    }
+    switch (nqp) {
+        case 16: return launch_unit_t<16, 0>(p, n_units, smem, stream);
+        case 32: return launch_unit_t<32, 0>(p, n_units, smem, stream);
+        case 48: return launch_unit_t<48, 0>(p, n_units, smem, stream);
+        case 64: return launch_unit_t<64, 0>(p, n_units, smem, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace rkv

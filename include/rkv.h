@@ -106,7 +106,9 @@ typedef struct {
                                 first N - window candidates of every compressed unit */
     rkv_event_t main_begin;  /* if not NULL: recorded on `stream` just before the main kernel */
     rkv_event_t main_end;    /* if not NULL: recorded on `stream` just after the main kernel */
-    int32_t cluster_size;    /* CTAs per unit: 0 = automatic, else 2, 4, 8 or 16 */
+    int32_t cluster_size;    /* CTAs per unit: 0 = automatic, 1 = one CTA per unit (K
+                                streamed twice through shared memory), else a cluster of
+                                2, 4, 8 or 16 CTAs that holds the unit's K on chip */
 } rkv_step_options;
 
 /* Human-readable name of a status code (static storage). */
@@ -132,12 +134,15 @@ RKV_API size_t rkv_workspace_size(const rkv_config *cfg, int32_t n_layers, int32
 RKV_API rkv_status rkv_workspace_status(const void *workspace, rkv_stream_t stream);
 
 /*
- * The launch shape rkv_compress_step picks for caches of `cap` rows: CTAs per
- * (sequence, layer, KV head) cluster, rows each CTA owns, and dynamic shared
- * memory per CTA.  Host-only (no CUDA call).  RKV_ERR_UNSUPPORTED when no
- * shape fits; any output pointer may be NULL.
+ * The launch shape rkv_compress_step picks (cluster_size = 0) for n_units
+ * (sequence, layer, KV head) units in one call (n_layers * batch * n_kv_heads)
+ * with caches of `cap` rows: CTAs per unit (1: one CTA per unit, the choice
+ * once the call has at least one unit per SM; else the cluster size), rows
+ * each CTA owns, and dynamic shared memory per CTA.  Host-only (no CUDA
+ * call).  RKV_ERR_UNSUPPORTED when no shape fits; any output pointer may be
+ * NULL.
  */
-RKV_API rkv_status rkv_query_step_shape(const rkv_config *cfg, int32_t cap,
+RKV_API rkv_status rkv_query_step_shape(const rkv_config *cfg, int64_t n_units, int32_t cap,
                                         int32_t *cluster_size, int32_t *rows_per_cta,
                                         size_t *smem_bytes);
 

@@ -54,6 +54,7 @@ def lib() -> ctypes.CDLL:
         _lib.rkv_oracle_softmax.argtypes = [P, i32, P]
         _lib.rkv_oracle_joint.argtypes = [P, P, i32, f64, P]
         _lib.rkv_oracle_select.argtypes = [P, i32, i32, i32, P]
+        _lib.rkv_oracle_shared_select.argtypes = [P, i32, i64, i32, i32, i32, P, P]
         _lib.rkv_oracle_compact.argtypes = [P, P, i32, i32, P]
         _lib.rkv_oracle_unit.argtypes = [P, P, i32, i32, i32, i32, i32, f64, i32, i32,
                                          P, P, P, P, P]
@@ -61,7 +62,8 @@ def lib() -> ctypes.CDLL:
                                           P, P, P, P, i64, P, i64, i32]
         for f in ("rkv_oracle_importance", "rkv_oracle_inv_norm", "rkv_oracle_redundancy",
                   "rkv_oracle_softmax", "rkv_oracle_joint", "rkv_oracle_select",
-                  "rkv_oracle_compact", "rkv_oracle_unit", "rkv_oracle_units"):
+                  "rkv_oracle_compact", "rkv_oracle_unit", "rkv_oracle_units",
+                  "rkv_oracle_shared_select"):
             getattr(_lib, f).restype = None
     return _lib
 
@@ -165,4 +167,28 @@ def units(q_bits, k_bits, N, budget, lam, red_mode: int = RED_MEAN, pool: int = 
                            _ptr(out["R"]), _ptr(out["Z"]), rows, _ptr(kept), bmax,
                            int(n_threads))
     out["kept"] = kept
+    return out
+
+
+def shared_select(Z_heads, N: int, budget: int):
+    """Shared selection over the heads of one (sequence, layer): Z_heads [H, M]
+    per-head joint scores of the M = N - w candidates.  Returns (Zsum [M],
+    kept [budget]): the top budget - w candidates of the head sum plus the window."""
+    Z = np.ascontiguousarray(Z_heads, dtype=np.float64)
+    H, M = Z.shape
+    out = np.empty(M, dtype=np.float64)
+    kept = np.empty(budget, dtype=np.int32)
+    lib().rkv_oracle_shared_select(_ptr(Z), H, M, M, N, budget, _ptr(out), _ptr(kept))
+    return out, kept
+
+
+def shared_units(q_bits, k_bits, N: int, budget: int, lam: float, red_mode: int = RED_MEAN,
+                 pool: int = POOL_MAX, n_threads: int = 1) -> Dict[str, np.ndarray]:
+    """The shared-selection step of one (sequence, layer): q_bits [H, G, w, D],
+    k_bits [H, rows, D] (every head N rows).  Per-head I, r, R, Z as in `units`,
+    plus Zsum [M] and the one kept set [budget] every head uses."""
+    out = units(q_bits, k_bits, N, budget, lam, red_mode=red_mode, pool=pool, n_threads=n_threads)
+    w = _u16(q_bits).shape[2]
+    M = N - w
+    out["Zsum"], out["kept_shared"] = shared_select(out["Z"][:, :M], N, budget)
     return out

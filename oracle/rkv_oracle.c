@@ -258,6 +258,29 @@ void rkv_oracle_unit(const uint16_t *q, const uint16_t *k, int G, int w, int D, 
 }
 
 /*
+ * Shared selection across the KV heads of one (sequence, layer): the eviction
+ * score of candidate i is the sum over the H heads of their joint scores,
+ * Zsum_i = sum_h Z_h[i] (h ascending, double), and every head keeps the same
+ * set: the top k of Zsum by (score desc, index asc) plus the window.  This is
+ * what a tensor-parallel deployment needs so that all ranks evict the
+ * identical tokens: each rank sums its own heads and an all-reduce (sum) over
+ * the ranks completes Zsum (hysenlabs write-up, decode-time section: the vLLM
+ * port's cross-rank eviction-score all-reduce; every TP rank evicts the
+ * identical set).  Z: H rows of stride zstride; Zsum: [M]; kept: [budget].
+ */
+void rkv_oracle_shared_select(const double *Z, int H, long long zstride, int M, int N,
+                              int budget, double *Zsum, int32_t *kept)
+{
+    for (int i = 0; i < M; ++i) {
+        double s = 0.0;
+        for (int h = 0; h < H; ++h)
+            s += Z[(size_t)h * zstride + i];
+        Zsum[i] = s;
+    }
+    rkv_oracle_select(Zsum, M, N, budget, kept);
+}
+
+/*
  * Many units at once (OpenMP over units when built with -fopenmp).
  * q: [U][G*w*D]; k: [U][kstride] with the first N[u] rows valid;
  * outputs with row strides ostride (I, r, R, Z) and kstride_out (kept).

@@ -102,6 +102,13 @@ def compact(src_bits, kept):
     return np.asarray(src_bits)[np.asarray(kept)]
 
 
+def shared_select(Z_heads, N, budget):
+    """One kept set for all heads of a (sequence, layer): the heads' joint scores
+    summed (the tensor-parallel ranks' all-reduce), then the per-head rule."""
+    Zsum = np.asarray(Z_heads, dtype=np.float64).sum(axis=0)
+    return Zsum, select(Zsum, N, budget)
+
+
 def unit(q_bits, k_bits, N, budget, lam, red_mode=RED_MEAN, pool=POOL_MAX):
     """Whole step for one unit; returns dict of I, r, R, Z (float64 [M]) and kept."""
     w = q_bits.shape[1]

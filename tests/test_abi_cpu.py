@@ -122,10 +122,21 @@ def test_per_head_entry_points_host_validation():
 
 
 def test_step_shape_query():
-    """Two CTAs of the fused kernel must share an SM at the benchmark shapes."""
-    cs, rows, smem = rkv.rkv_query_step_shape(rkv.make_config(), 1152)
+    """Few units: a cluster per unit, two CTAs per SM.  One unit per SM or more:
+    one CTA per unit, two CTAs per SM at the 8B-model shapes."""
+    cfg = rkv.make_config()
+    cs, rows, smem = rkv.rkv_query_step_shape(cfg, 8, 1152)
     assert (cs, rows) == (8, 144) and smem <= 233472 // 2 - 1024
-    cs, rows, smem = rkv.rkv_query_step_shape(rkv.make_config(2048, n_q_heads=40), 2176)
+    cs, rows, smem = rkv.rkv_query_step_shape(cfg, 256, 1152)
+    assert (cs, rows) == (1, 1152) and smem <= 233472 // 2 - 1024
+    cs, rows, smem = rkv.rkv_query_step_shape(rkv.make_config(2048, n_q_heads=40), 8, 2176)
     assert rows * cs >= 2176 and smem <= 233472 // 2 - 1024
+    cs, rows, smem = rkv.rkv_query_step_shape(rkv.make_config(2048, n_q_heads=40), 6144, 2176)
+    assert (cs, rows) == (1, 2176) and smem <= 232448
+    # a unit too long for either kernel's shared memory
     with pytest.raises(rkv.RkvError):
-        rkv.rkv_query_step_shape(rkv.make_config(head_dim=64), 1152)
+        rkv.rkv_query_step_shape(cfg, 6144, 8000)
+    with pytest.raises(rkv.RkvError):
+        rkv.rkv_query_step_shape(rkv.make_config(head_dim=64), 8, 1152)
+    with pytest.raises(rkv.RkvError):
+        rkv.rkv_query_step_shape(cfg, 0, 1152)
