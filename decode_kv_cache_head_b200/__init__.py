@@ -21,6 +21,7 @@ __all__ = [
     "rkv_query_step_shape",
     "rkv_score_importance", "rkv_score_redundancy", "rkv_select_topk", "rkv_compact_kv",
     "rkv_compress_step", "rkv_append_kv",
+    "rkv_workspace_size_shared", "rkv_score_shared", "rkv_select_compact_shared",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -81,6 +82,10 @@ def _load() -> ctypes.CDLL:
         "rkv_compress_step": (ctypes.c_int, [CFG, I32, I32, I32, P, P, P, P, P, P,
                                              ctypes.POINTER(rkv_step_options), P, SZ, P]),
         "rkv_append_kv": (ctypes.c_int, [CFG, I32, I32, I32, P, P, P, P, I32, P, P, SZ, P]),
+        "rkv_workspace_size_shared": (SZ, [CFG, I32, I32, I32]),
+        "rkv_score_shared": (ctypes.c_int, [CFG, I32, I32, I32, P, P, P, P, P, P, P, SZ, P]),
+        "rkv_select_compact_shared": (ctypes.c_int, [CFG, I32, I32, I32, P, P, P, P, P, P, P, SZ,
+                                                     P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -89,6 +94,11 @@ def _load() -> ctypes.CDLL:
     return lib
 
 
+# Compile the library first when it is missing or older than its sources (the
+# build module itself needs no library); without nvcc this raises.
+from . import build as _build  # noqa: E402
+
+_build.build()
 _lib = _load()
 
 
@@ -255,3 +265,45 @@ def rkv_append_kv(cfg, k_layers, v_layers, k_new_layers, v_new_layers, cur_len, 
                                      _ptr_array(k_new_layers), _ptr_array(v_new_layers), n_new,
                                      _ptr(cur_len), _ptr(workspace), ws, _stream(stream)),
                   "rkv_append_kv")
+
+
+def rkv_workspace_size_shared(cfg: rkv_config, n_layers: int, batch: int, cap: int) -> int:
+    return int(_lib.rkv_workspace_size_shared(ctypes.byref(cfg), int(n_layers), int(batch),
+                                              int(cap)))
+
+
+def rkv_score_shared(cfg, k_layers, q_layers, cur_len, z_sum, workspace, budgets=None,
+                     lambdas=None, stream=None):
+    """Shared selection, part 1: z_sum [n_layers, batch, cap] fp32 = the sum over
+    this call's KV heads of their joint scores (cur_len is only read)."""
+    k_layers, q_layers = list(k_layers), list(q_layers)
+    batch, _, cap, _ = k_layers[0].shape
+    for t in k_layers + q_layers:
+        _dtype(t, torch.bfloat16, "k/q")
+    _dtype(cur_len, torch.int32, "cur_len"); _dtype(budgets, torch.int32, "budgets")
+    _dtype(lambdas, torch.float32, "lambdas"); _dtype(z_sum, torch.float32, "z_sum")
+    ws = workspace.numel() * workspace.element_size()
+    return _check(_lib.rkv_score_shared(ctypes.byref(cfg), len(k_layers), batch, cap,
+                                        _ptr_array(k_layers), _ptr_array(q_layers), _ptr(budgets),
+                                        _ptr(lambdas), _ptr(cur_len), _ptr(z_sum),
+                                        _ptr(workspace), ws, _stream(stream)),
+                  "rkv_score_shared", allow_disabled=True)
+
+
+def rkv_select_compact_shared(cfg, k_layers, v_layers, cur_len, z_sum, workspace, budgets=None,
+                              kept_out=None, stream=None):
+    """Shared selection, part 2 (after z_sum is complete over the ranks): one kept
+    set per (layer, sequence), every head of this call compacted in place."""
+    k_layers, v_layers = list(k_layers), list(v_layers)
+    batch, _, cap, _ = k_layers[0].shape
+    for t in k_layers + v_layers:
+        _dtype(t, torch.bfloat16, "k/v")
+    _dtype(cur_len, torch.int32, "cur_len"); _dtype(budgets, torch.int32, "budgets")
+    _dtype(z_sum, torch.float32, "z_sum"); _dtype(kept_out, torch.int32, "kept_out")
+    ws = workspace.numel() * workspace.element_size()
+    return _check(_lib.rkv_select_compact_shared(ctypes.byref(cfg), len(k_layers), batch, cap,
+                                                 _ptr_array(k_layers), _ptr_array(v_layers),
+                                                 _ptr(budgets), _ptr(cur_len), _ptr(z_sum),
+                                                 _ptr(kept_out), _ptr(workspace), ws,
+                                                 _stream(stream)),
+                  "rkv_select_compact_shared", allow_disabled=True)

@@ -142,7 +142,7 @@ struct UnitShape {
 UnitShape unit_shape(int cap, int nqp) {
     UnitShape u = {};
     if (cap > kUnitMaxRows) return u;
-    u.tmem_cols = pow2_at_least(2 * (nqp + 16));
+    u.tmem_cols = pow2_at_least(2 * (nqp + 16) + 16);   // two tile slots + the S accumulator
     u.smem = make_unit_layout(cap, nqp).total;
     const int max_res = 512 / u.tmem_cols;   // CTAs whose TMEM fits one SM
     const size_t floor_smem = static_cast<size_t>(kSmemPerSM / (max_res + 1) - 1024 + 16);
@@ -158,12 +158,104 @@ bool use_unit_kernel(int64_t n_units, int cap, int nqp, int cs_req) {
     return n_units >= kB200SMs && unit_shape(cap, nqp).ok;
 }
 
+// The one-CTA-per-unit kernel over all layers, 32 per launch.  z_heads != null:
+// scores only (shared selection), no cache writes.
+cudaError_t launch_unit_layers(const rkv_config *cfg, int32_t n_layers, int32_t batch, int32_t cap,
+                               const rkv_bf16 *const *k_layers, rkv_bf16 *const *v_layers,
+                               const rkv_bf16 *const *q_layers, const int32_t *budgets,
+                               const float *lambdas, const int32_t *n_eff, const float *r_ext,
+                               int32_t *kept_out, float *scores_out, float *z_heads,
+                               uint32_t *status, const UnitShape &us, int nqp, cudaStream_t strm) {
+    UnitParams *up = new UnitParams();
+    std::memset(up, 0, sizeof(*up));
+    up->batch = batch;
+    up->n_kv = cfg->n_kv_heads;
+    up->group = cfg->n_q_heads / cfg->n_kv_heads;
+    up->window = cfg->window;
+    up->cap = cap;
+    up->nmax = cap;
+    up->tmem_cols = us.tmem_cols;
+    up->budget_cfg = cfg->budget;
+    up->lambda_cfg = cfg->mix_lambda;
+    up->logit_scale_log2 =
+        static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(kHeadDim)));
+    up->red_mode = cfg->redundancy_mode;
+    up->gqa_pool = cfg->gqa_pool;
+    up->budgets = budgets;
+    up->lambdas = lambdas;
+    up->n_eff = n_eff;
+    up->r_ext = r_ext;
+    up->kept_out = kept_out;
+    up->scores_out = scores_out;
+    up->z_heads = z_heads;
+    up->status = status;
+    cudaError_t e = cudaSuccess;
+    for (int l0 = 0; e == cudaSuccess && l0 < n_layers; l0 += kMaxLayersPerLaunch) {
+        const int nl = (n_layers - l0 < kMaxLayersPerLaunch) ? n_layers - l0 : kMaxLayersPerLaunch;
+        up->layer_base = l0;
+        for (int i = 0; i < nl; ++i) {
+            const int l = l0 + i;
+            if (!encode_rows128(&up->tmap_k[i], k_layers[l],
+                                static_cast<uint64_t>(batch) * cfg->n_kv_heads * cap, 128) ||
+                !encode_rows128(&up->tmap_q[i], q_layers[l],
+                                static_cast<uint64_t>(batch) * cfg->n_q_heads * cfg->window,
+                                static_cast<uint32_t>(nqp))) {
+                e = cudaErrorInvalidValue;
+                break;
+            }
+            up->k[i] = const_cast<uint16_t *>(k_layers[l]);
+            up->v[i] = v_layers ? v_layers[l] : nullptr;
+        }
+        if (e == cudaSuccess) e = launch_unit(*up, nl * batch * cfg->n_kv_heads, nqp, us.smem, strm);
+    }
+    delete up;
+    return e;
+}
+
+// MAX mode: raw r of every candidate of every due unit, by the similarity kernel.
+cudaError_t launch_gram_layers(const rkv_config *cfg, int32_t n_layers, int32_t batch, int32_t cap,
+                               const rkv_bf16 *const *k_layers, const int32_t *n_eff, float *r_ext,
+                               uint32_t *status, cudaStream_t strm) {
+    GramParams *gp = new GramParams();
+    std::memset(gp, 0, sizeof(*gp));
+    gp->batch = batch;
+    gp->n_kv = cfg->n_kv_heads;
+    gp->window = cfg->window;
+    gp->cap = cap;
+    gp->nblk = (cap - cfg->window + 127) / 128;
+    gp->n_eff = n_eff;
+    gp->r_out = r_ext;
+    gp->status = status;
+    cudaError_t e = cudaSuccess;
+    for (int l0 = 0; e == cudaSuccess && l0 < n_layers; l0 += kMaxLayersPerLaunch) {
+        const int nl = (n_layers - l0 < kMaxLayersPerLaunch) ? n_layers - l0 : kMaxLayersPerLaunch;
+        gp->layer_base = l0;
+        for (int i = 0; i < nl && e == cudaSuccess; ++i)
+            if (!encode_rows128(&gp->tmap[i], k_layers[l0 + i],
+                                static_cast<uint64_t>(batch) * cfg->n_kv_heads * cap, 128))
+                e = cudaErrorInvalidValue;
+        if (e == cudaSuccess) e = launch_gram_max(*gp, nl * batch * cfg->n_kv_heads, strm);
+    }
+    delete gp;
+    return e;
+}
+
+// Workspace of the shared-selection calls: the step's, then the per-head Z of
+// every unit and the destination of every row of every (layer, sequence).
+size_t ws_bytes_shared(const rkv_config *cfg, int32_t n_layers, int32_t batch, int32_t cap);
+
 size_t ws_bytes_for(const rkv_config *cfg, int32_t n_layers, int32_t batch, int32_t cap) {
     size_t n = kStatusBytes;
     n += align256(static_cast<size_t>(batch) * 4);
     if (cfg->redundancy_mode == RKV_RED_MAX)
         n += align256(static_cast<size_t>(n_layers) * batch * cfg->n_kv_heads * cap * 4);
     return n;
+}
+
+size_t ws_bytes_shared(const rkv_config *cfg, int32_t n_layers, int32_t batch, int32_t cap) {
+    const size_t units = static_cast<size_t>(n_layers) * batch * cfg->n_kv_heads;
+    return ws_bytes_for(cfg, n_layers, batch, cap) + align256(units * cap * 4) +
+           align256(static_cast<size_t>(n_layers) * batch * cap * 4);
 }
 
 void fill_common(StepParams &p, const rkv_config *cfg, const Shape &s, int batch, int cap) {
@@ -466,72 +558,16 @@ rkv_status rkv_compress_step(const rkv_config *cfg, int32_t n_layers, int32_t ba
     if (e == cudaSuccess)
         e = launch_plan(batch, budgets, cfg->budget, cfg->buffer, cfg->window, cap, cur_len, n_eff,
                         status, strm);
-    if (red_max) {   // raw r of every candidate: the tcgen05 similarity kernel
-        GramParams *gp = new GramParams();
-        std::memset(gp, 0, sizeof(*gp));
-        gp->batch = batch;
-        gp->n_kv = cfg->n_kv_heads;
-        gp->window = cfg->window;
-        gp->cap = cap;
-        gp->nblk = (cap - cfg->window + 127) / 128;
-        gp->n_eff = n_eff;
-        gp->r_out = r_ext;
-        gp->status = status;
-        for (int l0 = 0; e == cudaSuccess && l0 < n_layers; l0 += kMaxLayersPerLaunch) {
-            const int nl = (n_layers - l0 < kMaxLayersPerLaunch) ? n_layers - l0 : kMaxLayersPerLaunch;
-            gp->layer_base = l0;
-            for (int i = 0; i < nl && e == cudaSuccess; ++i)
-                if (!encode_rows128(&gp->tmap[i], k_layers[l0 + i],
-                                    static_cast<uint64_t>(batch) * cfg->n_kv_heads * cap, 128))
-                    e = cudaErrorInvalidValue;
-            if (e == cudaSuccess) e = launch_gram_max(*gp, nl * batch * cfg->n_kv_heads, strm);
-        }
-        delete gp;
-    }
+    if (red_max && e == cudaSuccess)   // raw r of every candidate: the tcgen05 similarity kernel
+        e = launch_gram_layers(cfg, n_layers, batch, cap,
+                               const_cast<const rkv_bf16 *const *>(k_layers), n_eff, r_ext, status,
+                               strm);
     if (e == cudaSuccess && opts && opts->main_begin)
         e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->main_begin), strm);
-    if (unit_path) {
-        UnitParams *up = new UnitParams();
-        std::memset(up, 0, sizeof(*up));
-        up->batch = batch;
-        up->n_kv = cfg->n_kv_heads;
-        up->group = cfg->n_q_heads / cfg->n_kv_heads;
-        up->window = cfg->window;
-        up->cap = cap;
-        up->nmax = cap;
-        up->tmem_cols = us.tmem_cols;
-        up->budget_cfg = cfg->budget;
-        up->lambda_cfg = cfg->mix_lambda;
-        up->logit_scale_log2 = p.logit_scale_log2;
-        up->red_mode = cfg->redundancy_mode;
-        up->gqa_pool = cfg->gqa_pool;
-        up->budgets = budgets;
-        up->lambdas = lambdas;
-        up->n_eff = n_eff;
-        up->r_ext = p.r_ext;
-        up->kept_out = p.kept_out;
-        up->scores_out = p.scores_out;
-        up->status = status;
-        for (int l0 = 0; e == cudaSuccess && l0 < n_layers; l0 += kMaxLayersPerLaunch) {
-            const int nl = (n_layers - l0 < kMaxLayersPerLaunch) ? n_layers - l0 : kMaxLayersPerLaunch;
-            up->layer_base = l0;
-            for (int i = 0; i < nl; ++i) {
-                const int l = l0 + i;
-                if (!encode_rows128(&up->tmap_k[i], k_layers[l],
-                                    static_cast<uint64_t>(batch) * cfg->n_kv_heads * cap, 128) ||
-                    !encode_rows128(&up->tmap_q[i], q_layers[l],
-                                    static_cast<uint64_t>(batch) * cfg->n_q_heads * cfg->window,
-                                    static_cast<uint32_t>(nqp))) {
-                    e = cudaErrorInvalidValue;
-                    break;
-                }
-                up->k[i] = k_layers[l];
-                up->v[i] = v_layers[l];
-            }
-            if (e == cudaSuccess) e = launch_unit(*up, nl * batch * cfg->n_kv_heads, nqp, us.smem, strm);
-        }
-        delete up;
-    }
+    if (unit_path && e == cudaSuccess)
+        e = launch_unit_layers(cfg, n_layers, batch, cap, k_layers, v_layers, q_layers, budgets,
+                               lambdas, n_eff, p.r_ext, p.kept_out, p.scores_out, nullptr, status,
+                               us, nqp, strm);
     for (int l0 = 0; !unit_path && e == cudaSuccess && l0 < n_layers; l0 += kMaxLayersPerLaunch) {
         const int nl = (n_layers - l0 < kMaxLayersPerLaunch) ? n_layers - l0 : kMaxLayersPerLaunch;
         p.n_layers = nl;
@@ -604,6 +640,145 @@ rkv_status rkv_append_kv(const rkv_config *cfg, int32_t n_layers, int32_t batch,
         e = launch_append(p, nl, strm);
     }
     if (e == cudaSuccess) e = launch_bump(batch, n_new, cap, cur_len, strm);
+    return cuda_status(e);
+}
+
+size_t rkv_workspace_size_shared(const rkv_config *cfg, int32_t n_layers, int32_t batch,
+                                 int32_t cap) {
+    if (check_cfg(cfg) != RKV_OK || n_layers < 1 || batch < 1 || cap < 2) return 0;
+    return ws_bytes_shared(cfg, n_layers, batch, cap);
+}
+
+}  // extern "C"
+
+namespace {
+
+// Checks shared by the two shared-selection calls (q_layers / v_layers may be
+// absent in one of them).
+rkv_status check_shared_args(const rkv_config *cfg, int32_t n_layers, int32_t batch, int32_t cap,
+                             const rkv_bf16 *const *k_layers, const rkv_bf16 *const *v_layers,
+                             const rkv_bf16 *const *q_layers, const int32_t *budgets,
+                             const void *cur_len, const void *z_sum, const void *workspace,
+                             size_t ws_bytes) {
+    rkv_status st = check_cfg(cfg);
+    if (st != RKV_OK) return st;
+    if (cfg->buffer <= 0 || (!budgets && cfg->budget <= 0)) return RKV_STATUS_DISABLED;
+    if (!k_layers || !cur_len || !z_sum) return RKV_ERR_NULL;
+    if (!workspace) return RKV_ERR_WORKSPACE;
+    if (n_layers < 1 || batch < 1 || cap < 2) return RKV_ERR_INVALID;
+    if (!budgets && (cfg->budget < cfg->window || cfg->budget >= cap)) return RKV_ERR_INVALID;
+    if (static_cast<int64_t>(batch) * cfg->n_kv_heads * cap > INT32_MAX ||
+        static_cast<int64_t>(batch) * cfg->n_q_heads * cfg->window > INT32_MAX)
+        return RKV_ERR_UNSUPPORTED;
+    const int nqp = nqp_of((cfg->n_q_heads / cfg->n_kv_heads) * cfg->window);
+    if (!unit_shape(cap, nqp).ok) return RKV_ERR_UNSUPPORTED;
+    const size_t layer_bytes = static_cast<size_t>(batch) * cfg->n_kv_heads * cap * kHeadDim * 2;
+    for (int l = 0; l < n_layers; ++l) {
+        if (!k_layers[l] || (v_layers && !v_layers[l]) || (q_layers && !q_layers[l]))
+            return RKV_ERR_NULL;
+        if (!aligned16(k_layers[l]) || (v_layers && !aligned16(v_layers[l])) ||
+            (q_layers && !aligned16(q_layers[l])))
+            return RKV_ERR_ALIGN;
+        if (v_layers && overlap(k_layers[l], layer_bytes, v_layers[l], layer_bytes))
+            return RKV_ERR_ALIAS;
+    }
+    if (!aligned16(z_sum)) return RKV_ERR_ALIGN;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return RKV_ERR_ALIGN;
+    if (ws_bytes < ws_bytes_shared(cfg, n_layers, batch, cap)) return RKV_ERR_WORKSPACE;
+    return RKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+rkv_status rkv_score_shared(const rkv_config *cfg, int32_t n_layers, int32_t batch, int32_t cap,
+                            const rkv_bf16 *const *k_layers, const rkv_bf16 *const *q_layers,
+                            const int32_t *budgets, const float *lambdas, const int32_t *cur_len,
+                            float *z_sum, void *workspace, size_t ws_bytes, rkv_stream_t stream) {
+    if (!q_layers) return check_cfg(cfg) != RKV_OK ? check_cfg(cfg) : RKV_ERR_NULL;
+    rkv_status st = check_shared_args(cfg, n_layers, batch, cap, k_layers, nullptr, q_layers,
+                                      budgets, cur_len, z_sum, workspace, ws_bytes);
+    if (st != RKV_OK) return st;
+    const int nqp = nqp_of((cfg->n_q_heads / cfg->n_kv_heads) * cfg->window);
+    const UnitShape us = unit_shape(cap, nqp);
+    cudaStream_t strm = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    uint32_t *status = reinterpret_cast<uint32_t *>(ws);
+    int32_t *n_eff = reinterpret_cast<int32_t *>(ws + kStatusBytes);
+    const size_t base = ws_bytes_for(cfg, n_layers, batch, cap);
+    float *r_ext = reinterpret_cast<float *>(ws + kStatusBytes + align256(static_cast<size_t>(batch) * 4));
+    float *z_heads = reinterpret_cast<float *>(ws + base);
+    const bool red_max = cfg->redundancy_mode == RKV_RED_MAX;
+    cudaError_t e = cudaMemsetAsync(ws, 0, kStatusBytes, strm);
+    if (e == cudaSuccess)
+        e = launch_plan(batch, budgets, cfg->budget, cfg->buffer, cfg->window, cap,
+                        const_cast<int32_t *>(cur_len), n_eff, status, strm, false);
+    if (red_max && e == cudaSuccess)
+        e = launch_gram_layers(cfg, n_layers, batch, cap, k_layers, n_eff, r_ext, status, strm);
+    if (e == cudaSuccess)
+        e = launch_unit_layers(cfg, n_layers, batch, cap, k_layers, nullptr, q_layers, budgets,
+                               lambdas, n_eff, red_max ? r_ext : nullptr, nullptr, nullptr, z_heads,
+                               status, us, nqp, strm);
+    SharedParams sp;
+    std::memset(&sp, 0, sizeof(sp));
+    sp.batch = batch;
+    sp.n_kv = cfg->n_kv_heads;
+    sp.window = cfg->window;
+    sp.cap = cap;
+    sp.n_eff = n_eff;
+    sp.z_heads = z_heads;
+    sp.z_sum = z_sum;
+    sp.status = status;
+    if (e == cudaSuccess) e = launch_head_sum(sp, n_layers * batch, strm);
+    return cuda_status(e);
+}
+
+rkv_status rkv_select_compact_shared(const rkv_config *cfg, int32_t n_layers, int32_t batch,
+                                     int32_t cap, rkv_bf16 *const *k_layers,
+                                     rkv_bf16 *const *v_layers, const int32_t *budgets,
+                                     int32_t *cur_len, const float *z_sum, int32_t *kept_out,
+                                     void *workspace, size_t ws_bytes, rkv_stream_t stream) {
+    if (!v_layers) return check_cfg(cfg) != RKV_OK ? check_cfg(cfg) : RKV_ERR_NULL;
+    rkv_status st = check_shared_args(cfg, n_layers, batch, cap,
+                                      const_cast<const rkv_bf16 *const *>(k_layers),
+                                      const_cast<const rkv_bf16 *const *>(v_layers), nullptr,
+                                      budgets, cur_len, z_sum, workspace, ws_bytes);
+    if (st != RKV_OK) return st;
+    cudaStream_t strm = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    uint32_t *status = reinterpret_cast<uint32_t *>(ws);
+    int32_t *n_eff = reinterpret_cast<int32_t *>(ws + kStatusBytes);
+    const size_t units = static_cast<size_t>(n_layers) * batch * cfg->n_kv_heads;
+    int32_t *dst = reinterpret_cast<int32_t *>(ws + ws_bytes_for(cfg, n_layers, batch, cap) +
+                                               align256(units * cap * 4));
+    cudaError_t e = cudaMemsetAsync(ws, 0, kStatusBytes, strm);
+    if (e == cudaSuccess)
+        e = launch_plan(batch, budgets, cfg->budget, cfg->buffer, cfg->window, cap, cur_len, n_eff,
+                        status, strm, true);
+    SharedParams sp;
+    std::memset(&sp, 0, sizeof(sp));
+    sp.batch = batch;
+    sp.n_kv = cfg->n_kv_heads;
+    sp.window = cfg->window;
+    sp.cap = cap;
+    sp.budget_cfg = cfg->budget;
+    sp.budgets = budgets;
+    sp.n_eff = n_eff;
+    sp.status = status;
+    for (int l0 = 0; e == cudaSuccess && l0 < n_layers; l0 += kMaxLayersPerLaunch) {
+        const int nl = (n_layers - l0 < kMaxLayersPerLaunch) ? n_layers - l0 : kMaxLayersPerLaunch;
+        const size_t off = static_cast<size_t>(l0) * batch * cap;
+        sp.z_sum = const_cast<float *>(z_sum) + off;
+        sp.dst = dst + off;
+        sp.kept_out = kept_out ? kept_out + off : nullptr;
+        for (int i = 0; i < nl; ++i) {
+            sp.k[i] = k_layers[l0 + i];
+            sp.v[i] = v_layers[l0 + i];
+        }
+        e = launch_shared_select(sp, nl * batch, strm);
+        if (e == cudaSuccess) e = launch_shared_compact(sp, nl * batch * cfg->n_kv_heads, strm);
+    }
     return cuda_status(e);
 }
 

@@ -125,7 +125,7 @@ inline cudaError_t ensure_smem_attr(K kernel, size_t bytes, std::atomic<int> &gr
 // Launchers (defined in the .cu files); all return cudaSuccess or the launch error.
 cudaError_t launch_plan(int batch, const int32_t *budgets, int32_t budget_cfg, int32_t buffer,
                         int32_t window, int32_t cap, int32_t *cur_len, int32_t *n_eff,
-                        uint32_t *status, cudaStream_t stream);
+                        uint32_t *status, cudaStream_t stream, bool update = true);
 cudaError_t launch_step(const StepParams &p, int n_units, int nqp, size_t smem,
                         cudaStream_t stream);
 size_t step_smem_bytes(int rp, int rmax, int cap, int nqp, int cs);
@@ -158,6 +158,8 @@ struct alignas(64) UnitParams {
     const float *r_ext;
     int32_t *kept_out;
     float *scores_out;
+    float *z_heads;        // shared selection: Z of every candidate [units][cap]; then no
+                           // select, no compaction
     uint32_t *status;
 };
 
@@ -165,11 +167,13 @@ constexpr int kUnitThreads = 256;
 constexpr int kUnitMaxRows = 7680;     // keys + destinations + histograms fit the 64 KB ring
 
 struct UnitLayout {
-    uint32_t stage, b, inv, self, ia, ib, r, scr, s, colm, colf, vis, red, bars, total;
+    uint32_t stage, b, bs, inv, self, ia, ib, r, scr, s, colm, colf, vis, red, bars, total;
 };
 
-// Offsets from a 1024-byte-aligned base.  The two 32 KB ring stages are reused
-// after the last tile for the select keys, the destinations and the histograms.
+// Offsets from a 1024-byte-aligned base.  Lifetimes share bytes: the two 32 KB
+// ring stages hold, after the last tile, the select keys, the destinations and
+// the histograms; the B operand of the S UMMA (pass 1) shares bytes with the
+// pass-2 arrays Ihat halves and r (the last S UMMA completes between the passes).
 __host__ __device__ inline UnitLayout make_unit_layout(int nmax, int nqp) {
     UnitLayout L;
     uint32_t o = 0;
@@ -178,10 +182,13 @@ __host__ __device__ inline UnitLayout make_unit_layout(int nmax, int nqp) {
     const uint32_t arr = align_up(static_cast<uint32_t>(nmax) * 4u, 16);
     L.inv = o;    o += arr;
     L.self = o;   o += arr;
-    L.ia = o;     o += arr;
-    L.ib = o;     o += arr;
-    L.r = o;      o += arr;
-    L.scr = o;    o += 8192u;
+    o = align_up(o, 1024);
+    L.bs = o;                                          // pass 1: inv split, 2 x 4 KB
+    L.ia = o;                                          // pass 2: Ihat halves and r
+    L.ib = o + arr;
+    L.r = o + 2u * arr;
+    o += (3u * arr > 8192u) ? 3u * arr : 8192u;
+    L.scr = o;    o += 2048u;                          // column (max, sum) per warp
     L.s = o;      o += 512u;
     L.colm = o;   o += 256u;
     L.colf = o;   o += 256u;
@@ -194,6 +201,25 @@ __host__ __device__ inline UnitLayout make_unit_layout(int nmax, int nqp) {
 
 cudaError_t launch_unit(const UnitParams &p, int n_units, int nqp, size_t smem,
                         cudaStream_t stream);
+
+// Shared selection (rkv_shared.cu): pointers already offset to the launch's
+// first layer.
+struct SharedParams {
+    uint16_t *k[kMaxLayersPerLaunch];
+    uint16_t *v[kMaxLayersPerLaunch];
+    int32_t batch, n_kv, window, cap, budget_cfg;
+    const int32_t *budgets;
+    const int32_t *n_eff;
+    const float *z_heads;    // [layers][batch][Hkv][cap] per-head Z
+    float *z_sum;            // [layers][batch][cap]
+    int32_t *dst;            // [layers][batch][cap] destination row or -1
+    int32_t *kept_out;       // optional [layers][batch][cap]
+    uint32_t *status;
+};
+cudaError_t launch_head_sum(const SharedParams &p, int n_lb, cudaStream_t stream);
+cudaError_t launch_shared_select(const SharedParams &p, int n_lb, cudaStream_t stream);
+cudaError_t launch_shared_compact(const SharedParams &p, int n_units, cudaStream_t stream);
+size_t shared_select_smem(int cap);
 
 // MAX-mode similarity kernel: raw r of every candidate of every due unit.
 struct alignas(64) GramParams {

@@ -227,6 +227,21 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t smem_addr) {
     return d;
 }
 
+// UMMA shared-memory descriptor of an MN-major operand stored with the
+// 128-byte swizzle: 128-byte rows each hold 64 consecutive M (or N) elements of
+// one K index; rows of consecutive K are 128 bytes apart, 8-row K groups
+// `sbo` bytes apart, and 64-element M blocks `lbo` bytes apart.
+__device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t smem_addr, uint32_t lbo,
+                                                       uint32_t sbo) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+    d |= static_cast<uint64_t>(1u) << 46;
+    d |= static_cast<uint64_t>(2u) << 61;
+    return d;
+}
+
 // UMMA instruction descriptor, kind::f16: A = B = bf16, D = fp32, both K-major.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
     return (1u << 4)                                   // D format: F32
@@ -234,6 +249,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
            | (1u << 10)                                // B format: BF16
            | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
            | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
+}
+
+// The same with A stored MN-major (B K-major).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_amn(int M, int N) {
+    return idesc_bf16_f32(M, N) | (1u << 15);
 }
 
 // Byte offset of 16-byte chunk `c` (0..7) of row `r` inside a 128-byte-swizzled

@@ -61,7 +61,8 @@ namespace rkv {
 __global__ void rkv_plan_kernel(int batch, const int32_t *__restrict__ budgets,
                                 int32_t budget_cfg, int32_t buffer, int32_t window,
                                 int32_t cap, int32_t *__restrict__ cur_len,
-                                int32_t *__restrict__ n_eff, uint32_t *__restrict__ status) {
+                                int32_t *__restrict__ n_eff, uint32_t *__restrict__ status,
+                                int update) {
     const int b = blockIdx.x * blockDim.x + threadIdx.x;
     if (b >= batch) return;
     const int32_t bud = budgets ? budgets[b] : budget_cfg;
@@ -73,16 +74,16 @@ __global__ void rkv_plan_kernel(int batch, const int32_t *__restrict__ budgets,
         due = false;
     }
     n_eff[b] = due ? n : 0;
-    if (due) cur_len[b] = bud;
+    if (due && update) cur_len[b] = bud;
 }
 
 cudaError_t launch_plan(int batch, const int32_t *budgets, int32_t budget_cfg, int32_t buffer,
                         int32_t window, int32_t cap, int32_t *cur_len, int32_t *n_eff,
-                        uint32_t *status, cudaStream_t stream) {
+                        uint32_t *status, cudaStream_t stream, bool update) {
     const int threads = 128;
     const int blocks = (batch + threads - 1) / threads;
     rkv_plan_kernel<<<blocks, threads, 0, stream>>>(batch, budgets, budget_cfg, buffer, window,
-                                                    cap, cur_len, n_eff, status);
+                                                    cap, cur_len, n_eff, status, update ? 1 : 0);
     return cudaGetLastError();
 }
 

@@ -151,8 +151,8 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
     uint64_t *sVis = reinterpret_cast<uint64_t *>(base + L.vis);
     float *sRed = reinterpret_cast<float *>(base + L.red);
     uint32_t *sRedU = reinterpret_cast<uint32_t *>(base + L.red);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(base + L.bars);   // full[2], mma[2]
-    uint32_t *sTmem = reinterpret_cast<uint32_t *>(bars + 4);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(base + L.bars);   // full[2], mma[2], smma[2]
+    uint32_t *sTmem = reinterpret_cast<uint32_t *>(bars + 6);
     // after the last tile the ring holds the keys, the destinations and the histograms
     const uint32_t arr = align_up(static_cast<uint32_t>(p.nmax) * 4u, 16);
     uint32_t *sKeys = reinterpret_cast<uint32_t *>(sStage);
@@ -167,20 +167,25 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
     }();
 
     // ---- set-up
+    uint8_t *sBs = base + L.bs;   // B operand of the S UMMA, two buffers of 16 rows x 128 tokens
+    uint64_t *full = bars, *mmab = bars + 2, *smma = bars + 4;
     if (warp == 0) {
         tmem_alloc(sTmem, static_cast<uint32_t>(p.tmem_cols));
         tmem_relinquish();
     }
     if (tid == 32) {
-        for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 6; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
     }
-    // B operand rows past the queries start as zeros (the split S lands in three of them)
+    // B operand rows past the queries start as zeros (the split S lands in three of
+    // them), and so do both S-UMMA B buffers (rows 3..15 stay zero)
     for (int i = tid; i < 2 * 16 * 8; i += NT) {
         const int half = i >> 7, row = NQP + ((i & 127) >> 3), ch = i & 7;
         *reinterpret_cast<uint4 *>(sB + half * kBRows * 128u + row * 128u + ch * 16u) =
             make_uint4(0u, 0u, 0u, 0u);
     }
+    for (int i = tid; i < 2 * 4096 / 16; i += NT)
+        reinterpret_cast<uint4 *>(sBs)[i] = make_uint4(0u, 0u, 0u, 0u);
     // window key M + d is seen by query column g*w + j only when j >= d (causal)
     if (warp == 0) {
         const int j0 = lane % w, j1 = (lane + 32) % w;
@@ -195,23 +200,43 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *sTmem;
+    const uint32_t scol = static_cast<uint32_t>(2 * SLOT);   // S accumulator columns
 
+    // last tile / logits UMMA / S UMMA issued (thread 0's copies), for the error path
+    int tma_last = 1, mma_last = -1, smma_last = -1;
     const CUtensorMap *mk = &p.tmap_k[l];
     auto issue_tile = [&](int g) {   // global tile g: pass 1 for g < T, pass 2 after
+        tma_last = g;
         const int tt = g < T ? g : g - T;
         uint8_t *stg = sStage + (g & 1) * kStageBytes;
         const int32_t y = static_cast<int32_t>(krow0 + tt * kTileRows);
-        tma_load_2d(stg, mk, &bars[g & 1], 0, y);
-        tma_load_2d(stg + kHalfBytes, mk, &bars[g & 1], 64, y);
+        tma_load_2d(stg, mk, &full[g & 1], 0, y);
+        tma_load_2d(stg + kHalfBytes, mk, &full[g & 1], 64, y);
     };
-    if (tid == 32) {
+    // logits (and in pass 2 of MEAN mode k . S) of tile g into TMEM slot g & 1
+    auto issue_logits = [&](int g) {
+        mma_last = g;
+        tc_fence_after();
+        const bool with_s = g >= T && !red_max;
+        const uint32_t idesc = with_s ? idesc_bf16_f32(128, NQP + 16) : idesc_bf16_f32(128, NQP);
+        const uint32_t a_base = smem_u32(sStage + (g & 1) * kStageBytes), b_base = smem_u32(sB);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t half = ks >> 2, koff = (ks & 3) * 32u;
+            const uint64_t ad = desc_kmajor_sw128(a_base + half * kHalfBytes + koff);
+            const uint64_t bd = desc_kmajor_sw128(b_base + half * kBRows * 128u + koff);
+            umma_bf16(tmem_base + static_cast<uint32_t>((g & 1) * SLOT), ad, bd, idesc, ks > 0 ? 1u : 0u);
+        }
+        umma_commit(&mmab[g & 1]);
+    };
+    if (tid == 0) {
         const CUtensorMap *mq = &p.tmap_q[l];
         const int32_t yq = (b * p.n_kv + h) * NQ;   // the KV head's query rows
-        mbar_arrive_expect_tx(&bars[0], kStageBytes + static_cast<uint32_t>(NQP) * 256u);
-        tma_load_2d(sB, mq, &bars[0], 0, yq);
-        tma_load_2d(sB + kBRows * 128u, mq, &bars[0], 64, yq);
+        mbar_arrive_expect_tx(&full[0], kStageBytes + static_cast<uint32_t>(NQP) * 256u);
+        tma_load_2d(sB, mq, &full[0], 0, yq);
+        tma_load_2d(sB + kBRows * 128u, mq, &full[0], 64, yq);
         issue_tile(0);
-        mbar_arrive_expect_tx(&bars[1], kStageBytes);
+        mbar_arrive_expect_tx(&full[1], kStageBytes);
         issue_tile(1);
     }
 
@@ -223,8 +248,7 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
     const int lrow = (warp & 3) * 32 + lane;   // TMEM lane = tile row
     // norms: lanes 0-7 / 16-23 take the first 64 columns of rows (l & 7) + 8 (l >> 4)
     const int nrow = (lane & 7) + 8 * (lane >> 4), nhalf = (lane >> 3) & 1;
-    // S partial: lane owns columns shalf * 64 + (lane & 15) * 4 .. + 3
-    const int shalf = lane >> 4, schunk = (lane & 15) >> 1, ssub = lane & 1;
+    const int row_t = 16 * warp + nrow;        // this lane's tile row in the norms
 
     float cm[HC], cs[HC];
 #pragma unroll
@@ -232,7 +256,6 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
         cm[c] = -INFINITY;
         cs[c] = 0.f;
     }
-    float2 sacc0 = make_float2(0.f, 0.f), sacc1 = make_float2(0.f, 0.f);
     bool ok = true;
     int g = 0;
     for (; g < 2 * T; ++g) {
@@ -240,12 +263,82 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
         const int tt = pass2 ? g - T : g;
         const int s = g & 1;
         const uint32_t par = static_cast<uint32_t>((g >> 1) & 1);
-        const uint8_t *stg = sStage + s * kStageBytes;
+        uint8_t *stg = sStage + s * kStageBytes;
         const uint32_t tslot = static_cast<uint32_t>(s * SLOT);
+        bool wait_ok = true;
 
-        if (g == T) {
+        if (!pass2) {
+            wait_ok = mbar_wait(&full[s], par);
+            if (tid == 0 && wait_ok) issue_logits(g);
+            if (!red_max) {
+                if (wait_ok) {
+                    // ||k_i||^2 and 1 / max(||k_i||, 1e-12): two lanes per row, 64 columns each
+                    const int i = tt * kTileRows + row_t;
+                    const uint8_t *hp = stg + nhalf * kHalfBytes + row_t * 128;
+                    float2 ss2 = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint4 raw = *reinterpret_cast<const uint4 *>(hp + ((c ^ (row_t & 7)) << 4));
+                        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f = __bfloat1622float2(h2[e]);
+                            ss2 = __ffma2_rn(f, f, ss2);
+                        }
+                    }
+                    const float ssh = ss2.x + ss2.y;
+                    const float ss = ssh + __shfl_xor_sync(kFull, ssh, 8);
+                    const float inv = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
+                    if (nhalf == 0) {
+                        // inv as hi + mid + lo bf16: column row_t of the S-UMMA B operand
+                        const bool in = i < N;
+                        const uint16_t hi = in ? bf16_rn_bits(inv) : 0;
+                        const float r1 = inv - bf16_bits_to_float(hi);
+                        const uint16_t mid = in ? bf16_rn_bits(r1) : 0;
+                        const uint16_t lo = in ? bf16_rn_bits(r1 - bf16_bits_to_float(mid)) : 0;
+                        uint8_t *bb = sBs + s * 4096 + (row_t >> 6) * 2048;
+                        const uint32_t c = (row_t & 63) >> 3, e = (row_t & 7) * 2u;
+                        *reinterpret_cast<uint16_t *>(bb + sw128_offset(0, c) + e) = hi;
+                        *reinterpret_cast<uint16_t *>(bb + sw128_offset(1, c) + e) = mid;
+                        *reinterpret_cast<uint16_t *>(bb + sw128_offset(2, c) + e) = lo;
+                        if (in) {
+                            sInv[i] = inv;
+                            sSelf[i] = inv * inv * ss;
+                        }
+                    }
+                }
+                if (tt == T - 1 && N < T * kTileRows) {
+                    // rows past N (stale cache memory) become zeros before the S UMMA
+                    // sums over them; the logits UMMA has finished reading them
+                    wait_ok = wait_ok && mbar_wait(&mmab[s], par);
+                    const int nv = N - tt * kTileRows;
+                    for (int idx = tid; idx < (kTileRows - nv) * 16; idx += NT) {
+                        const int r = nv + (idx >> 4), c = idx & 15;
+                        *reinterpret_cast<uint4 *>(stg + (c >> 3) * kHalfBytes + r * 128 + ((c & 7) << 4)) =
+                            make_uint4(0u, 0u, 0u, 0u);
+                    }
+                }
+                fence_proxy_async_smem();
+                __syncthreads();
+                if (tid == 0 && wait_ok) {
+                    // S += K_tile^T . inv: A = the K tile read MN-major (M = 128 columns,
+                    // 64-column blocks 16 KB apart, 8-row groups 1 KB apart), B = inv split
+                    tc_fence_after();
+                    constexpr uint32_t idesc_s = idesc_bf16_f32_amn(128, 16);
+                    const uint32_t a_base = smem_u32(stg), b_base = smem_u32(sBs + s * 4096);
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint64_t ad = desc_mnmajor_sw128(a_base + ks * 2048u, kHalfBytes, 1024u);
+                        const uint64_t bd = desc_kmajor_sw128(b_base + (ks >> 2) * 2048u + (ks & 3) * 32u);
+                        umma_bf16(tmem_base + scol, ad, bd, idesc_s, (g > 0 || ks > 0) ? 1u : 0u);
+                    }
+                    umma_commit(&smma[s]);
+                    smma_last = g;
+                }
+            }
+        } else if (g == T) {
             // ---- between the passes: column (max, sum) over the CTA; S split into B
-            float *xm = sScr + 1024;   // [8 warps][HC] (m, s) pairs
+            float *xm = sScr;   // [8 warps][HC] (m, s) pairs
 #pragma unroll
             for (int c0 = 0; c0 < HC; c0 += 8) {
                 float m8[8], s8[8];
@@ -261,9 +354,25 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
                 }
             }
             if (!red_max) {
-                const int col = shalf * 64 + (lane & 15) * 4;
-                *reinterpret_cast<float4 *>(sScr + warp * 128 + col) =
-                    make_float4(sacc0.x, sacc0.y, sacc1.x, sacc1.y);
+                wait_ok = mbar_wait(&smma[(T - 1) & 1], static_cast<uint32_t>(((T - 1) >> 1) & 1));
+                tc_fence_after();
+                if (warp < 4 && wait_ok) {
+                    uint32_t sv[4];
+                    tmem_ld4_nowait(tmem_lane + scol, sv);
+                    tmem_wait_ld();
+                    reg_tie4(sv);
+                    const float S = (__uint_as_float(sv[0]) + __uint_as_float(sv[1])) + __uint_as_float(sv[2]);
+                    const int d = 32 * warp + lane;
+                    const uint16_t hi = bf16_rn_bits(S);
+                    const float r1 = S - bf16_bits_to_float(hi);
+                    const uint16_t mid = bf16_rn_bits(r1);
+                    const uint16_t lo = bf16_rn_bits(r1 - bf16_bits_to_float(mid));
+                    uint8_t *hb = sB + (d >> 6) * kBRows * 128u;
+                    const uint32_t c = (d & 63) >> 3, e = (d & 7) * 2u;
+                    *reinterpret_cast<uint16_t *>(hb + sw128_offset(NQP + 0, c) + e) = hi;
+                    *reinterpret_cast<uint16_t *>(hb + sw128_offset(NQP + 1, c) + e) = mid;
+                    *reinterpret_cast<uint16_t *>(hb + sw128_offset(NQP + 2, c) + e) = lo;
+                }
             }
             __syncthreads();
             if (tid < NQP) {
@@ -275,81 +384,15 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
                 sColM[q] = m;
                 sColF[q] = sm > 0.f ? 1.0f / sm : 0.f;
             }
-            if (!red_max && tid >= 128) {
-                const int d = tid - 128;
-                float S = sScr[d];
-#pragma unroll
-                for (int k = 1; k < NW; ++k) S += sScr[k * 128 + d];
-                const uint16_t hi = bf16_rn_bits(S);
-                const float r1 = S - bf16_bits_to_float(hi);
-                const uint16_t mid = bf16_rn_bits(r1);
-                const uint16_t lo = bf16_rn_bits(r1 - bf16_bits_to_float(mid));
-                uint8_t *hb = sB + (d >> 6) * kBRows * 128u;
-                const uint32_t c = (d & 63) >> 3, e = (d & 7) * 2u;
-                *reinterpret_cast<uint16_t *>(hb + sw128_offset(NQP + 0, c) + e) = hi;
-                *reinterpret_cast<uint16_t *>(hb + sw128_offset(NQP + 1, c) + e) = mid;
-                *reinterpret_cast<uint16_t *>(hb + sw128_offset(NQP + 2, c) + e) = lo;
-            }
             fence_proxy_async_smem();
+            tc_fence_before();
             __syncthreads();
-        }
-
-        bool wait_ok = mbar_wait(&bars[s], par);
-        if (tid == 0 && wait_ok) {
-            tc_fence_after();
-            const uint32_t idesc = (pass2 && !red_max) ? idesc_bf16_f32(128, NQP + 16)
-                                                       : idesc_bf16_f32(128, NQP);
-            const uint32_t a_base = smem_u32(stg), b_base = smem_u32(sB);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t half = ks >> 2, koff = (ks & 3) * 32u;
-                const uint64_t ad = desc_kmajor_sw128(a_base + half * kHalfBytes + koff);
-                const uint64_t bd = desc_kmajor_sw128(b_base + half * kBRows * 128u + koff);
-                umma_bf16(tmem_base + tslot, ad, bd, idesc, ks > 0 ? 1u : 0u);
-            }
-            umma_commit(&bars[2 + s]);
-        }
-
-        if (!pass2 && !red_max && wait_ok) {
-            // ||k_i||^2 and 1 / max(||k_i||, 1e-12): two lanes per row, 64 columns each
-            const int row_t = 16 * warp + nrow;
-            const int i = tt * kTileRows + row_t;
-            const uint8_t *hp = stg + nhalf * kHalfBytes;
-            float2 ss2 = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const uint4 raw = *reinterpret_cast<const uint4 *>(hp + sw128_offset(row_t, c));
-                const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 f = __bfloat1622float2(h2[e]);
-                    ss2 = __ffma2_rn(f, f, ss2);
-                }
-            }
-            float ssh = ss2.x + ss2.y;
-            const float ss = ssh + __shfl_xor_sync(kFull, ssh, 8);
-            const float inv = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
-            if (nhalf == 0 && i < N) {
-                sInv[i] = inv;
-                sSelf[i] = inv * inv * ss;
-            }
-            // this warp's 16 rows into the S partial (each lane 4 columns)
-            const uint8_t *sp = stg + shalf * kHalfBytes;
-#pragma unroll 4
-            for (int r = 0; r < 16; ++r) {
-                const float iv = __shfl_sync(kFull, inv, (r & 7) + 16 * (r >> 3));
-                if (tt * kTileRows + 16 * warp + r < N) {
-                    const uint2 raw = *reinterpret_cast<const uint2 *>(
-                        sp + sw128_offset(16 * warp + r, schunk) + ssub * 8);
-                    const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-                    const float2 iv2 = make_float2(iv, iv);
-                    sacc0 = __ffma2_rn(__bfloat1622float2(h2[0]), iv2, sacc0);
-                    sacc1 = __ffma2_rn(__bfloat1622float2(h2[1]), iv2, sacc1);
-                }
+            if (tid == 0 && wait_ok) {
+                if (mbar_wait(&full[s], par)) issue_logits(g);
             }
         }
 
-        wait_ok = wait_ok && mbar_wait(&bars[2 + s], par);
+        wait_ok = wait_ok && mbar_wait(&mmab[s], par);
         tc_fence_after();
         const int i = tt * kTileRows + lrow;
         if (wait_ok && !pass2) {
@@ -472,20 +515,42 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
             ok = false;
             break;
         }
-        if (tid == 32 && g + 2 < 2 * T) {
-            mbar_arrive_expect_tx(&bars[s], kStageBytes);
-            issue_tile(g + 2);
+        if (tid == 0) {
+            // stage s is free once every UMMA reading it is done: the logits one
+            // (waited above by everyone) and, in pass 1, the S one
+            if (g + 2 < 2 * T) {
+                if (pass2 || red_max || mbar_wait(&smma[s], par)) {
+                    mbar_arrive_expect_tx(&full[s], kStageBytes);
+                    issue_tile(g + 2);
+                } else {
+                    ok = false;
+                }
+            }
+            // pass 2: the next tile's UMMA now, so that it runs during this warp's wait
+            if (pass2 && ok && g + 1 < 2 * T) {
+                if (mbar_wait(&full[(g + 1) & 1], static_cast<uint32_t>(((g + 1) >> 1) & 1)))
+                    issue_logits(g + 1);
+                else
+                    ok = false;
+            }
+        }
+        if (__syncthreads_or(!ok)) {
+            ok = false;
+            break;
         }
     }
 
     if (!ok) {
         // A wait ran out: record it, wait (bounded) for this CTA's copies and
         // UMMAs still in flight, free TMEM and leave without writing anything.
-        if (tid == 32) {
+        if (tid == 0) {
             record_flag(p.status, kDevFlagTimeout);
-            for (int gg = g; gg < g + 2 && gg < 2 * T; ++gg)
-                (void)mbar_wait(&bars[gg & 1], static_cast<uint32_t>((gg >> 1) & 1));
-            (void)mbar_wait(&bars[2 + (g & 1)], static_cast<uint32_t>((g >> 1) & 1));
+            for (int gg = g; gg <= tma_last; ++gg)
+                (void)mbar_wait(&full[gg & 1], static_cast<uint32_t>((gg >> 1) & 1));
+            for (int gg = g; gg <= mma_last; ++gg)
+                (void)mbar_wait(&mmab[gg & 1], static_cast<uint32_t>((gg >> 1) & 1));
+            for (int gg = g; gg <= smma_last; ++gg)
+                (void)mbar_wait(&smma[gg & 1], static_cast<uint32_t>((gg >> 1) & 1));
         }
         __syncthreads();
         if (warp == 0) {
@@ -500,12 +565,31 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
     uint32_t Tk = 0xffffffffu;
     int n_gt = 0;
     const float invG = 1.0f / static_cast<float>(G);
+    const bool scores_only = p.z_heads != nullptr;
     post_scores_any<NT, 1>(
         [&](int j) {
             const float a = sIa[j], c = sIb[j];
             return make_float2(pool_max ? fmaxf(a, c) : (a + c) * invG, sR[j]);
         },
-        sKeys, sHist, sRed, M, kk, lam, true, inv_sumI, rmax_g, inv_rsum, Tk, n_gt);
+        sKeys, sHist, sRed, M, kk, lam, !scores_only, inv_sumI, rmax_g, inv_rsum, Tk, n_gt);
+
+    if (scores_only) {
+        // shared selection: this head's joint score of every candidate; the
+        // heads (and ranks) are summed and one set is selected afterwards
+        float *zo = p.z_heads + unit_g * p.cap;
+        for (int row = tid; row < M; row += NT) {
+            const float a = sIa[row], c = sIb[row];
+            const float I = (pool_max ? fmaxf(a, c) : (a + c) * invG) * inv_sumI;
+            const float Rv = ex2_approx((sR[row] - rmax_g) * kLog2e) * inv_rsum;
+            zo[row] = joint_score(lam, I, Rv);
+        }
+        __syncthreads();
+        if (warp == 0) {
+            tc_fence_after();
+            tmem_dealloc(tmem_base, static_cast<uint32_t>(p.tmem_cols));
+        }
+        return;
+    }
 
     // ---- destination of every row: G_i = rows above the threshold or in the
     // window before i, E_i = tied candidates before i;

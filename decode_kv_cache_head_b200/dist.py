@@ -4,6 +4,11 @@ Every (sequence, layer, KV head) unit of the step is independent, so ranks
 shard sequences and never exchange data on the compute path.  What they share
 is bookkeeping: which sequences a rank owns, a distinct input seed per rank
 (for synthetic runs), and the step time taken as the maximum over ranks.
+
+The one exchange is the shared selection of tensor-parallel ranks (each rank
+holds some KV heads and all ranks must evict the same tokens): the ranks'
+eviction scores are summed by an all-reduce between the scoring call and the
+select-and-compact call.
 """
 from __future__ import annotations
 
@@ -49,3 +54,30 @@ def barrier(device=None) -> None:
             torch.distributed.barrier(device_ids=[device.index])
         else:
             torch.distributed.barrier()
+
+
+def head_range(n_kv_heads: int, world_size: int, rank: int) -> Tuple[int, int]:
+    """Tensor parallelism: the contiguous KV heads [start, stop) of `rank`."""
+    if n_kv_heads % world_size:
+        raise ValueError(f"{n_kv_heads} KV heads do not split over {world_size} ranks")
+    per = n_kv_heads // world_size
+    return rank * per, (rank + 1) * per
+
+
+def allreduce_eviction_scores(z_sum: torch.Tensor, group=None) -> torch.Tensor:
+    """Sum of the ranks' eviction scores, in place (identity on one rank)."""
+    ws, _ = world()
+    if ws > 1:
+        torch.distributed.all_reduce(z_sum, op=torch.distributed.ReduceOp.SUM, group=group)
+    return z_sum
+
+
+def compress_step_shared(rkv, cfg, k_layers, v_layers, q_layers, cur_len, z_sum, workspace,
+                         budgets=None, lambdas=None, kept_out=None, group=None, stream=None):
+    """The tensor-parallel step: this rank's heads scored, the scores summed over
+    the ranks, and one kept set per (layer, sequence) applied to this rank's heads."""
+    rkv.rkv_score_shared(cfg, k_layers, q_layers, cur_len, z_sum, workspace, budgets=budgets,
+                         lambdas=lambdas, stream=stream)
+    allreduce_eviction_scores(z_sum, group)
+    return rkv.rkv_select_compact_shared(cfg, k_layers, v_layers, cur_len, z_sum, workspace,
+                                         budgets=budgets, kept_out=kept_out, stream=stream)

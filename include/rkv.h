@@ -287,6 +287,52 @@ RKV_API rkv_status rkv_compress_step_noalloc(const rkv_config *cfg, int32_t n_la
                                              int32_t *cur_len, const rkv_step_options *opts,
                                              rkv_stream_t stream);
 
+/*
+ * Shared selection: every KV head of a (sequence, layer) keeps the same
+ * tokens, and with the heads split over tensor-parallel ranks every rank
+ * evicts the identical set (hysenlabs write-up, decode-time section: the vLLM
+ * port's cross-rank eviction-score all-reduce; "every TP rank evicts the
+ * identical set").  The score of candidate i is the sum over all KV heads of
+ * the per-head joint scores, Zsum_i = sum_h Z_h[i]; the kept set is the top
+ * budget - window candidates of Zsum by (score desc, index asc) plus the
+ * window.  Two calls around the caller's all-reduce:
+ *
+ *   rkv_score_shared            per-head Z of this call's KV heads, summed
+ *                               over them into z_sum (the rank's part)
+ *   (caller)                    all-reduce (sum) of z_sum over the ranks
+ *   rkv_select_compact_shared   one select per (sequence, layer) on the
+ *                               complete z_sum; every head of this call is
+ *                               compacted in place with that set
+ *
+ * Arguments as rkv_compress_step; n_kv_heads / n_q_heads are this rank's
+ * heads.  z_sum: device [n_layers][batch][cap] fp32, 16-byte aligned; every
+ * entry is written (0 past the candidates and for sequences that are not
+ * due), so ranks reduce defined data.  Due sequences are those with
+ * cur_len >= budget + buffer; rkv_score_shared leaves cur_len unchanged and
+ * rkv_select_compact_shared sets it to the budget.  kept_out (optional):
+ * device [n_layers][batch][cap] int32, entries 0..budget-1 of every compressed
+ * (layer, sequence) get the kept rows in ascending order.  Both calls use one
+ * workspace of rkv_workspace_size_shared bytes (which also carries the
+ * per-head scores from the first call to nothing but itself; the second call
+ * needs only z_sum).  Caches up to about 6700 rows (one CTA per head);
+ * longer caches: RKV_ERR_UNSUPPORTED.
+ */
+RKV_API size_t rkv_workspace_size_shared(const rkv_config *cfg, int32_t n_layers, int32_t batch,
+                                         int32_t cap);
+
+RKV_API rkv_status rkv_score_shared(const rkv_config *cfg, int32_t n_layers, int32_t batch,
+                                    int32_t cap, const rkv_bf16 *const *k_layers,
+                                    const rkv_bf16 *const *q_layers, const int32_t *budgets,
+                                    const float *lambdas, const int32_t *cur_len, float *z_sum,
+                                    void *workspace, size_t ws_bytes, rkv_stream_t stream);
+
+RKV_API rkv_status rkv_select_compact_shared(const rkv_config *cfg, int32_t n_layers,
+                                             int32_t batch, int32_t cap, rkv_bf16 *const *k_layers,
+                                             rkv_bf16 *const *v_layers, const int32_t *budgets,
+                                             int32_t *cur_len, const float *z_sum,
+                                             int32_t *kept_out, void *workspace, size_t ws_bytes,
+                                             rkv_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

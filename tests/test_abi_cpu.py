@@ -140,3 +140,31 @@ def test_step_shape_query():
         rkv.rkv_query_step_shape(rkv.make_config(head_dim=64), 8, 1152)
     with pytest.raises(rkv.RkvError):
         rkv.rkv_query_step_shape(cfg, 0, 1152)
+
+
+def test_shared_selection_host_validation():
+    L = rkv._lib
+    c = rkv.make_config()
+    cfgp = ctypes.byref(c)
+    arr = ctypes.c_void_p * 2
+    k = arr(A, A + (1 << 30))
+    v = arr(A + (1 << 36), A + (1 << 36) + (1 << 30))
+    q = arr(A + (1 << 37), A + (1 << 37) + (1 << 20))
+    need = rkv.rkv_workspace_size_shared(c, 2, 1, 1152)
+    assert need > rkv.rkv_workspace_size(c, 2, 1, 1152)
+    ws, cur, z = A + (1 << 38), A + 7 * 4096, A + (1 << 39)
+    # score: missing q, z or workspace; workspace too small; misaligned z
+    assert L.rkv_score_shared(cfgp, 2, 1, 1152, k, None, None, None, cur, z, ws, need, None) == -1
+    assert L.rkv_score_shared(cfgp, 2, 1, 1152, k, q, None, None, cur, None, ws, need, None) == -1
+    assert L.rkv_score_shared(cfgp, 2, 1, 1152, k, q, None, None, cur, z, None, need, None) == -5
+    assert L.rkv_score_shared(cfgp, 2, 1, 1152, k, q, None, None, cur, z, ws, need - 256, None) == -5
+    assert L.rkv_score_shared(cfgp, 2, 1, 1152, k, q, None, None, cur, z + 4, ws, need, None) == -3
+    assert L.rkv_score_shared(ctypes.byref(rkv.make_config(buffer=0)), 2, 1, 1152, k, q, None,
+                              None, cur, z, ws, need, None) == 1
+    # select + compact: K overlapping V, caches too long for one CTA per head
+    vbad = arr(A + 4096, A + (1 << 36))
+    assert L.rkv_select_compact_shared(cfgp, 2, 1, 1152, k, vbad, None, cur, z, None, ws, need,
+                                       None) == -4
+    big = rkv.rkv_workspace_size_shared(c, 2, 1, 9000)
+    assert L.rkv_select_compact_shared(cfgp, 2, 1, 9000, k, v, None, cur, z, None, ws, big,
+                                       None) == -6
