@@ -194,7 +194,7 @@ __host__ __device__ inline UnitLayout make_unit_layout(int nmax, int nqp) {
     L.colf = o;   o += 256u;
     L.vis = o;    o += 512u;
     L.red = o;    o += 256u;
-    L.bars = o;   o += 64u;
+    L.bars = o;   o += 128u;
     L.total = o + 1024u;
     return L;
 }

@@ -45,6 +45,11 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                  : "memory");
 }
 
+// One plain arrival (no transaction bytes).
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // One probe of phase `parity`; while it is incomplete the thread may sleep in
 // hardware for up to kSuspendHintNs instead of spinning on issue slots.
 constexpr uint32_t kSuspendHintNs = 1000000u;
@@ -95,6 +100,11 @@ __device__ __forceinline__ void bulk_g2s(void *smem_dst, const void *gsrc, uint3
             "r"(smem_u32(smem_dst)),
         "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
+}
+
+// Hint: bring `bytes` (multiple of 16, 16-aligned) of global memory into L2.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *gsrc, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gsrc), "r"(bytes) : "memory");
 }
 
 // ---------------------------------------------------------------- tcgen05

@@ -28,8 +28,9 @@
 //     similarity kernel (MAX).
 //   then the normalisers, the joint scores, the radix select and the
 //   destinations of the kept rows, and the in-place compaction in ascending
-//   chunks of 128 rows (every source row of a chunk is read before any row of
-//   it is written; later chunks only read rows above the current chunk).
+//   chunks of 64 rows (every source row of a chunk is read before any row of
+//   it is written; later chunks only read rows above the current chunk, so the
+//   next chunk's reads overlap this chunk's writes).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -50,7 +51,7 @@ namespace {
 constexpr int kTileRows = 128;
 constexpr uint32_t kStageBytes = 32768u;
 constexpr uint32_t kHalfBytes = 16384u;
-constexpr int kChunkRows = 128;          // compaction chunk
+constexpr int kChunkRows = 64;           // compaction chunk (two in flight)
 constexpr float kRescaleLog2 = 8.0f;     // online softmax: rescale past 2^8
 
 // Merges (m2, s2) into (m, s): s = sum of 2^(x - m) over the values seen.
@@ -151,8 +152,11 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
     uint64_t *sVis = reinterpret_cast<uint64_t *>(base + L.vis);
     float *sRed = reinterpret_cast<float *>(base + L.red);
     uint32_t *sRedU = reinterpret_cast<uint32_t *>(base + L.red);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(base + L.bars);   // full[2], mma[2], smma[2]
+    // full[2] (TMA), mma[2] (logits UMMA), smma[2] (S UMMA); then the TMEM base and
+    // the per-stage count of warps whose S-UMMA operand is written
+    uint64_t *bars = reinterpret_cast<uint64_t *>(base + L.bars);
     uint32_t *sTmem = reinterpret_cast<uint32_t *>(bars + 6);
+    uint32_t *sBsCount = sTmem + 2;
     // after the last tile the ring holds the keys, the destinations and the histograms
     const uint32_t arr = align_up(static_cast<uint32_t>(p.nmax) * 4u, 16);
     uint32_t *sKeys = reinterpret_cast<uint32_t *>(sStage);
@@ -175,6 +179,7 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
     }
     if (tid == 32) {
         for (int i = 0; i < 6; ++i) mbar_init(&bars[i], 1);
+        sBsCount[0] = sBsCount[1] = 0;
         fence_mbar_init();
     }
     // B operand rows past the queries start as zeros (the split S lands in three of
@@ -203,7 +208,7 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
     const uint32_t scol = static_cast<uint32_t>(2 * SLOT);   // S accumulator columns
 
     // last tile / logits UMMA / S UMMA issued (thread 0's copies), for the error path
-    int tma_last = 1, mma_last = -1, smma_last = -1;
+    int tma_last = 1, mma_last = -1;
     const CUtensorMap *mk = &p.tmap_k[l];
     auto issue_tile = [&](int g) {   // global tile g: pass 1 for g < T, pass 2 after
         tma_last = g;
@@ -250,12 +255,15 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
     const int nrow = (lane & 7) + 8 * (lane >> 4), nhalf = (lane >> 3) & 1;
     const int row_t = 16 * warp + nrow;        // this lane's tile row in the norms
 
-    float cm[HC], cs[HC];
+    // pass-1 column pairs of this warpgroup's HC columns, two columns per float2:
+    // ncm = -(running reference), cs = sum of 2^(x - reference)
+    float2 ncm[HC / 2], cs[HC / 2];
 #pragma unroll
-    for (int c = 0; c < HC; ++c) {
-        cm[c] = -INFINITY;
-        cs[c] = 0.f;
+    for (int c = 0; c < HC / 2; ++c) {
+        ncm[c] = make_float2(INFINITY, INFINITY);
+        cs[c] = make_float2(0.f, 0.f);
     }
+    const float2 sc2 = make_float2(p.logit_scale_log2, p.logit_scale_log2);
     bool ok = true;
     int g = 0;
     for (; g < 2 * T; ++g) {
@@ -318,9 +326,19 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
                             make_uint4(0u, 0u, 0u, 0u);
                     }
                 }
+                // each warp's S-operand (and tail) writes, then a count: the warp that
+                // completes it issues the S UMMA, so no warp waits for the others here
                 fence_proxy_async_smem();
-                __syncthreads();
-                if (tid == 0 && wait_ok) {
+                __syncwarp();
+                uint32_t last = 0;
+                if (lane == 0) {
+                    __threadfence_block();
+                    last = atomicAdd(&sBsCount[s], 1u) == NW - 1 ? 1u : 0u;
+                }
+                last = __shfl_sync(kFull, last, 0);
+                if (last && lane == 0) {
+                    __threadfence_block();
+                    sBsCount[s] = 0;   // the stage's next pass-1 tile counts from zero
                     // S += K_tile^T . inv: A = the K tile read MN-major (M = 128 columns,
                     // 64-column blocks 16 KB apart, 8-row groups 1 KB apart), B = inv split
                     tc_fence_after();
@@ -333,7 +351,6 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
                         umma_bf16(tmem_base + scol, ad, bd, idesc_s, (g > 0 || ks > 0) ? 1u : 0u);
                     }
                     umma_commit(&smma[s]);
-                    smma_last = g;
                 }
             }
         } else if (g == T) {
@@ -343,9 +360,11 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
             for (int c0 = 0; c0 < HC; c0 += 8) {
                 float m8[8], s8[8];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    m8[j] = cm[c0 + j];
-                    s8[j] = cs[c0 + j];
+                for (int j = 0; j < 8; j += 2) {
+                    m8[j] = -ncm[(c0 + j) / 2].x;
+                    m8[j + 1] = -ncm[(c0 + j) / 2].y;
+                    s8[j] = cs[(c0 + j) / 2].x;
+                    s8[j + 1] = cs[(c0 + j) / 2].y;
                 }
                 warp_fold8_ms(m8, s8);
                 if (lane < 8) {
@@ -381,7 +400,7 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
 #pragma unroll
                 for (int k = 1; k < 4; ++k)
                     ms_merge(m, sm, xm[((gq * 4 + k) * HC + c) * 2], xm[((gq * 4 + k) * HC + c) * 2 + 1]);
-                sColM[q] = m;
+                sColM[q] = -m;   // negated: pass 2 adds it
                 sColF[q] = sm > 0.f ? 1.0f / sm : 0.f;
             }
             fence_proxy_async_smem();
@@ -399,39 +418,73 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
             // ---- pass 1: fold this row's logits into the running column pairs
             const uint64_t rmask = i < M ? colmask : (i < N ? sVis[i - M] : 0ull);
             const bool all_cand = __all_sync(kFull, i < M);
-            uint32_t raw[HC / 8][8];
+            // up to 16 columns: all loads in flight at once; more: one 8-column load at a time
+            constexpr int NB = HC <= 16 ? HC / 8 : 1;
+            uint32_t raw[NB][8];
+            if (HC <= 16) {
 #pragma unroll
-            for (int c0 = 0; c0 < HC; c0 += 8)
-                tmem_ld8_nowait(tmem_lane + tslot + static_cast<uint32_t>(wg * HC + c0), raw[c0 / 8]);
-            tmem_wait_ld();
+                for (int c0 = 0; c0 < HC; c0 += 8)
+                    tmem_ld8_nowait(tmem_lane + tslot + static_cast<uint32_t>(wg * HC + c0), raw[(c0 / 8) % NB]);
+                tmem_wait_ld();
 #pragma unroll
-            for (int c0 = 0; c0 < HC; c0 += 8) reg_tie8(raw[c0 / 8]);
+                for (int c0 = 0; c0 < HC; c0 += 8) reg_tie8(raw[(c0 / 8) % NB]);
+            }
 #pragma unroll
             for (int c0 = 0; c0 < HC; c0 += 8) {
                 const int q0 = wg * HC + c0;
-                float x[8];
-                bool vis[8];
+                if (HC > 16) {
+                    tmem_ld8_nowait(tmem_lane + tslot + static_cast<uint32_t>(q0), raw[0]);
+                    tmem_wait_ld();
+                    reg_tie8(raw[0]);
+                }
+                const bool allv = all_cand && q0 + 8 <= NQ;   // warp-uniform
+                float2 x[4], d[4];
                 bool big = false;
 #pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    x[j] = __fmul2_rn(make_float2(__uint_as_float(raw[(c0 / 8) % NB][2 * j]),
+                                                  __uint_as_float(raw[(c0 / 8) % NB][2 * j + 1])), sc2);
+                    d[j] = __fadd2_rn(x[j], ncm[c0 / 2 + j]);   // x - reference
+                }
+                if (allv) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) big |= (d[j].x > kRescaleLog2) | (d[j].y > kRescaleLog2);
+                    if (!__any_sync(kFull, big)) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            cs[c0 / 2 + j] = __fadd2_rn(cs[c0 / 2 + j],
+                                                        make_float2(ex2_approx(d[j].x), ex2_approx(d[j].y)));
+                        continue;
+                    }
+                }
+                // masked columns or rows, or a logit past the rescale margin
+                bool vis[8];
+                big = false;
+#pragma unroll
                 for (int j = 0; j < 8; ++j) {
-                    x[j] = __uint_as_float(raw[c0 / 8][j]) * sc;
-                    vis[j] = (all_cand && q0 + 8 <= NQ) ? true : (((rmask >> (q0 + j)) & 1ull) != 0);
-                    big |= vis[j] && (x[j] > cm[c0 + j] + kRescaleLog2);
+                    vis[j] = allv || (((rmask >> (q0 + j)) & 1ull) != 0);
+                    const float dj = (j & 1) ? d[j / 2].y : d[j / 2].x;
+                    big |= vis[j] && (dj > kRescaleLog2);
                 }
                 if (__any_sync(kFull, big)) {
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         if (vis[j]) {
-                            const float mn = fmaxf(cm[c0 + j], x[j]);
-                            cs[c0 + j] = cs[c0 + j] * ex2_approx(cm[c0 + j] - mn) + ex2_approx(x[j] - mn);
-                            cm[c0 + j] = mn;
+                            float &nm = (j & 1) ? ncm[(c0 + j) / 2].y : ncm[(c0 + j) / 2].x;
+                            float &sj = (j & 1) ? cs[(c0 + j) / 2].y : cs[(c0 + j) / 2].x;
+                            const float xj = (j & 1) ? x[j / 2].y : x[j / 2].x;
+                            const float mn = fmaxf(-nm, xj);
+                            sj = sj * ex2_approx(-nm - mn) + ex2_approx(xj - mn);
+                            nm = -mn;
                         }
                     }
                 } else {
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
-                        const float e = ex2_approx(x[j] - cm[c0 + j]);
-                        cs[c0 + j] += vis[j] ? e : 0.f;
+                        const float dj = (j & 1) ? d[j / 2].y : d[j / 2].x;
+                        float &sj = (j & 1) ? cs[(c0 + j) / 2].y : cs[(c0 + j) / 2].x;
+                        const float e = ex2_approx(dj);
+                        sj += vis[j] ? e : 0.f;
                     }
                 }
             }
@@ -456,12 +509,24 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
                     for (int k = 0; k < MAXH; ++k) {
                         if (k < nh) {
                             const int q0 = (h0 + k) * 8;
-                            float run = 0.f;
+                            const float4 *nm4 = reinterpret_cast<const float4 *>(sColM + q0);
+                            const float4 *f4 = reinterpret_cast<const float4 *>(sColF + q0);
+                            float2 run2 = make_float2(0.f, 0.f);
 #pragma unroll
-                            for (int j = 0; j < 8; ++j)
-                                run = fmaf(ex2_approx(fmaf(__uint_as_float(raw[k][j]), sc, -sColM[q0 + j])),
-                                           sColF[q0 + j], run);
-                            const float a = run * inv_w;
+                            for (int j = 0; j < 2; ++j) {
+                                const float4 nm = nm4[j], f = f4[j];
+                                const float2 a0 = __ffma2_rn(make_float2(__uint_as_float(raw[k][4 * j]),
+                                                                         __uint_as_float(raw[k][4 * j + 1])),
+                                                             sc2, make_float2(nm.x, nm.y));
+                                const float2 a1 = __ffma2_rn(make_float2(__uint_as_float(raw[k][4 * j + 2]),
+                                                                         __uint_as_float(raw[k][4 * j + 3])),
+                                                             sc2, make_float2(nm.z, nm.w));
+                                run2 = __ffma2_rn(make_float2(ex2_approx(a0.x), ex2_approx(a0.y)),
+                                                  make_float2(f.x, f.y), run2);
+                                run2 = __ffma2_rn(make_float2(ex2_approx(a1.x), ex2_approx(a1.y)),
+                                                  make_float2(f.z, f.w), run2);
+                            }
+                            const float a = (run2.x + run2.y) * inv_w;
                             pool = pool_max ? fmaxf(pool, a) : pool + a;
                         }
                     }
@@ -477,7 +542,7 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
 #pragma unroll
                     for (int q = 0; q < NQP; ++q) {
                         if (q < NQ) {
-                            run = fmaf(ex2_approx(fmaf(__uint_as_float(raw[q / 8][q % 8]), sc, -sColM[q])),
+                            run = fmaf(ex2_approx(fmaf(__uint_as_float(raw[q / 8][q % 8]), sc, sColM[q])),
                                        sColF[q], run);
                             if ((lastmask >> q) & 1ull) {
                                 const float a = run * inv_w;
@@ -511,7 +576,7 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
             }
         }
         tc_fence_before();
-        if (__syncthreads_or(!wait_ok)) {
+        if (__syncthreads_or(!wait_ok || !ok)) {
             ok = false;
             break;
         }
@@ -534,11 +599,9 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
                     ok = false;
             }
         }
-        if (__syncthreads_or(!ok)) {
-            ok = false;
-            break;
-        }
     }
+    // a wait of thread 0 after the last barrier of the loop
+    if (__syncthreads_or(!ok)) ok = false;
 
     if (!ok) {
         // A wait ran out: record it, wait (bounded) for this CTA's copies and
@@ -549,8 +612,8 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
                 (void)mbar_wait(&full[gg & 1], static_cast<uint32_t>((gg >> 1) & 1));
             for (int gg = g; gg <= mma_last; ++gg)
                 (void)mbar_wait(&mmab[gg & 1], static_cast<uint32_t>((gg >> 1) & 1));
-            for (int gg = g; gg <= smma_last; ++gg)
-                (void)mbar_wait(&smma[gg & 1], static_cast<uint32_t>((gg >> 1) & 1));
+            // the S UMMA of a pass-1 tile may come from any warp: wait for this one's
+            if (g < T && !red_max) (void)mbar_wait(&smma[g & 1], static_cast<uint32_t>((g >> 1) & 1));
         }
         __syncthreads();
         if (warp == 0) {
@@ -558,6 +621,15 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
             tmem_dealloc(tmem_base, static_cast<uint32_t>(p.tmem_cols));
         }
         return;
+    }
+
+    // The compaction reads most of the unit's V rows: start bringing them into L2
+    // now, while the select runs (HBM is otherwise idle in this phase).
+    if (tid == 32 && p.v[l] != nullptr && !p.z_heads) {
+        const uint8_t *vrow = reinterpret_cast<const uint8_t *>(p.v[l] + krow0 * kHeadDim);
+        const uint32_t total = static_cast<uint32_t>(N) * 256u;
+        for (uint32_t off = 0; off < total; off += 65536u)
+            bulk_prefetch_l2(vrow + off, min(65536u, total - off));
     }
 
     // ---- normalisers, keys and the select (one per unit)
@@ -596,21 +668,46 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
     // kept = above || window || (tied && E_i < need_eq), dst = G_i + min(E_i, need_eq)
     const int need_eq = (kk > 0) ? kk - n_gt : 0;
     {
-        uint32_t g_run = 0, e_run = 0;
-        for (int c0 = 0; c0 < N; c0 += NT) {
-            const int row = c0 + tid;
-            const bool in = row < N;
+        // warp w owns rows [w*seg, w*seg + seg): count, one block exchange of the
+        // eight warp totals, then each warp walks its rows 32 at a time with ballots
+        const int seg = ((N + NW - 1) / NW + 31) / 32 * 32;
+        const int r0 = warp * seg, r1 = min(N, r0 + seg);
+        const uint32_t lt = (1u << lane) - 1u;
+        auto flags = [&](int row, bool &eq, bool &gw) {
+            const bool in = row < r1;
             const bool cand = row < M;
-            const uint32_t key = cand ? sKeys[row] : 0u;
-            const bool eq = cand && kk > 0 && key == Tk;
-            const bool gw = in && (!cand || (kk > 0 && key > Tk));
-            uint32_t tot2;
-            const uint32_t ex = block_excl_scan_u32<NT>((eq ? 65536u : 0u) + (gw ? 1u : 0u), sRedU, tot2);
-            const uint32_t Ei = e_run + (ex >> 16), Gi = g_run + (ex & 0xffffu);
+            const uint32_t key = (in && cand) ? sKeys[row] : 0u;
+            eq = in && cand && kk > 0 && key == Tk;
+            gw = in && (!cand || (kk > 0 && key > Tk));
+        };
+        uint32_t ng = 0, ne = 0;
+        for (int rb = r0; rb < r1; rb += 32) {
+            bool eq, gw;
+            flags(rb + lane, eq, gw);
+            ng += __popc(__ballot_sync(kFull, gw));
+            ne += __popc(__ballot_sync(kFull, eq));
+        }
+        if (lane == 0) {
+            sRedU[warp] = ng;
+            sRedU[NW + warp] = ne;
+        }
+        __syncthreads();
+        uint32_t g_run = 0, e_run = 0;
+        for (int w2 = 0; w2 < warp; ++w2) {
+            g_run += sRedU[w2];
+            e_run += sRedU[NW + w2];
+        }
+        for (int rb = r0; rb < r1; rb += 32) {
+            bool eq, gw;
+            const int row = rb + lane;
+            flags(row, eq, gw);
+            const uint32_t bg = __ballot_sync(kFull, gw), be = __ballot_sync(kFull, eq);
+            const uint32_t Gi = g_run + __popc(bg & lt), Ei = e_run + __popc(be & lt);
             const bool kept = gw || (eq && Ei < static_cast<uint32_t>(need_eq));
-            if (in) sDst[row] = kept ? static_cast<int32_t>(Gi + min(Ei, static_cast<uint32_t>(need_eq))) : -1;
-            e_run += tot2 >> 16;
-            g_run += tot2 & 0xffffu;
+            if (row < r1)
+                sDst[row] = kept ? static_cast<int32_t>(Gi + min(Ei, static_cast<uint32_t>(need_eq))) : -1;
+            g_run += __popc(bg);
+            e_run += __popc(be);
         }
     }
     __syncthreads();
@@ -648,10 +745,11 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
         for (int k = 1; k < NW; ++k) first = min(first, sRedU[k]);
         uint16_t *kb = p.k[l] + krow0 * kHeadDim;
         uint16_t *vb = p.v[l] + krow0 * kHeadDim;
+        // Software-pipelined: chunk c + 1 is read before chunk c is written.  Its
+        // rows lie above every destination of chunk c, and every read of chunk c
+        // precedes the barrier before chunk c's writes.
         constexpr int PER = kChunkRows * 16 / NT;   // 16-byte pieces per thread per chunk
-        for (int c0 = static_cast<int>(first); c0 < N; c0 += kChunkRows) {
-            uint4 kx[PER], vx[PER];
-            int dd[PER];
+        auto load = [&](int c0, uint4 (&kx)[PER], uint4 (&vx)[PER], int (&dd)[PER]) {
 #pragma unroll
             for (int k = 0; k < PER; ++k) {
                 const int idx = tid + k * NT;
@@ -663,7 +761,8 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
                     vx[k] = __ldcg(reinterpret_cast<const uint4 *>(vb + static_cast<int64_t>(row) * kHeadDim) + pc);
                 }
             }
-            __syncthreads();
+        };
+        auto store = [&](const uint4 (&kx)[PER], const uint4 (&vx)[PER], const int (&dd)[PER]) {
 #pragma unroll
             for (int k = 0; k < PER; ++k) {
                 if (dd[k] >= 0) {
@@ -672,6 +771,22 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
                     reinterpret_cast<uint4 *>(vb + static_cast<int64_t>(dd[k]) * kHeadDim)[pc] = vx[k];
                 }
             }
+        };
+        uint4 ka[PER], va[PER], kc[PER], vc[PER];
+        int da[PER], dc[PER];
+        int c0 = static_cast<int>(first);
+        if (c0 < N) load(c0, ka, va, da);
+        while (c0 < N) {
+            const int c1 = c0 + kChunkRows;
+            if (c1 < N) load(c1, kc, vc, dc);
+            __syncthreads();
+            store(ka, va, da);
+            if (c1 >= N) break;
+            const int c2 = c1 + kChunkRows;
+            if (c2 < N) load(c2, ka, va, da);
+            __syncthreads();
+            store(kc, vc, dc);
+            c0 = c2;
         }
     }
 

@@ -118,3 +118,26 @@ def unit(q_bits, k_bits, N, budget, lam, red_mode=RED_MEAN, pool=POOL_MAX):
     Z = joint(I, R, lam)
     kept = select(Z, N, budget)
     return {"I": I, "r": r, "R": R, "Z": Z, "kept": kept}
+
+
+# ---------------------------------------------------------------- paged caches
+# A paged cache keeps each layer's keys (and values) in a pool of fixed-size
+# pages, pool[page, head, slot, :], and each sequence owns a list of pages
+# (its block table): logical row i of a sequence lives in page
+# block_table[i // P] at slot i % P.  Compressing a sequence to `budget` rows
+# leaves its pages ceil(budget / P) .. ceil(N / P) - 1 empty, and they go back
+# to the allocator -- the FREE_BLOCKS return path of the vLLM port (hysenlabs
+# write-up, decode-time section: physical eviction returns freed blocks).
+
+def paged_rows(pool_bits, block_table_row, h, n_rows, page_rows):
+    """Logical rows 0..n_rows-1 of KV head h, gathered through the block table."""
+    pool = np.asarray(pool_bits)
+    bt = np.asarray(block_table_row)
+    return np.stack([pool[bt[i // page_rows], h, i % page_rows] for i in range(n_rows)])
+
+
+def freed_pages(block_table_row, n_tokens, budget, page_rows):
+    """Pages a sequence no longer needs after compaction from n_tokens to budget rows."""
+    keep = -(-budget // page_rows)
+    used = -(-n_tokens // page_rows)
+    return [int(x) for x in np.asarray(block_table_row)[keep:used]]
