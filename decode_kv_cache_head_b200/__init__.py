@@ -22,6 +22,7 @@ __all__ = [
     "rkv_score_importance", "rkv_score_redundancy", "rkv_select_topk", "rkv_compact_kv",
     "rkv_compress_step", "rkv_append_kv",
     "rkv_workspace_size_shared", "rkv_score_shared", "rkv_select_compact_shared",
+    "rkv_paged_kv", "rkv_compress_step_paged",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -44,6 +45,17 @@ class rkv_config(ctypes.Structure):
         ("mix_lambda", ctypes.c_float),
         ("redundancy_mode", ctypes.c_int32),
         ("gqa_pool", ctypes.c_int32),
+    ]
+
+
+class rkv_paged_kv(ctypes.Structure):
+    _fields_ = [
+        ("block_table", ctypes.c_void_p),
+        ("max_blocks", ctypes.c_int32),
+        ("page_rows", ctypes.c_int32),
+        ("num_pages", ctypes.c_int32),
+        ("freed_pages", ctypes.c_void_p),
+        ("n_freed", ctypes.c_void_p),
     ]
 
 
@@ -83,6 +95,9 @@ def _load() -> ctypes.CDLL:
                                              ctypes.POINTER(rkv_step_options), P, SZ, P]),
         "rkv_append_kv": (ctypes.c_int, [CFG, I32, I32, I32, P, P, P, P, I32, P, P, SZ, P]),
         "rkv_workspace_size_shared": (SZ, [CFG, I32, I32, I32]),
+        "rkv_compress_step_paged": (ctypes.c_int, [CFG, I32, I32, ctypes.POINTER(rkv_paged_kv), P,
+                                                   P, P, P, P, P, ctypes.POINTER(rkv_step_options),
+                                                   P, SZ, P]),
         "rkv_score_shared": (ctypes.c_int, [CFG, I32, I32, I32, P, P, P, P, P, P, P, SZ, P]),
         "rkv_select_compact_shared": (ctypes.c_int, [CFG, I32, I32, I32, P, P, P, P, P, P, P, SZ,
                                                      P]),
@@ -307,3 +322,39 @@ def rkv_select_compact_shared(cfg, k_layers, v_layers, cur_len, z_sum, workspace
                                                  _ptr(kept_out), _ptr(workspace), ws,
                                                  _stream(stream)),
                   "rkv_select_compact_shared", allow_disabled=True)
+
+
+def rkv_compress_step_paged(cfg, k_pools, v_pools, q_layers, cur_len, workspace, block_table,
+                            page_rows, freed_pages, n_freed, budgets=None, lambdas=None,
+                            kept_out=None, scores_out=None, events=None, stream=None):
+    """The step on paged caches, in place.
+
+    k_pools / v_pools: per layer [num_pages, Hkv, page_rows, 128] bf16 (or one
+    [n_layers, ...] tensor); block_table [batch, max_blocks] int32 (logical page
+    j of sequence b); freed_pages [batch, max_blocks] / n_freed [batch] int32
+    receive the pages each compressed sequence gives back.  kept_out /
+    scores_out as in rkv_compress_step with cap = max_blocks * page_rows.
+    """
+    k_pools, v_pools, q_layers = list(k_pools), list(v_pools), list(q_layers)
+    num_pages = k_pools[0].shape[0]
+    batch, max_blocks = block_table.shape
+    for t in k_pools + v_pools + q_layers:
+        _dtype(t, torch.bfloat16, "k/v/q")
+    for t, n in ((cur_len, "cur_len"), (budgets, "budgets"), (block_table, "block_table"),
+                 (freed_pages, "freed_pages"), (n_freed, "n_freed"), (kept_out, "kept_out")):
+        _dtype(t, torch.int32, n)
+    _dtype(lambdas, torch.float32, "lambdas"); _dtype(scores_out, torch.float32, "scores_out")
+    pg = rkv_paged_kv(_ptr(block_table), int(max_blocks), int(page_rows), int(num_pages),
+                      _ptr(freed_pages), _ptr(n_freed))
+    opts = rkv_step_options(_ptr(kept_out), _ptr(scores_out), None, None, 0)
+    if events is not None:
+        opts.main_begin = events[0].cuda_event
+        opts.main_end = events[1].cuda_event
+    ws = workspace.numel() * workspace.element_size()
+    return _check(_lib.rkv_compress_step_paged(ctypes.byref(cfg), len(k_pools), batch,
+                                               ctypes.byref(pg), _ptr_array(k_pools),
+                                               _ptr_array(v_pools), _ptr_array(q_layers),
+                                               _ptr(budgets), _ptr(lambdas), _ptr(cur_len),
+                                               ctypes.byref(opts), _ptr(workspace), ws,
+                                               _stream(stream)),
+                  "rkv_compress_step_paged", allow_disabled=True)

@@ -158,6 +158,12 @@ bool use_unit_kernel(int64_t n_units, int cap, int nqp, int cs_req) {
     return n_units >= kB200SMs && unit_shape(cap, nqp).ok;
 }
 
+// Paged caches: the page pools' geometry and the block table (null: contiguous).
+struct PagedArgs {
+    const int32_t *block_table;
+    int32_t max_blocks, page_rows, num_pages;
+};
+
 // The one-CTA-per-unit kernel over all layers, 32 per launch.  z_heads != null:
 // scores only (shared selection), no cache writes.
 cudaError_t launch_unit_layers(const rkv_config *cfg, int32_t n_layers, int32_t batch, int32_t cap,
@@ -165,7 +171,8 @@ cudaError_t launch_unit_layers(const rkv_config *cfg, int32_t n_layers, int32_t 
                                const rkv_bf16 *const *q_layers, const int32_t *budgets,
                                const float *lambdas, const int32_t *n_eff, const float *r_ext,
                                int32_t *kept_out, float *scores_out, float *z_heads,
-                               uint32_t *status, const UnitShape &us, int nqp, cudaStream_t strm) {
+                               uint32_t *status, const UnitShape &us, int nqp, cudaStream_t strm,
+                               const PagedArgs &pg = PagedArgs{nullptr, 0, 0, 0}) {
     UnitParams *up = new UnitParams();
     std::memset(up, 0, sizeof(*up));
     up->batch = batch;
@@ -188,15 +195,21 @@ cudaError_t launch_unit_layers(const rkv_config *cfg, int32_t n_layers, int32_t 
     up->kept_out = kept_out;
     up->scores_out = scores_out;
     up->z_heads = z_heads;
+    up->block_table = pg.block_table;
+    up->max_blocks = pg.max_blocks;
+    up->page_rows = pg.page_rows;
     up->status = status;
+    const uint64_t k_rows = pg.block_table
+                                ? static_cast<uint64_t>(pg.num_pages) * cfg->n_kv_heads * pg.page_rows
+                                : static_cast<uint64_t>(batch) * cfg->n_kv_heads * cap;
+    const uint32_t k_box = pg.block_table ? static_cast<uint32_t>(pg.page_rows) : 128u;
     cudaError_t e = cudaSuccess;
     for (int l0 = 0; e == cudaSuccess && l0 < n_layers; l0 += kMaxLayersPerLaunch) {
         const int nl = (n_layers - l0 < kMaxLayersPerLaunch) ? n_layers - l0 : kMaxLayersPerLaunch;
         up->layer_base = l0;
         for (int i = 0; i < nl; ++i) {
             const int l = l0 + i;
-            if (!encode_rows128(&up->tmap_k[i], k_layers[l],
-                                static_cast<uint64_t>(batch) * cfg->n_kv_heads * cap, 128) ||
+            if (!encode_rows128(&up->tmap_k[i], k_layers[l], k_rows, k_box) ||
                 !encode_rows128(&up->tmap_q[i], q_layers[l],
                                 static_cast<uint64_t>(batch) * cfg->n_q_heads * cfg->window,
                                 static_cast<uint32_t>(nqp))) {
@@ -779,6 +792,66 @@ rkv_status rkv_select_compact_shared(const rkv_config *cfg, int32_t n_layers, in
         e = launch_shared_select(sp, nl * batch, strm);
         if (e == cudaSuccess) e = launch_shared_compact(sp, nl * batch * cfg->n_kv_heads, strm);
     }
+    return cuda_status(e);
+}
+
+rkv_status rkv_compress_step_paged(const rkv_config *cfg, int32_t n_layers, int32_t batch,
+                                   const rkv_paged_kv *pg, rkv_bf16 *const *k_pools,
+                                   rkv_bf16 *const *v_pools, const rkv_bf16 *const *q_layers,
+                                   const int32_t *budgets, const float *lambdas, int32_t *cur_len,
+                                   const rkv_step_options *opts, void *workspace, size_t ws_bytes,
+                                   rkv_stream_t stream) {
+    rkv_status st = check_cfg(cfg);
+    if (st != RKV_OK) return st;
+    if (cfg->buffer <= 0 || (!budgets && cfg->budget <= 0)) return RKV_STATUS_DISABLED;
+    if (!pg || !k_pools || !v_pools || !q_layers || !cur_len) return RKV_ERR_NULL;
+    if (!pg->block_table || !pg->freed_pages || !pg->n_freed) return RKV_ERR_NULL;
+    if (!workspace) return RKV_ERR_WORKSPACE;
+    const int P = pg->page_rows;
+    if (P != 16 && P != 32 && P != 64 && P != 128) return RKV_ERR_UNSUPPORTED;
+    if (n_layers < 1 || batch < 1 || pg->max_blocks < 1 || pg->num_pages < 1) return RKV_ERR_INVALID;
+    if (cfg->redundancy_mode != RKV_RED_MEAN) return RKV_ERR_UNSUPPORTED;
+    if (opts && opts->cluster_size != 0 && opts->cluster_size != 1) return RKV_ERR_UNSUPPORTED;
+    const int64_t cap64 = static_cast<int64_t>(pg->max_blocks) * P;
+    if (cap64 > kUnitMaxPages * static_cast<int64_t>(P) ||
+        static_cast<int64_t>(pg->num_pages) * cfg->n_kv_heads * P > INT32_MAX)
+        return RKV_ERR_UNSUPPORTED;
+    const int cap = static_cast<int>(cap64);
+    if (!budgets && (cfg->budget < cfg->window || cfg->budget >= cap)) return RKV_ERR_INVALID;
+    const int nqp = nqp_of((cfg->n_q_heads / cfg->n_kv_heads) * cfg->window);
+    const UnitShape us = unit_shape(cap, nqp);
+    if (!us.ok) return RKV_ERR_UNSUPPORTED;
+    const size_t pool_bytes = static_cast<size_t>(pg->num_pages) * cfg->n_kv_heads * P * kHeadDim * 2;
+    for (int l = 0; l < n_layers; ++l) {
+        if (!k_pools[l] || !v_pools[l] || !q_layers[l]) return RKV_ERR_NULL;
+        if (!aligned16(k_pools[l]) || !aligned16(v_pools[l]) || !aligned16(q_layers[l]))
+            return RKV_ERR_ALIGN;
+        if (overlap(k_pools[l], pool_bytes, v_pools[l], pool_bytes)) return RKV_ERR_ALIAS;
+    }
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return RKV_ERR_ALIGN;
+    if (ws_bytes < ws_bytes_for(cfg, n_layers, batch, cap)) return RKV_ERR_WORKSPACE;
+
+    cudaStream_t strm = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    uint32_t *status = reinterpret_cast<uint32_t *>(ws);
+    int32_t *n_eff = reinterpret_cast<int32_t *>(ws + kStatusBytes);
+    cudaError_t e = cudaMemsetAsync(ws, 0, kStatusBytes, strm);
+    if (e == cudaSuccess)
+        e = launch_plan(batch, budgets, cfg->budget, cfg->buffer, cfg->window, cap, cur_len, n_eff,
+                        status, strm, true);
+    if (e == cudaSuccess)
+        e = launch_freed_pages(batch, budgets, cfg->budget, n_eff, pg->block_table, pg->max_blocks,
+                               P, pg->freed_pages, pg->n_freed, strm);
+    if (e == cudaSuccess && opts && opts->main_begin)
+        e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->main_begin), strm);
+    if (e == cudaSuccess)
+        e = launch_unit_layers(cfg, n_layers, batch, cap,
+                               const_cast<const rkv_bf16 *const *>(k_pools), v_pools, q_layers,
+                               budgets, lambdas, n_eff, nullptr, opts ? opts->kept_out : nullptr,
+                               opts ? opts->scores_out : nullptr, nullptr, status, us, nqp, strm,
+                               PagedArgs{pg->block_table, pg->max_blocks, P, pg->num_pages});
+    if (e == cudaSuccess && opts && opts->main_end)
+        e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->main_end), strm);
     return cuda_status(e);
 }
 

@@ -160,14 +160,19 @@ struct alignas(64) UnitParams {
     float *scores_out;
     float *z_heads;        // shared selection: Z of every candidate [units][cap]; then no
                            // select, no compaction
+    // paged caches: k / v are page pools [pages][Hkv][page_rows][128], tmap_k boxes are
+    // one page; logical row i of sequence b is in page block_table[b][i / page_rows]
+    const int32_t *block_table;   // [batch][max_blocks] or null (contiguous caches)
+    int32_t max_blocks, page_rows;
     uint32_t *status;
 };
 
 constexpr int kUnitThreads = 256;
+constexpr int kUnitMaxPages = 512;     // pages of one sequence staged in shared memory
 constexpr int kUnitMaxRows = 7680;     // keys + destinations + histograms fit the 64 KB ring
 
 struct UnitLayout {
-    uint32_t stage, b, bs, inv, self, ia, ib, r, scr, s, colm, colf, vis, red, bars, total;
+    uint32_t stage, b, bs, inv, self, ia, ib, r, scr, s, colm, colf, vis, red, bt, bars, total;
 };
 
 // Offsets from a 1024-byte-aligned base.  Lifetimes share bytes: the two 32 KB
@@ -194,6 +199,7 @@ __host__ __device__ inline UnitLayout make_unit_layout(int nmax, int nqp) {
     L.colf = o;   o += 256u;
     L.vis = o;    o += 512u;
     L.red = o;    o += 256u;
+    L.bt = o;     o += 4u * kUnitMaxPages;             // the sequence's page list (paged caches)
     L.bars = o;   o += 128u;
     L.total = o + 1024u;
     return L;
@@ -220,6 +226,11 @@ cudaError_t launch_head_sum(const SharedParams &p, int n_lb, cudaStream_t stream
 cudaError_t launch_shared_select(const SharedParams &p, int n_lb, cudaStream_t stream);
 cudaError_t launch_shared_compact(const SharedParams &p, int n_units, cudaStream_t stream);
 size_t shared_select_smem(int cap);
+
+cudaError_t launch_freed_pages(int batch, const int32_t *budgets, int32_t budget_cfg,
+                               const int32_t *n_eff, const int32_t *block_table, int max_blocks,
+                               int page_rows, int32_t *freed, int32_t *n_freed,
+                               cudaStream_t stream);
 
 // MAX-mode similarity kernel: raw r of every candidate of every due unit.
 struct alignas(64) GramParams {

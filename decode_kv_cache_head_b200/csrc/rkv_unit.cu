@@ -38,6 +38,7 @@
 #include <atomic>
 #include <cfloat>
 #include <cstdint>
+#include <type_traits>
 
 #include "rkv_block.cuh"
 #include "rkv_internal.h"
@@ -136,6 +137,10 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
     const bool pool_max = p.gqa_pool == RKV_GQA_MAX;
     const int T = (N + kTileRows - 1) / kTileRows;
     const int64_t krow0 = (static_cast<int64_t>(b) * p.n_kv + h) * p.cap;
+    // paged caches: row r of this unit is row prow(r) of the layer's page pool
+    const bool paged = p.block_table != nullptr;
+    const int psh = paged ? 31 - __clz(p.page_rows) : 7;   // page_rows is a power of two
+    const int P = 1 << psh;
     const int64_t unit_g = (static_cast<int64_t>(p.layer_base + l) * p.batch + b) * p.n_kv + h;
 
     const UnitLayout L = make_unit_layout(p.nmax, NQP);
@@ -162,6 +167,11 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
     uint32_t *sKeys = reinterpret_cast<uint32_t *>(sStage);
     int32_t *sDst = reinterpret_cast<int32_t *>(sStage + arr);
     uint32_t *sHist = reinterpret_cast<uint32_t *>(sStage + 2u * arr);
+    int32_t *sBT = reinterpret_cast<int32_t *>(base + L.bt);
+    auto prow = [&](int r) -> int64_t {   // row of the layer's 2-D view holding unit row r
+        return paged ? ((static_cast<int64_t>(sBT[r >> psh]) * p.n_kv + h) << psh) + (r & (P - 1))
+                     : krow0 + r;
+    };
 
     const uint64_t colmask = NQ >= 64 ? ~0ull : ((1ull << NQ) - 1ull);
     const uint64_t lastmask = [&] {
@@ -191,6 +201,8 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
     }
     for (int i = tid; i < 2 * 4096 / 16; i += NT)
         reinterpret_cast<uint4 *>(sBs)[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (paged)
+        for (int j = tid; j < (N + P - 1) / P; j += NT) sBT[j] = p.block_table[static_cast<int64_t>(b) * p.max_blocks + j];
     // window key M + d is seen by query column g*w + j only when j >= d (causal)
     if (warp == 0) {
         const int j0 = lane % w, j1 = (lane + 32) % w;
@@ -214,9 +226,21 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
         tma_last = g;
         const int tt = g < T ? g : g - T;
         uint8_t *stg = sStage + (g & 1) * kStageBytes;
-        const int32_t y = static_cast<int32_t>(krow0 + tt * kTileRows);
-        tma_load_2d(stg, mk, &full[g & 1], 0, y);
-        tma_load_2d(stg + kHalfBytes, mk, &full[g & 1], 64, y);
+        if (!paged) {
+            const int32_t y = static_cast<int32_t>(krow0 + tt * kTileRows);
+            tma_load_2d(stg, mk, &full[g & 1], 0, y);
+            tma_load_2d(stg + kHalfBytes, mk, &full[g & 1], 64, y);
+        } else {
+            // one box per page; pages past the sequence's last read as zeros (a row
+            // coordinate below the pool)
+            const int npg = (N + P - 1) / P;
+            for (int j = 0; j < kTileRows / P; ++j) {
+                const int pg = tt * (kTileRows / P) + j;
+                const int32_t y = pg < npg ? static_cast<int32_t>(prow(pg * P)) : -P;
+                tma_load_2d(stg + j * P * 128, mk, &full[g & 1], 0, y);
+                tma_load_2d(stg + kHalfBytes + j * P * 128, mk, &full[g & 1], 64, y);
+            }
+        }
     };
     // logits (and in pass 2 of MEAN mode k . S) of tile g into TMEM slot g & 1
     auto issue_logits = [&](int g) {
@@ -626,10 +650,15 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
     // The compaction reads most of the unit's V rows: start bringing them into L2
     // now, while the select runs (HBM is otherwise idle in this phase).
     if (tid == 32 && p.v[l] != nullptr && !p.z_heads) {
-        const uint8_t *vrow = reinterpret_cast<const uint8_t *>(p.v[l] + krow0 * kHeadDim);
-        const uint32_t total = static_cast<uint32_t>(N) * 256u;
-        for (uint32_t off = 0; off < total; off += 65536u)
-            bulk_prefetch_l2(vrow + off, min(65536u, total - off));
+        if (!paged) {
+            const uint8_t *vrow = reinterpret_cast<const uint8_t *>(p.v[l] + krow0 * kHeadDim);
+            const uint32_t total = static_cast<uint32_t>(N) * 256u;
+            for (uint32_t off = 0; off < total; off += 65536u)
+                bulk_prefetch_l2(vrow + off, min(65536u, total - off));
+        } else {
+            for (int r = 0; r < N; r += P)
+                bulk_prefetch_l2(p.v[l] + prow(r) * kHeadDim, static_cast<uint32_t>(min(P, N - r)) * 256u);
+        }
     }
 
     // ---- normalisers, keys and the select (one per unit)
@@ -743,51 +772,67 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
         first = sRedU[0];
 #pragma unroll
         for (int k = 1; k < NW; ++k) first = min(first, sRedU[k]);
-        uint16_t *kb = p.k[l] + krow0 * kHeadDim;
-        uint16_t *vb = p.v[l] + krow0 * kHeadDim;
         // Software-pipelined: chunk c + 1 is read before chunk c is written.  Its
         // rows lie above every destination of chunk c, and every read of chunk c
-        // precedes the barrier before chunk c's writes.
-        constexpr int PER = kChunkRows * 16 / NT;   // 16-byte pieces per thread per chunk
-        auto load = [&](int c0, uint4 (&kx)[PER], uint4 (&vx)[PER], int (&dd)[PER]) {
+        // precedes the barrier before chunk c's writes.  The two cache layouts are
+        // compiled separately so the contiguous one carries no page lookups.
+        auto compaction = [&](auto paged_c) {
+            constexpr bool PG = decltype(paged_c)::value;
+            uint16_t *kb = p.k[l];
+            uint16_t *vb = p.v[l];
+            auto row_of = [&](int r) -> int64_t {
+                if constexpr (PG)
+                    return ((static_cast<int64_t>(sBT[r >> psh]) * p.n_kv + h) << psh) + (r & (P - 1));
+                else
+                    return krow0 + r;
+            };
+            constexpr int PER = kChunkRows * 16 / NT;   // 16-byte pieces per thread per chunk
+            auto load = [&](int c0, uint4 (&kx)[PER], uint4 (&vx)[PER], int (&dd)[PER]) {
 #pragma unroll
-            for (int k = 0; k < PER; ++k) {
-                const int idx = tid + k * NT;
-                const int row = c0 + (idx >> 4), pc = idx & 15;
-                const int d = row < N ? sDst[row] : -1;
-                dd[k] = (d >= 0 && d != row) ? d : -1;
-                if (dd[k] >= 0) {
-                    kx[k] = __ldcg(reinterpret_cast<const uint4 *>(kb + static_cast<int64_t>(row) * kHeadDim) + pc);
-                    vx[k] = __ldcg(reinterpret_cast<const uint4 *>(vb + static_cast<int64_t>(row) * kHeadDim) + pc);
+                for (int k = 0; k < PER; ++k) {
+                    const int idx = tid + k * NT;
+                    const int row = c0 + (idx >> 4), pc = idx & 15;
+                    const int d = row < N ? sDst[row] : -1;
+                    dd[k] = (d >= 0 && d != row) ? d : -1;
+                    if (dd[k] >= 0) {
+                        const int64_t src = row_of(row) * kHeadDim;
+                        kx[k] = __ldcg(reinterpret_cast<const uint4 *>(kb + src) + pc);
+                        vx[k] = __ldcg(reinterpret_cast<const uint4 *>(vb + src) + pc);
+                    }
                 }
+            };
+            auto store = [&](const uint4 (&kx)[PER], const uint4 (&vx)[PER], const int (&dd)[PER]) {
+#pragma unroll
+                for (int k = 0; k < PER; ++k) {
+                    if (dd[k] >= 0) {
+                        const int pc = (tid + k * NT) & 15;
+                        const int64_t dst = row_of(dd[k]) * kHeadDim;
+                        reinterpret_cast<uint4 *>(kb + dst)[pc] = kx[k];
+                        reinterpret_cast<uint4 *>(vb + dst)[pc] = vx[k];
+                    }
+                }
+            };
+            uint4 ka[PER], va[PER], kc[PER], vc[PER];
+            int da[PER], dc[PER];
+            int c0 = static_cast<int>(first);
+            if (c0 < N) load(c0, ka, va, da);
+            while (c0 < N) {
+                const int c1 = c0 + kChunkRows;
+                if (c1 < N) load(c1, kc, vc, dc);
+                __syncthreads();
+                store(ka, va, da);
+                if (c1 >= N) break;
+                const int c2 = c1 + kChunkRows;
+                if (c2 < N) load(c2, ka, va, da);
+                __syncthreads();
+                store(kc, vc, dc);
+                c0 = c2;
             }
         };
-        auto store = [&](const uint4 (&kx)[PER], const uint4 (&vx)[PER], const int (&dd)[PER]) {
-#pragma unroll
-            for (int k = 0; k < PER; ++k) {
-                if (dd[k] >= 0) {
-                    const int pc = (tid + k * NT) & 15;
-                    reinterpret_cast<uint4 *>(kb + static_cast<int64_t>(dd[k]) * kHeadDim)[pc] = kx[k];
-                    reinterpret_cast<uint4 *>(vb + static_cast<int64_t>(dd[k]) * kHeadDim)[pc] = vx[k];
-                }
-            }
-        };
-        uint4 ka[PER], va[PER], kc[PER], vc[PER];
-        int da[PER], dc[PER];
-        int c0 = static_cast<int>(first);
-        if (c0 < N) load(c0, ka, va, da);
-        while (c0 < N) {
-            const int c1 = c0 + kChunkRows;
-            if (c1 < N) load(c1, kc, vc, dc);
-            __syncthreads();
-            store(ka, va, da);
-            if (c1 >= N) break;
-            const int c2 = c1 + kChunkRows;
-            if (c2 < N) load(c2, ka, va, da);
-            __syncthreads();
-            store(kc, vc, dc);
-            c0 = c2;
-        }
+        if (paged)
+            compaction(std::true_type{});
+        else
+            compaction(std::false_type{});
     }
 
     __syncthreads();

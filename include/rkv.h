@@ -333,6 +333,44 @@ RKV_API rkv_status rkv_select_compact_shared(const rkv_config *cfg, int32_t n_la
                                              int32_t *kept_out, void *workspace, size_t ws_bytes,
                                              rkv_stream_t stream);
 
+/*
+ * Paged caches: each layer's keys and values
+ * live in page pools [num_pages][Hkv][page_rows][128] bf16, and sequence b
+ * owns the pages block_table[b][0..] in logical order (logical row i of a
+ * sequence is slot i % page_rows of page block_table[b][i / page_rows]; the
+ * table is shared by all layers).  The step is rkv_compress_step's, reading
+ * and compacting rows through the table; afterwards the pages a compressed
+ * sequence no longer needs, ceil(budget / P) .. ceil(N / P) - 1, are listed
+ * for the caller's allocator: physical eviction that returns freed blocks
+ * (hysenlabs write-up, decode-time section: the FREE_BLOCKS return path).
+ */
+typedef struct {
+    const int32_t *block_table; /* device [batch][max_blocks] page ids */
+    int32_t max_blocks;         /* row stride of block_table; max_blocks * page_rows = cap */
+    int32_t page_rows;          /* P: 16, 32, 64 or 128 */
+    int32_t num_pages;          /* pages in each layer's pool */
+    int32_t *freed_pages;       /* device [batch][max_blocks]: entries 0..n_freed[b]-1 get the
+                                   page ids sequence b gave back (in logical order) */
+    int32_t *n_freed;           /* device [batch]: pages given back (0 when not compressed) */
+} rkv_paged_kv;
+
+/*
+ * The step on paged caches.  k_pools / v_pools: host arrays [n_layers] of
+ * device pointers to the page pools; q_layers, budgets, lambdas, cur_len,
+ * opts (kept_out / scores_out / events; cluster_size 0 or 1) and the
+ * workspace (rkv_workspace_size with cap = max_blocks * page_rows) as in
+ * rkv_compress_step.  MEAN redundancy only (MAX: RKV_ERR_UNSUPPORTED); pages
+ * of different sequences must be distinct.  Caches up to 512 pages per
+ * sequence and one CTA's rows (rkv_query_step_shape cluster_size 1).
+ */
+RKV_API rkv_status rkv_compress_step_paged(const rkv_config *cfg, int32_t n_layers, int32_t batch,
+                                           const rkv_paged_kv *pg, rkv_bf16 *const *k_pools,
+                                           rkv_bf16 *const *v_pools,
+                                           const rkv_bf16 *const *q_layers,
+                                           const int32_t *budgets, const float *lambdas,
+                                           int32_t *cur_len, const rkv_step_options *opts,
+                                           void *workspace, size_t ws_bytes, rkv_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
