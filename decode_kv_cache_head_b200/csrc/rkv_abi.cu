@@ -238,15 +238,20 @@ cudaError_t launch_gram_layers(const rkv_config *cfg, int32_t n_layers, int32_t 
     gp->nblk = (cap - cfg->window + 127) / 128;
     gp->n_eff = n_eff;
     gp->r_out = r_ext;
+    gp->inv = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(r_ext) +
+                                        align256(static_cast<size_t>(n_layers) * batch *
+                                                 cfg->n_kv_heads * cap * 4));
     gp->status = status;
     cudaError_t e = cudaSuccess;
     for (int l0 = 0; e == cudaSuccess && l0 < n_layers; l0 += kMaxLayersPerLaunch) {
         const int nl = (n_layers - l0 < kMaxLayersPerLaunch) ? n_layers - l0 : kMaxLayersPerLaunch;
         gp->layer_base = l0;
-        for (int i = 0; i < nl && e == cudaSuccess; ++i)
+        for (int i = 0; i < nl && e == cudaSuccess; ++i) {
+            gp->k[i] = k_layers[l0 + i];
             if (!encode_rows128(&gp->tmap[i], k_layers[l0 + i],
                                 static_cast<uint64_t>(batch) * cfg->n_kv_heads * cap, 128))
                 e = cudaErrorInvalidValue;
+        }
         if (e == cudaSuccess) e = launch_gram_max(*gp, nl * batch * cfg->n_kv_heads, strm);
     }
     delete gp;
@@ -260,8 +265,8 @@ size_t ws_bytes_shared(const rkv_config *cfg, int32_t n_layers, int32_t batch, i
 size_t ws_bytes_for(const rkv_config *cfg, int32_t n_layers, int32_t batch, int32_t cap) {
     size_t n = kStatusBytes;
     n += align256(static_cast<size_t>(batch) * 4);
-    if (cfg->redundancy_mode == RKV_RED_MAX)
-        n += align256(static_cast<size_t>(n_layers) * batch * cfg->n_kv_heads * cap * 4);
+    if (cfg->redundancy_mode == RKV_RED_MAX)   // r, then the inverse norms, per unit
+        n += 2 * align256(static_cast<size_t>(n_layers) * batch * cfg->n_kv_heads * cap * 4);
     return n;
 }
 
@@ -331,6 +336,9 @@ rkv_status run_per_head_scores(const rkv_config *cfg, const rkv_bf16 *q, const r
         gp->nblk = (cap - cfg->window + 127) / 128;
         gp->n_tokens_fixed = n_tokens;
         gp->r_out = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + kStatusBytes + 256);
+        gp->inv = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(gp->r_out) +
+                                            align256(static_cast<size_t>(cfg->n_kv_heads) * cap * 4));
+        gp->k[0] = k;
         gp->status = static_cast<uint32_t *>(ws);
         p.r_ext = gp->r_out;
     }

@@ -9,11 +9,13 @@
 // One CTA per (unit, block of 128 candidate rows).  The Gram tiles
 // K_I . K_J^T are computed by tcgen05 UMMA (bf16 in, fp32 accumulate) into
 // TMEM and folded to row maxima on chip; the N x N matrix never reaches HBM.
+// A first pass (rkv_inv_norm_kernel) writes 1 / max(||k_j||, 1e-12) of every
+// row once, so the row blocks of a unit do not each recompute the norms of
+// every column tile.
 // Warp roles (320 threads):
-//   warps 0-7  epilogue: inverse norms of each key tile (two threads per row,
-//              from shared memory), then per row max_j acc_ij * inv_j from TMEM;
-//              warps w and w + 4 read the same 32 TMEM lanes (rows) and split
-//              the tile's 128 columns;
+//   warps 0-7  epilogue: per row max_j acc_ij * inv_j from TMEM; warps w and
+//              w + 4 read the same 32 TMEM lanes (rows) and split the tile's
+//              128 columns;
 //   warp 8     producer: TMA of the row block once, then 128-row column tiles
 //              into a two-stage ring;
 //   warp 9     MMA issuer: 8 UMMAs (K = 128) per column tile into one of two
@@ -55,25 +57,6 @@ __device__ __forceinline__ void named_sync_epilogue() {
     asm volatile("bar.sync 1, 256;" ::: "memory");
 }
 
-// Inverse norm of row r of a swizzled 128 x 128 bf16 tile, computed by the two
-// adjacent lanes 2r (columns 0-63) and 2r + 1 (columns 64-127).
-__device__ __forceinline__ float tile_row_inv_pair(const uint8_t *tile, int r, int half) {
-    float2 ss2 = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        const uint4 raw = *reinterpret_cast<const uint4 *>(tile + half * 16384 + sw128_offset(r, c));
-        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(h2[e]);
-            ss2 = __ffma2_rn(f, f, ss2);
-        }
-    }
-    float ss = ss2.x + ss2.y;
-    ss += __shfl_xor_sync(kFull, ss, 1);
-    return 1.0f / fmaxf(sqrtf(ss), 1e-12f);
-}
-
 }  // namespace
 
 __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __grid_constant__ GramParams p) {
@@ -102,7 +85,7 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
         mbar_init(&S.bar_a, 1);
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&S.full[s], 1);
-            mbar_init(&S.empty[s], 2);   // MMA done reading + norms done reading
+            mbar_init(&S.empty[s], 1);   // the MMA is done reading the tile
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(&S.tfull[t], 1);
@@ -160,52 +143,57 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
         // ---------------- epilogue warps 0-7: row i0 + (tid & 127), column half tid >> 7
         const int lrow = tid & 127, chalf = tid >> 7;
         const int i = i0 + lrow;
-        const int nrow = tid >> 1, nhalf = tid & 1;   // norms: two threads per row
-        if (!mbar_wait(&S.bar_a, 0)) ok = false;
-        {
-            const float iv = tile_row_inv_pair(S.a, nrow, nhalf);
-            if (nhalf == 0) S.inv_a[nrow] = iv;
+        const float *inv_g = p.inv + unit_g * p.cap;
+        if (tid < 128) {
+            S.inv_a[tid] = (i0 + tid < N) ? inv_g[i0 + tid] : 0.f;
+            S.inv_b[0][tid] = (tid < N) ? inv_g[tid] : 0.f;
         }
+        named_sync_epilogue();
         float best = -INFINITY;
         for (int jt = 0; jt < n_tiles; ++jt) {
-            const int s = jt % kStages, t = jt & 1;
-            if (ok && !mbar_wait(&S.full[s], (jt / kStages) & 1)) ok = false;
-            {
-                const float iv = tile_row_inv_pair(S.b[s], nrow, nhalf);
-                if (nhalf == 0) S.inv_b[t][nrow] = iv;
-            }
-            named_sync_epilogue();
-            if (tid == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&S.empty[s])) : "memory");
+            const int t = jt & 1;
+            // the next tile's inverse norms: loaded now, stored after this tile's epilogue
+            float nxt = 0.f;
+            if (tid < 128 && jt + 1 < n_tiles && (jt + 1) * 128 + tid < N) nxt = inv_g[(jt + 1) * 128 + tid];
             if (ok && !mbar_wait(&S.tfull[t], (jt >> 1) & 1)) ok = false;
             tc_fence_after();
             const int j0 = jt * 128 + chalf * 64;
             const bool clean = (jt * 128 + 128 <= N) && (jt != bi);
             const uint32_t taddr = tmem_base + ((32u * (warp & 3)) << 16) + t * 128u + chalf * 64u;
             const float *invt = &S.inv_b[t][chalf * 64];
-#pragma unroll 1
-            for (int c0 = 0; c0 < 64; c0 += 16) {
-                float v[16];
-                tmem_ld16(taddr + c0, v);
-                const float4 *iv4 = reinterpret_cast<const float4 *>(invt + c0);
-                float c[16];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
+            for (int c0 = 0; c0 < 64; c0 += 32) {
+                // 32 columns in flight per wait
+                uint32_t r0[16], r1[16];
+                tmem_ld16_nowait(taddr + c0, r0);
+                tmem_ld16_nowait(taddr + c0 + 16, r1);
+                tmem_wait_ld();
+                reg_tie16(r0);
+                reg_tie16(r1);
+                float c[32];
+                const float4 *iv4 = reinterpret_cast<const float4 *>(invt + c0);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
                     const float4 iv = iv4[q];
-                    const float2 a = __fmul2_rn(make_float2(v[4 * q], v[4 * q + 1]), make_float2(iv.x, iv.y));
-                    const float2 b = __fmul2_rn(make_float2(v[4 * q + 2], v[4 * q + 3]), make_float2(iv.z, iv.w));
-                    c[4 * q] = a.x; c[4 * q + 1] = a.y; c[4 * q + 2] = b.x; c[4 * q + 3] = b.y;
+                    const uint32_t *rr = q < 4 ? &r0[4 * q] : &r1[4 * (q - 4)];
+                    const float2 a = __fmul2_rn(make_float2(__uint_as_float(rr[0]), __uint_as_float(rr[1])),
+                                                make_float2(iv.x, iv.y));
+                    const float2 bb = __fmul2_rn(make_float2(__uint_as_float(rr[2]), __uint_as_float(rr[3])),
+                                                 make_float2(iv.z, iv.w));
+                    c[4 * q] = a.x; c[4 * q + 1] = a.y; c[4 * q + 2] = bb.x; c[4 * q + 3] = bb.y;
                 }
                 if (clean) {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) best = fmaxf(best, c[e]);
+                    for (int e = 0; e < 32; ++e) best = fmaxf(best, c[e]);
                 } else {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
+                    for (int e = 0; e < 32; ++e) {
                         const int j = j0 + c0 + e;
                         best = (j < N && j != i) ? fmaxf(best, c[e]) : best;
                     }
                 }
             }
+            if (tid < 128 && jt + 1 < n_tiles) S.inv_b[t ^ 1][tid] = nxt;   // read last in tile jt - 1
             tc_fence_before();
             named_sync_epilogue();
             if (tid == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&S.tempty[t])) : "memory");
@@ -222,12 +210,49 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
     }
 }
 
+// 1 / max(||k_j||, 1e-12) of every row of every due unit: half a warp per row
+// (16 lanes x 8 columns), 64 rows per CTA.
+__global__ void __launch_bounds__(256) rkv_inv_norm_kernel(const __grid_constant__ GramParams p,
+                                                           int nchunk) {
+    const int unit = blockIdx.x / nchunk, chunk = blockIdx.x % nchunk;
+    const int h = unit % p.n_kv;
+    const int b = (unit / p.n_kv) % p.batch;
+    const int l = unit / (p.n_kv * p.batch);
+    const int N = p.n_tokens_fixed > 0 ? p.n_tokens_fixed : p.n_eff[b];
+    if (N <= 0 || chunk * 64 >= N) return;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, half = lane >> 4, sub = lane & 15;
+    const int64_t krow0 = (static_cast<int64_t>(b) * p.n_kv + h) * p.cap;
+    const int64_t unit_g = (static_cast<int64_t>(p.layer_base + l) * p.batch + b) * p.n_kv + h;
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+        const int row = chunk * 64 + warp * 8 + it * 2 + half;
+        float2 ss2 = make_float2(0.f, 0.f);
+        if (row < N) {
+            const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(p.k[l] + (krow0 + row) * kHeadDim) + sub);
+            const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(h2[e]);
+                ss2 = __ffma2_rn(f, f, ss2);
+            }
+        }
+        float ss = ss2.x + ss2.y;
+#pragma unroll
+        for (int off = 8; off >= 1; off >>= 1) ss += __shfl_xor_sync(kFull, ss, off);
+        if (row < N && sub == 0) p.inv[unit_g * p.cap + row] = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
+    }
+}
+
 size_t gram_smem_bytes() { return sizeof(GramSmem) + 1024; }
 
 cudaError_t launch_gram_max(const GramParams &p, int n_units, cudaStream_t stream) {
     const size_t smem = gram_smem_bytes();
     static std::atomic<int> granted{0};
     cudaError_t e = ensure_smem_attr(rkv_gram_max_kernel, smem, granted);
+    if (e != cudaSuccess) return e;
+    const int nchunk = (p.cap + 63) / 64;
+    rkv_inv_norm_kernel<<<static_cast<unsigned>(n_units * nchunk), 256, 0, stream>>>(p, nchunk);
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     rkv_gram_max_kernel<<<n_units * p.nblk, kGramThreads, smem, stream>>>(p);
     return cudaGetLastError();

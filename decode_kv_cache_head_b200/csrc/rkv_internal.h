@@ -235,10 +235,12 @@ cudaError_t launch_freed_pages(int batch, const int32_t *budgets, int32_t budget
 // MAX-mode similarity kernel: raw r of every candidate of every due unit.
 struct alignas(64) GramParams {
     CUtensorMap tmap[kMaxLayersPerLaunch];   // [B*Hkv*cap rows, 128] bf16, box 64 x 128, SW128
+    const uint16_t *k[kMaxLayersPerLaunch];  // the same caches, for the inverse-norm pass
     int32_t layer_base, batch, n_kv, window, cap, nblk;
     int32_t n_tokens_fixed;  // > 0: per-head entry point, N fixed
     const int32_t *n_eff;
     float *r_out;            // [units][cap]
+    float *inv;              // [units][cap] 1 / max(||k||, 1e-12), written by the first pass
     uint32_t *status;
 };
 cudaError_t launch_gram_max(const GramParams &p, int n_units, cudaStream_t stream);
