@@ -647,20 +647,6 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
         return;
     }
 
-    // The compaction reads most of the unit's V rows: start bringing them into L2
-    // now, while the select runs (HBM is otherwise idle in this phase).
-    if (tid == 32 && p.v[l] != nullptr && !p.z_heads) {
-        if (!paged) {
-            const uint8_t *vrow = reinterpret_cast<const uint8_t *>(p.v[l] + krow0 * kHeadDim);
-            const uint32_t total = static_cast<uint32_t>(N) * 256u;
-            for (uint32_t off = 0; off < total; off += 65536u)
-                bulk_prefetch_l2(vrow + off, min(65536u, total - off));
-        } else {
-            for (int r = 0; r < N; r += P)
-                bulk_prefetch_l2(p.v[l] + prow(r) * kHeadDim, static_cast<uint32_t>(min(P, N - r)) * 256u);
-        }
-    }
-
     // ---- normalisers, keys and the select (one per unit)
     float inv_sumI, rmax_g, inv_rsum;
     uint32_t Tk = 0xffffffffu;
