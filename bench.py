@@ -58,6 +58,11 @@ def parse_args():
     ap.add_argument("--cluster-size", type=int, default=0,
                     help="CTAs per unit: 0 = the library's choice, 1 = one CTA per unit, "
                          "2/4/8/16 = a cluster per unit")
+    ap.add_argument("--mode", default="step", choices=["step", "shared", "paged"],
+                    help="step: rkv_compress_step (the headline); shared: one kept set per "
+                         "(layer, sequence) across the KV heads (rkv_score_shared, all-reduce "
+                         "over ranks, rkv_select_compact_shared); paged: rkv_compress_step_paged")
+    ap.add_argument("--page-rows", type=int, default=16)
     ap.add_argument("--loop", action="store_true",
                     help="run the whole decode loop of the workload (append + compress steps)")
     ap.add_argument("--generated", type=int, default=16384,
@@ -239,8 +244,9 @@ def workload_config(w, red_mode, args):
             "redundancy": "max" if red_mode else "mean", "gqa_pool": "max",
             "cached_len": w.n_tokens()[0] if len(set(w.n_tokens())) == 1 else "ragged",
             "near_duplicate_frac": list(w.dup_frac) if len(w.dup_frac) > 1 else w.dup_frac[0],
-            "l2": "fresh in-HBM replica per step (K+V larger than L2) and a 256 MB L2 flush "
-                  "before the timed region",
+            "l2": "pristine in-HBM caches every step (a fresh replica, or the working copy "
+                  "restored outside the per-step events when replicas do not fit; K+V larger "
+                  "than L2) and a 256 MB L2 flush before the timed region",
             "parallelism": f"dp{args.gpus} (independent sequences per rank)"}
 
 
@@ -297,18 +303,30 @@ def run_rkv(args, w, red_mode):
     G = w.n_q_heads // w.n_kv_heads
     alg_bytes = 256 * (L * H * int(n_tok.sum()) + units * G * w.window + 3 * moved)
 
-    # replicas: one pristine copy per warm-up and timed step
+    # replicas: one pristine copy per warm-up and timed step when they fit in memory;
+    # otherwise one working copy restored from the pristine one before every step,
+    # with the restore outside per-step events
     n_rep = args.warmup + args.steps
-    reps = [(K0.clone(), V0.clone(), cur0.clone()) for _ in range(n_rep)]
+    rep_bytes = 2 * K0.numel() * K0.element_size()
+    fits = n_rep * rep_bytes < 0.7 * torch.cuda.mem_get_info(dev)[0]
+    reps = [(K0.clone(), V0.clone(), cur0.clone()) for _ in range(n_rep if fits else 1)]
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
+    st = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
     for a, b in ev:        # materialise the events before handing them to the library
         a.record(stream); b.record(stream)
+
+    def restore():
+        reps[0][0].copy_(K0); reps[0][1].copy_(V0); reps[0][2].copy_(cur0)
+
     sampler = ClockSampler(local)
     sampler.start()
     for i in range(args.warmup):
-        step(*reps[i])
+        if not fits:
+            restore()
+        step(*reps[i if fits else 0])
     flush.fill_(1.0)
     torch.cuda.synchronize()
     rdist.barrier(dev)
@@ -316,13 +334,20 @@ def run_rkv(args, w, red_mode):
     t_start, t_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
     for i in range(args.steps):
-        step(*reps[args.warmup + i], events=ev[i])
+        if not fits:
+            restore()
+        st[i][0].record(stream)
+        step(*reps[args.warmup + i if fits else 0], events=ev[i])
+        st[i][1].record(stream)
     t_stop.record(stream)
     torch.cuda.synchronize()
     rdist.barrier(dev)
     clocks = sampler.stop()
     assert rkv.rkv_workspace_status(ws) == 0
-    elapsed_ms = t_start.elapsed_time(t_stop)
+    if fits:
+        elapsed_ms = t_start.elapsed_time(t_stop)
+    else:
+        elapsed_ms = sum(a.elapsed_time(b) for a, b in st)
     kern_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
     elapsed_ms, kern_ms = rdist.max_over_ranks([elapsed_ms, kern_ms], dev)
     del reps
@@ -331,7 +356,8 @@ def run_rkv(args, w, red_mode):
 
     # end to end through host buffers: H2D of the inputs, the step, D2H of the result
     e2e = None
-    if args.e2e_steps > 0:
+    # the end-to-end leg pins two host copies of the caches: only for caches of a few GB
+    if args.e2e_steps > 0 and rep_bytes <= 4 * 1024 ** 3:
         hK, hV, hQ = K0.cpu().pin_memory(), V0.cpu().pin_memory(), Q.cpu().pin_memory()
         hc = cur0.cpu().pin_memory()
         oK, oV, oc = torch.empty_like(hK).pin_memory(), torch.empty_like(hV).pin_memory(), \
@@ -494,6 +520,111 @@ def run_loop(args, w, red_mode):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- other modes
+def run_mode(args, w, red_mode):
+    """The shared-selection or paged-cache variant of the step on the same workload:
+    device-timed with CUDA events over the whole call sequence, a fresh replica per step."""
+    world, rank, local = dist_setup(args)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=dev)
+    from decode_kv_cache_head_b200 import build
+    build.build()
+    import decode_kv_cache_head_b200 as rkv
+    from decode_kv_cache_head_b200 import dist as rdist
+
+    tp = args.mode == "shared" and world > 1
+    # shared selection across ranks is tensor parallelism: every rank holds the same
+    # sequences and its own share of the KV heads; the other modes shard sequences
+    x = make_inputs(w, device=str(dev), seed=w.seed if tp else rdist.rank_seed(w.seed, rank))
+    K0, V0, Q, cur0 = x["K"], x["V"], x["Q"], x["cur_len"].to(dev)
+    G = w.n_q_heads // w.n_kv_heads
+    if tp:
+        h0, h1 = rdist.head_range(w.n_kv_heads, world, rank)
+        K0, V0 = K0[:, :, h0:h1].contiguous(), V0[:, :, h0:h1].contiguous()
+        Q = Q[:, :, h0 * G:h1 * G].contiguous()
+    L, B, H, cap, D = K0.shape
+    cfg = rkv.make_config(w.budget_of(0), w.buffer, w.window, 128, H, H * G,
+                          w.mix_lambda, redundancy_mode=red_mode)
+    budgets = None
+    if len(w.budgets) > 1:
+        budgets = torch.tensor([w.budget_of(b) for b in range(B)], dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+    n_rep = args.warmup + args.steps
+    extra = {}
+    if args.mode == "shared":
+        ws = torch.zeros(rkv.rkv_workspace_size_shared(cfg, L, B, cap), dtype=torch.uint8,
+                         device=dev)
+        z = torch.empty((L, B, cap), dtype=torch.float32, device=dev)
+        reps = [(K0.clone(), V0.clone(), cur0.clone()) for _ in range(n_rep)]
+
+        def call(r):
+            rdist.compress_step_shared(rkv, cfg, r[0], r[1], Q, r[2], z, ws, budgets=budgets,
+                                       stream=stream)
+        extra["all_reduce_bytes_per_step"] = z.numel() * 4 if world > 1 else 0
+    else:
+        P = args.page_rows
+        assert cap % P == 0, "cache length must be a multiple of the page size"
+        mb = cap // P
+        pages = B * mb
+        perm = torch.randperm(pages, generator=torch.Generator().manual_seed(7)).to(torch.int32)
+        bt = perm.view(B, mb).to(dev)
+        pk = torch.empty((L, pages, H, P, D), dtype=torch.bfloat16, device=dev)
+        pv = torch.empty_like(pk)
+        idx = bt.view(-1).long()
+        pk[:, idx] = K0.view(L, B, H, mb, P, D).permute(0, 1, 3, 2, 4, 5).reshape(L, pages, H, P, D)
+        pv[:, idx] = V0.view(L, B, H, mb, P, D).permute(0, 1, 3, 2, 4, 5).reshape(L, pages, H, P, D)
+        ws = torch.zeros(rkv.rkv_workspace_size(cfg, L, B, cap), dtype=torch.uint8, device=dev)
+        freed = torch.empty((B, mb), dtype=torch.int32, device=dev)
+        n_freed = torch.empty((B,), dtype=torch.int32, device=dev)
+        reps = [(pk.clone(), pv.clone(), cur0.clone()) for _ in range(n_rep)]
+        del pk, pv
+
+        def call(r):
+            rkv.rkv_compress_step_paged(cfg, r[0], r[1], Q, r[2], ws, bt, P, freed, n_freed,
+                                        budgets=budgets, stream=stream)
+        extra["page_rows"] = P
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    sampler = ClockSampler(local)
+    sampler.start()
+    for i in range(args.warmup):
+        call(reps[i])
+    flush.fill_(1.0)
+    torch.cuda.synchronize()
+    rdist.barrier(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(args.steps):
+        call(reps[args.warmup + i])
+    b.record(stream)
+    torch.cuda.synchronize()
+    rdist.barrier(dev)
+    clocks = sampler.stop()
+    assert rkv.rkv_workspace_status(ws) == 0
+    ms = rdist.max_over_ranks([a.elapsed_time(b) / args.steps], dev)[0]
+    token_heads = w.token_heads() * (1 if tp else world)   # whole job
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": token_heads / (ms / 1e3), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "us_per_step": ms * 1e3, "higher_is_better": True,
+            "scaling": "strong" if tp else "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": dict(workload_config(w, red_mode, args), mode=args.mode, **extra,
+                           **({"parallelism": f"tp{world} (KV heads split over ranks)"}
+                              if tp else {})),
+            "gpu_launches": (4 if args.mode == "shared" else 3) * args.steps,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def main():
     args = parse_args()
     w = WORKLOADS[args.workload]
@@ -502,6 +633,8 @@ def main():
         run_reference(args, w, red_mode)
     elif args.loop:
         run_loop(args, w, red_mode)
+    elif args.mode != "step":
+        run_mode(args, w, red_mode)
     else:
         run_rkv(args, w, red_mode)
 
