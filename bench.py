@@ -410,7 +410,8 @@ def run_rkv(args, w, red_mode):
         torch.distributed.destroy_process_group()
     if rank != 0:
         return
-    n_main_launches = (L + 31) // 32
+    # per 32-layer chunk: the step kernel, plus the inverse-norm and similarity kernels in MAX mode
+    n_main_launches = ((L + 31) // 32) * (3 if red_mode else 1)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "us_per_step": ms_per_step * 1e3,
@@ -616,7 +617,11 @@ def run_mode(args, w, red_mode):
             "config": dict(workload_config(w, red_mode, args), mode=args.mode, **extra,
                            **({"parallelism": f"tp{world} (KV heads split over ranks)"}
                               if tp else {})),
-            "gpu_launches": (4 if args.mode == "shared" else 3) * args.steps,
+            # shared: plan, scoring kernels, head sum, plan, select+compact per 32-layer chunk;
+            # paged: plan, freed pages, step kernel per chunk
+            "gpu_launches": args.steps * (
+                3 + ((L + 31) // 32) * (2 + (2 if red_mode else 0)) if args.mode == "shared"
+                else 2 + (L + 31) // 32),
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)

@@ -259,7 +259,7 @@ cudaError_t launch_gram_layers(const rkv_config *cfg, int32_t n_layers, int32_t 
 }
 
 // Workspace of the shared-selection calls: the step's, then the per-head Z of
-// every unit and the destination of every row of every (layer, sequence).
+// every unit.
 size_t ws_bytes_shared(const rkv_config *cfg, int32_t n_layers, int32_t batch, int32_t cap);
 
 size_t ws_bytes_for(const rkv_config *cfg, int32_t n_layers, int32_t batch, int32_t cap) {
@@ -272,8 +272,7 @@ size_t ws_bytes_for(const rkv_config *cfg, int32_t n_layers, int32_t batch, int3
 
 size_t ws_bytes_shared(const rkv_config *cfg, int32_t n_layers, int32_t batch, int32_t cap) {
     const size_t units = static_cast<size_t>(n_layers) * batch * cfg->n_kv_heads;
-    return ws_bytes_for(cfg, n_layers, batch, cap) + align256(units * cap * 4) +
-           align256(static_cast<size_t>(n_layers) * batch * cap * 4);
+    return ws_bytes_for(cfg, n_layers, batch, cap) + align256(units * cap * 4);
 }
 
 void fill_common(StepParams &p, const rkv_config *cfg, const Shape &s, int batch, int cap) {
@@ -771,8 +770,6 @@ rkv_status rkv_select_compact_shared(const rkv_config *cfg, int32_t n_layers, in
     uint32_t *status = reinterpret_cast<uint32_t *>(ws);
     int32_t *n_eff = reinterpret_cast<int32_t *>(ws + kStatusBytes);
     const size_t units = static_cast<size_t>(n_layers) * batch * cfg->n_kv_heads;
-    int32_t *dst = reinterpret_cast<int32_t *>(ws + ws_bytes_for(cfg, n_layers, batch, cap) +
-                                               align256(units * cap * 4));
     cudaError_t e = cudaMemsetAsync(ws, 0, kStatusBytes, strm);
     if (e == cudaSuccess)
         e = launch_plan(batch, budgets, cfg->budget, cfg->buffer, cfg->window, cap, cur_len, n_eff,
@@ -791,14 +788,12 @@ rkv_status rkv_select_compact_shared(const rkv_config *cfg, int32_t n_layers, in
         const int nl = (n_layers - l0 < kMaxLayersPerLaunch) ? n_layers - l0 : kMaxLayersPerLaunch;
         const size_t off = static_cast<size_t>(l0) * batch * cap;
         sp.z_sum = const_cast<float *>(z_sum) + off;
-        sp.dst = dst + off;
         sp.kept_out = kept_out ? kept_out + off : nullptr;
         for (int i = 0; i < nl; ++i) {
             sp.k[i] = k_layers[l0 + i];
             sp.v[i] = v_layers[l0 + i];
         }
-        e = launch_shared_select(sp, nl * batch, strm);
-        if (e == cudaSuccess) e = launch_shared_compact(sp, nl * batch * cfg->n_kv_heads, strm);
+        e = launch_shared_compact(sp, nl * batch * cfg->n_kv_heads, strm);
     }
     return cuda_status(e);
 }

@@ -1,9 +1,9 @@
 // rkv_block.cuh -- block-level building blocks, templated on the CTA's thread
 // count NT (a multiple of 32): deterministic reductions (fixed butterfly order,
-// then the warps in warp order), a merged (sum, max, sum-of-exp) reduction,
-// packed exclusive scans, a warp "transpose-reduce" that folds 16 per-thread
-// columns across the 32 lanes, the order-preserving key of a float, the joint
-// score, and a radix select of the k-th largest 32-bit key.
+// then the warps in warp order), packed exclusive scans, a warp
+// "transpose-reduce" that folds 16 per-thread columns across the 32 lanes, the
+// order-preserving key of a float, the joint score, and radix selects of the
+// k-th largest 32-bit key.
 #pragma once
 
 #include <cstdint>
@@ -50,57 +50,6 @@ __device__ __forceinline__ uint32_t block_sum_u32(uint32_t x, uint32_t *red) {
     uint32_t r = 0;
 #pragma unroll
     for (int w = 0; w < NT / 32; ++w) r += red[w];
-    __syncthreads();
-    return r;
-}
-
-// (s, m, l): a plain sum s, and a running max m with l = sum exp(x - m).
-struct SumMaxExp {
-    float s, m, l;
-};
-
-__device__ __forceinline__ SumMaxExp merge_sme(SumMaxExp a, SumMaxExp b) {
-    SumMaxExp r;
-    r.s = a.s + b.s;
-    r.m = fmaxf(a.m, b.m);
-    const float la = (a.m == -INFINITY) ? 0.f : a.l * exp2f((a.m - r.m) * kLog2e);
-    const float lb = (b.m == -INFINITY) ? 0.f : b.l * exp2f((b.m - r.m) * kLog2e);
-    r.l = la + lb;
-    return r;
-}
-
-__device__ __forceinline__ SumMaxExp sme_add(SumMaxExp a, float s, float x) {
-    a.s += s;
-    if (x > a.m) {
-        a.l = ((a.m == -INFINITY) ? 0.f : a.l * exp2f((a.m - x) * kLog2e)) + 1.0f;
-        a.m = x;
-    } else {
-        a.l += exp2f((x - a.m) * kLog2e);
-    }
-    return a;
-}
-
-// `red` needs 4 * NT/32 floats.  Every thread gets the same result.
-template <int NT>
-__device__ __forceinline__ SumMaxExp block_reduce_sme(SumMaxExp v, float *red) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-        SumMaxExp o;
-        o.s = __shfl_xor_sync(kFull, v.s, off);
-        o.m = __shfl_xor_sync(kFull, v.m, off);
-        o.l = __shfl_xor_sync(kFull, v.l, off);
-        v = merge_sme(v, o);
-    }
-    if (lane == 0) {
-        red[4 * warp + 0] = v.s;
-        red[4 * warp + 1] = v.m;
-        red[4 * warp + 2] = v.l;
-    }
-    __syncthreads();
-    SumMaxExp r = {red[0], red[1], red[2]};
-#pragma unroll
-    for (int w = 1; w < NT / 32; ++w) r = merge_sme(r, SumMaxExp{red[4 * w], red[4 * w + 1], red[4 * w + 2]});
     __syncthreads();
     return r;
 }
@@ -160,155 +109,6 @@ __device__ __forceinline__ uint32_t ordered_key(float z) {
 // from the same I and R gets the same bits.
 __device__ __forceinline__ float joint_score(float lambda, float I, float R) {
     return __fsub_rn(__fmul_rn(lambda, I), __fmul_rn(__fsub_rn(1.0f, lambda), R));
-}
-
-// Radix select over keys[0..n) in shared memory (all NT threads call): T =
-// the kk-th largest key (1 <= kk <= n) and n_gt = the number of keys > T.
-// Four rounds of 8-bit digits, most significant first.  Each warp counts into
-// its own 256-bin histogram (one atomic per warp when all its lanes share the
-// digit, which is the common case in the first rounds), the bins are summed
-// over the warps and a block-wide suffix scan finds the digit holding the
-// kk-th largest key.  Key j is keys[j * STRIDE].  hist: (NT/32) * 256 uint32;
-// scan: NT/32 + 4 uint32.
-template <int NT, int STRIDE = 1>
-__device__ __forceinline__ void block_select_kth(const uint32_t *keys, int n, int kk,
-                                                 uint32_t *hist, uint32_t *scan, uint32_t &T,
-                                                 int &n_gt) {
-    constexpr int NW = NT / 32;
-    static_assert(NT == 256, "one thread per histogram bin");
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    uint32_t *my = hist + warp * 256;
-    uint32_t prefix = 0, mask = 0;
-    int remaining = kk, above_total = 0;
-#pragma unroll 1
-    for (int round = 0; round < 4; ++round) {
-        const int shift = 24 - 8 * round;
-#pragma unroll
-        for (int i = lane; i < 256; i += 32) my[i] = 0;
-        __syncwarp();
-        for (int base = 0; base < n; base += NT) {
-            const int j = base + tid;
-            const uint32_t key = (j < n) ? keys[j * STRIDE] : 0u;
-            const bool part = (j < n) && ((key & mask) == prefix);
-            const uint32_t digit = (key >> shift) & 255u;
-            const unsigned act = __ballot_sync(kFull, part);
-            if (act == 0) continue;
-            const uint32_t d0 = __shfl_sync(kFull, digit, __ffs(act) - 1);
-            if (__all_sync(kFull, !part || digit == d0)) {
-                if (lane == 0) my[d0] += static_cast<uint32_t>(__popc(act));
-            } else if (part) {
-                atomicAdd(&my[digit], 1u);
-            }
-            __syncwarp();
-        }
-        __syncthreads();
-        // thread t owns bin 255 - t, so a prefix over threads is a suffix over bins
-        const int bin = 255 - tid;
-        uint32_t cnt = 0;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) cnt += hist[w * 256 + bin];
-        uint32_t inc = cnt;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const uint32_t o = __shfl_up_sync(kFull, inc, off);
-            if (lane >= off) inc += o;
-        }
-        if (lane == 31) scan[warp] = inc;
-        __syncthreads();
-        uint32_t above = inc - cnt;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) above += (w < warp) ? scan[w] : 0u;
-        if (above < static_cast<uint32_t>(remaining) && above + cnt >= static_cast<uint32_t>(remaining)) {
-            scan[NW + 0] = static_cast<uint32_t>(bin);
-            scan[NW + 1] = above;
-        }
-        __syncthreads();
-        const uint32_t d = scan[NW + 0];
-        const int ab = static_cast<int>(scan[NW + 1]);
-        prefix |= d << shift;
-        mask |= 255u << shift;
-        remaining -= ab;
-        above_total += ab;
-        __syncthreads();   // scan[] and the histograms are reused by the next round
-    }
-    T = prefix;
-    n_gt = above_total;
-}
-
-// The same select with each thread's keys held in registers across the four
-// rounds (key j = keys[j * STRIDE] for j = tid + k * NT, k < KPT); needs
-// n <= KPT * NT.  Three block barriers per round.
-template <int NT, int KPT, int STRIDE>
-__device__ __forceinline__ void block_select_kth_reg(const uint32_t *keys, int n, int kk,
-                                                     uint32_t *hist, uint32_t *scan, uint32_t &T,
-                                                     int &n_gt) {
-    constexpr int NW = NT / 32;
-    static_assert(NT == 256, "one thread per histogram bin");
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int kpt = (n + NT - 1) / NT;
-    uint32_t kr[KPT];
-#pragma unroll
-    for (int k = 0; k < KPT; ++k) {
-        const int j = tid + k * NT;
-        kr[k] = (k < kpt && j < n) ? keys[j * STRIDE] : 0u;
-    }
-    uint32_t *my = hist + warp * 256;
-    uint32_t prefix = 0, mask = 0;
-    int remaining = kk, above_total = 0;
-#pragma unroll 1
-    for (int round = 0; round < 4; ++round) {
-        const int shift = 24 - 8 * round;
-#pragma unroll
-        for (int i = lane; i < 256; i += 32) my[i] = 0;
-        __syncwarp();
-#pragma unroll
-        for (int k = 0; k < KPT; ++k) {
-            if (k < kpt) {
-                const int j = tid + k * NT;
-                const bool part = (j < n) && ((kr[k] & mask) == prefix);
-                const uint32_t digit = (kr[k] >> shift) & 255u;
-                const unsigned act = __ballot_sync(kFull, part);
-                if (act != 0) {
-                    const uint32_t d0 = __shfl_sync(kFull, digit, __ffs(act) - 1);
-                    if (__all_sync(kFull, !part || digit == d0)) {
-                        if (lane == 0) atomicAdd(&my[d0], static_cast<uint32_t>(__popc(act)));
-                    } else if (part) {
-                        atomicAdd(&my[digit], 1u);
-                    }
-                }
-            }
-        }
-        __syncthreads();
-        const int bin = 255 - tid;   // a prefix over threads is a suffix over bins
-        uint32_t cnt = 0;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) cnt += hist[w * 256 + bin];
-        uint32_t inc = cnt;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const uint32_t o = __shfl_up_sync(kFull, inc, off);
-            if (lane >= off) inc += o;
-        }
-        if (lane == 31) scan[warp] = inc;
-        __syncthreads();
-        uint32_t above = inc - cnt;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) above += (w < warp) ? scan[w] : 0u;
-        if (above < static_cast<uint32_t>(remaining) && above + cnt >= static_cast<uint32_t>(remaining)) {
-            scan[NW + 0] = static_cast<uint32_t>(bin);
-            scan[NW + 1] = above;
-        }
-        __syncthreads();
-        const uint32_t d = scan[NW + 0];
-        const int ab = static_cast<int>(scan[NW + 1]);
-        prefix |= d << shift;
-        mask |= 255u << shift;
-        remaining -= ab;
-        above_total += ab;
-    }
-    T = prefix;
-    n_gt = above_total;
-    __syncthreads();   // the scan slots and histograms may be reused by the caller
 }
 
 // Radix select with the keys already in registers (thread tid holds keys

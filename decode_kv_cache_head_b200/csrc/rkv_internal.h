@@ -218,12 +218,10 @@ struct SharedParams {
     const int32_t *n_eff;
     const float *z_heads;    // [layers][batch][Hkv][cap] per-head Z
     float *z_sum;            // [layers][batch][cap]
-    int32_t *dst;            // [layers][batch][cap] destination row or -1
     int32_t *kept_out;       // optional [layers][batch][cap]
     uint32_t *status;
 };
 cudaError_t launch_head_sum(const SharedParams &p, int n_lb, cudaStream_t stream);
-cudaError_t launch_shared_select(const SharedParams &p, int n_lb, cudaStream_t stream);
 cudaError_t launch_shared_compact(const SharedParams &p, int n_units, cudaStream_t stream);
 size_t shared_select_smem(int cap);
 

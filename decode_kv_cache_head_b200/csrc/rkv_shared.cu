@@ -6,14 +6,16 @@
 // "R-KV: Redundancy-aware KV Cache Compression for Reasoning Models",
 // decode-time section: the vLLM port's cross-rank eviction-score all-reduce).
 //
-// Three kernels after the per-head scoring (rkv_unit_kernel in scores-only
+// Two kernels around the per-head scoring (rkv_unit_kernel in scores-only
 // mode writes Z of every head):
-//   rkv_head_sum_kernel       z_sum[l][b][i] = sum_h Z[l][b][h][i], h ascending
-//   rkv_shared_select_kernel  one CTA per (layer, sequence): top budget - w of
-//                             z_sum by (score desc, index asc) plus the window;
-//                             destination of every row
-//   rkv_shared_compact_kernel one CTA per (layer, sequence, head): the rows
-//                             that move, in ascending chunks of 128 rows
+//   rkv_head_sum_kernel            z_sum[l][b][i] = sum_h Z[l][b][h][i], h ascending
+//   rkv_shared_compact_kernel      one CTA per (layer, sequence, head): the top
+//                                  budget - w candidates of z_sum by (score desc,
+//                                  index asc) plus the window -- the same select
+//                                  in every CTA of a (layer, sequence), so the
+//                                  destinations never leave shared memory -- then
+//                                  the head's in-place compaction in ascending
+//                                  chunks of 128 rows
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -49,9 +51,11 @@ __global__ void __launch_bounds__(256) rkv_head_sum_kernel(const SharedParams p)
     p.z_sum[static_cast<int64_t>(lb) * p.cap + i] = s;
 }
 
+// Keys of z_sum, the radix select and the destination of every row (sDst).
 template <int KPT>
 __device__ __forceinline__ void shared_select_body(const SharedParams &p, int lb, int N, int M,
-                                                   int kk, uint32_t *sKeys, uint32_t *sHist,
+                                                   int kk, bool write_kept, uint32_t *sKeys,
+                                                   int32_t *sDst, uint32_t *sHist,
                                                    uint32_t *sRedU) {
     constexpr int NT = kSelThreads;
     const int tid = threadIdx.x;
@@ -71,7 +75,6 @@ __device__ __forceinline__ void shared_select_body(const SharedParams &p, int lb
     int n_gt = 0;
     if (kk > 0) block_select_kth_fast<NT, KPT>(kr, kv, kk, sHist, T, n_gt);
     const int need_eq = (kk > 0) ? kk - n_gt : 0;
-    int32_t *dst = p.dst + static_cast<int64_t>(lb) * p.cap;
     uint32_t g_run = 0, e_run = 0;
     for (int c0 = 0; c0 < N; c0 += NT) {
         const int row = c0 + tid;
@@ -86,18 +89,27 @@ __device__ __forceinline__ void shared_select_body(const SharedParams &p, int lb
         const bool kept = gw || (eq && Ei < static_cast<uint32_t>(need_eq));
         if (in) {
             const int32_t d = kept ? static_cast<int32_t>(Gi + min(Ei, static_cast<uint32_t>(need_eq))) : -1;
-            dst[row] = d;
-            if (p.kept_out && d >= 0) p.kept_out[static_cast<int64_t>(lb) * p.cap + d] = row;
+            sDst[row] = d;
+            if (write_kept && p.kept_out && d >= 0) p.kept_out[static_cast<int64_t>(lb) * p.cap + d] = row;
         }
         e_run += tot2 >> 16;
         g_run += tot2 & 0xffffu;
     }
+    __syncthreads();
 }
 
-__global__ void __launch_bounds__(kSelThreads) rkv_shared_select_kernel(const SharedParams p) {
+// One CTA per (layer, sequence, head): the select of its (layer, sequence),
+// then the head's compaction.  In place: every source row of a chunk is read
+// before any row of the chunk is written, and later chunks read only rows
+// above it (destinations never exceed their source).
+__global__ void __launch_bounds__(kSelThreads) rkv_shared_compact_kernel(const SharedParams p) {
+    constexpr int NT = kSelThreads;
     extern __shared__ uint32_t sel_smem[];
-    const int lb = blockIdx.x;
+    const int unit = blockIdx.x;                 // (layer, sequence, head)
+    const int h = unit % p.n_kv;
+    const int lb = unit / p.n_kv;
     const int b = lb % p.batch;
+    const int l = lb / p.batch;
     const int N = p.n_eff[b];
     if (N <= 0) return;
     const int M = N - p.window;
@@ -106,40 +118,26 @@ __global__ void __launch_bounds__(kSelThreads) rkv_shared_select_kernel(const Sh
     uint32_t *sHist = sel_smem;                  // 4 x 256
     uint32_t *sRedU = sel_smem + 1024;           // 64
     uint32_t *sKeys = sel_smem + 1024 + 64;      // cap
-    constexpr int NT = kSelThreads;
-    if (M <= 5 * NT) shared_select_body<5>(p, lb, N, M, kk, sKeys, sHist, sRedU);
-    else if (M <= 9 * NT) shared_select_body<9>(p, lb, N, M, kk, sKeys, sHist, sRedU);
-    else if (M <= 16 * NT) shared_select_body<16>(p, lb, N, M, kk, sKeys, sHist, sRedU);
-    else shared_select_body<32>(p, lb, N, M, kk, sKeys, sHist, sRedU);
-}
+    int32_t *sDst = reinterpret_cast<int32_t *>(sKeys + p.cap);   // cap
+    const bool wk = h == 0;                      // one CTA writes kept_out
+    if (M <= 5 * NT) shared_select_body<5>(p, lb, N, M, kk, wk, sKeys, sDst, sHist, sRedU);
+    else if (M <= 9 * NT) shared_select_body<9>(p, lb, N, M, kk, wk, sKeys, sDst, sHist, sRedU);
+    else if (M <= 16 * NT) shared_select_body<16>(p, lb, N, M, kk, wk, sKeys, sDst, sHist, sRedU);
+    else shared_select_body<32>(p, lb, N, M, kk, wk, sKeys, sDst, sHist, sRedU);
 
-// In place: every source row of a chunk is read before any row of the chunk is
-// written, and later chunks read only rows above it (destinations never exceed
-// their source).
-__global__ void __launch_bounds__(256) rkv_shared_compact_kernel(const SharedParams p) {
-    constexpr int NT = 256;
-    const int unit = blockIdx.x;                 // (layer, sequence, head)
-    const int h = unit % p.n_kv;
-    const int lb = unit / p.n_kv;
-    const int b = lb % p.batch;
-    const int l = lb / p.batch;
-    const int N = p.n_eff[b];
-    if (N <= 0) return;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int32_t *dst = p.dst + static_cast<int64_t>(lb) * p.cap;
-    __shared__ uint32_t sFirst[NT / 32];
     uint32_t first = static_cast<uint32_t>(N);
     for (int row = tid; row < N; row += NT)
-        if (dst[row] != row) {
+        if (sDst[row] != row) {
             first = static_cast<uint32_t>(row);
             break;
         }
     first = __reduce_min_sync(kFull, first);
-    if (lane == 0) sFirst[warp] = first;
+    if (lane == 0) sRedU[warp] = first;
     __syncthreads();
-    first = sFirst[0];
+    first = sRedU[0];
 #pragma unroll
-    for (int k = 1; k < NT / 32; ++k) first = min(first, sFirst[k]);
+    for (int k = 1; k < NT / 32; ++k) first = min(first, sRedU[k]);
     const int64_t krow0 = (static_cast<int64_t>(b) * p.n_kv + h) * p.cap;
     uint16_t *kb = p.k[l] + krow0 * kHeadDim;
     uint16_t *vb = p.v[l] + krow0 * kHeadDim;
@@ -151,7 +149,7 @@ __global__ void __launch_bounds__(256) rkv_shared_compact_kernel(const SharedPar
         for (int k = 0; k < PER; ++k) {
             const int idx = tid + k * NT;
             const int row = c0 + (idx >> 4), pc = idx & 15;
-            const int d = row < N ? dst[row] : -1;
+            const int d = row < N ? sDst[row] : -1;
             dd[k] = (d >= 0 && d != row) ? d : -1;
             if (dd[k] >= 0) {
                 kx[k] = __ldcg(reinterpret_cast<const uint4 *>(kb + static_cast<int64_t>(row) * kHeadDim) + pc);
@@ -176,19 +174,14 @@ cudaError_t launch_head_sum(const SharedParams &p, int n_lb, cudaStream_t stream
     return cudaGetLastError();
 }
 
-size_t shared_select_smem(int cap) { return (1024u + 64u + static_cast<size_t>(cap)) * 4u; }
-
-cudaError_t launch_shared_select(const SharedParams &p, int n_lb, cudaStream_t stream) {
-    const size_t smem = shared_select_smem(p.cap);
-    static std::atomic<int> granted{0};
-    const cudaError_t e = ensure_smem_attr(rkv_shared_select_kernel, smem, granted);
-    if (e != cudaSuccess) return e;
-    rkv_shared_select_kernel<<<static_cast<unsigned>(n_lb), kSelThreads, smem, stream>>>(p);
-    return cudaGetLastError();
-}
+size_t shared_select_smem(int cap) { return (1024u + 64u + 2u * static_cast<size_t>(cap)) * 4u; }
 
 cudaError_t launch_shared_compact(const SharedParams &p, int n_units, cudaStream_t stream) {
-    rkv_shared_compact_kernel<<<static_cast<unsigned>(n_units), 256, 0, stream>>>(p);
+    const size_t smem = shared_select_smem(p.cap);
+    static std::atomic<int> granted{0};
+    const cudaError_t e = ensure_smem_attr(rkv_shared_compact_kernel, smem, granted);
+    if (e != cudaSuccess) return e;
+    rkv_shared_compact_kernel<<<static_cast<unsigned>(n_units), kSelThreads, smem, stream>>>(p);
     return cudaGetLastError();
 }
 
