@@ -230,6 +230,24 @@ def _ptr_array(ts: Sequence[torch.Tensor]):
     return arr
 
 
+def _layers(x, name: str):
+    """Per-layer device pointers of bf16 tensors: (ctypes array, n_layers, the shape
+    of one layer).  `x` is one contiguous [n_layers, ...] tensor, whose layer
+    pointers follow from its stride without a view per layer, or a sequence of
+    per-layer tensors."""
+    if isinstance(x, torch.Tensor):
+        _dtype(x, torch.bfloat16, name)
+        if not x.is_contiguous():
+            raise ValueError("tensors passed to librkv must be contiguous")
+        n = int(x.shape[0])
+        base, step = x.data_ptr(), x.stride(0) * x.element_size()
+        return (ctypes.c_void_p * n)(*[base + i * step for i in range(n)]), n, tuple(x.shape[1:])
+    ts = list(x)
+    for t in ts:
+        _dtype(t, torch.bfloat16, name)
+    return _ptr_array(ts), len(ts), tuple(ts[0].shape)
+
+
 def rkv_compress_step(cfg, k_layers, v_layers, q_layers, cur_len, workspace, budgets=None,
                       lambdas=None, kept_out=None, scores_out=None, events=None,
                       cluster_size=0, stream=None):
@@ -243,11 +261,9 @@ def rkv_compress_step(cfg, k_layers, v_layers, q_layers, cur_len, workspace, bud
     cap] fp32 optional; events: (begin, end) torch.cuda.Event recorded around
     the main kernel, or None.
     """
-    k_layers, v_layers, q_layers = list(k_layers), list(v_layers), list(q_layers)
-    n_layers = len(k_layers)
-    batch, _, cap, _ = k_layers[0].shape
-    for t in k_layers + v_layers + q_layers:
-        _dtype(t, torch.bfloat16, "k/v/q")
+    kp, n_layers, (batch, _, cap, _) = _layers(k_layers, "k")
+    vp, _, _ = _layers(v_layers, "v")
+    qp, _, _ = _layers(q_layers, "q")
     _dtype(cur_len, torch.int32, "cur_len"); _dtype(budgets, torch.int32, "budgets")
     _dtype(lambdas, torch.float32, "lambdas"); _dtype(kept_out, torch.int32, "kept_out")
     _dtype(scores_out, torch.float32, "scores_out")
@@ -257,8 +273,7 @@ def rkv_compress_step(cfg, k_layers, v_layers, q_layers, cur_len, workspace, bud
         opts.main_end = events[1].cuda_event
     ws = workspace.numel() * workspace.element_size()
     return _check(_lib.rkv_compress_step(ctypes.byref(cfg), n_layers, batch, cap,
-                                         _ptr_array(k_layers), _ptr_array(v_layers),
-                                         _ptr_array(q_layers), _ptr(budgets), _ptr(lambdas),
+                                         kp, vp, qp, _ptr(budgets), _ptr(lambdas),
                                          _ptr(cur_len), ctypes.byref(opts), _ptr(workspace), ws,
                                          _stream(stream)), "rkv_compress_step",
                   allow_disabled=True)
@@ -267,17 +282,14 @@ def rkv_compress_step(cfg, k_layers, v_layers, q_layers, cur_len, workspace, bud
 def rkv_append_kv(cfg, k_layers, v_layers, k_new_layers, v_new_layers, cur_len, workspace,
                   stream=None):
     """Appends [batch, Hkv, n_new, 128] rows per layer at cur_len, then cur_len += n_new."""
-    k_layers, v_layers = list(k_layers), list(v_layers)
-    k_new_layers, v_new_layers = list(k_new_layers), list(v_new_layers)
-    batch, _, cap, _ = k_layers[0].shape
-    n_new = k_new_layers[0].shape[2]
-    for t in k_layers + v_layers + k_new_layers + v_new_layers:
-        _dtype(t, torch.bfloat16, "k/v")
+    kp, n_layers, (batch, _, cap, _) = _layers(k_layers, "k")
+    vp, _, _ = _layers(v_layers, "v")
+    knp, _, (_, _, n_new, _) = _layers(k_new_layers, "k_new")
+    vnp, _, _ = _layers(v_new_layers, "v_new")
     _dtype(cur_len, torch.int32, "cur_len")
     ws = workspace.numel() * workspace.element_size()
-    return _check(_lib.rkv_append_kv(ctypes.byref(cfg), len(k_layers), batch, cap,
-                                     _ptr_array(k_layers), _ptr_array(v_layers),
-                                     _ptr_array(k_new_layers), _ptr_array(v_new_layers), n_new,
+    return _check(_lib.rkv_append_kv(ctypes.byref(cfg), n_layers, batch, cap,
+                                     kp, vp, knp, vnp, n_new,
                                      _ptr(cur_len), _ptr(workspace), ws, _stream(stream)),
                   "rkv_append_kv")
 
@@ -291,15 +303,13 @@ def rkv_score_shared(cfg, k_layers, q_layers, cur_len, z_sum, workspace, budgets
                      lambdas=None, stream=None):
     """Shared selection, part 1: z_sum [n_layers, batch, cap] fp32 = the sum over
     this call's KV heads of their joint scores (cur_len is only read)."""
-    k_layers, q_layers = list(k_layers), list(q_layers)
-    batch, _, cap, _ = k_layers[0].shape
-    for t in k_layers + q_layers:
-        _dtype(t, torch.bfloat16, "k/q")
+    kp, n_layers, (batch, _, cap, _) = _layers(k_layers, "k")
+    qp, _, _ = _layers(q_layers, "q")
     _dtype(cur_len, torch.int32, "cur_len"); _dtype(budgets, torch.int32, "budgets")
     _dtype(lambdas, torch.float32, "lambdas"); _dtype(z_sum, torch.float32, "z_sum")
     ws = workspace.numel() * workspace.element_size()
-    return _check(_lib.rkv_score_shared(ctypes.byref(cfg), len(k_layers), batch, cap,
-                                        _ptr_array(k_layers), _ptr_array(q_layers), _ptr(budgets),
+    return _check(_lib.rkv_score_shared(ctypes.byref(cfg), n_layers, batch, cap,
+                                        kp, qp, _ptr(budgets),
                                         _ptr(lambdas), _ptr(cur_len), _ptr(z_sum),
                                         _ptr(workspace), ws, _stream(stream)),
                   "rkv_score_shared", allow_disabled=True)
@@ -309,15 +319,13 @@ def rkv_select_compact_shared(cfg, k_layers, v_layers, cur_len, z_sum, workspace
                               kept_out=None, stream=None):
     """Shared selection, part 2 (after z_sum is complete over the ranks): one kept
     set per (layer, sequence), every head of this call compacted in place."""
-    k_layers, v_layers = list(k_layers), list(v_layers)
-    batch, _, cap, _ = k_layers[0].shape
-    for t in k_layers + v_layers:
-        _dtype(t, torch.bfloat16, "k/v")
+    kp, n_layers, (batch, _, cap, _) = _layers(k_layers, "k")
+    vp, _, _ = _layers(v_layers, "v")
     _dtype(cur_len, torch.int32, "cur_len"); _dtype(budgets, torch.int32, "budgets")
     _dtype(z_sum, torch.float32, "z_sum"); _dtype(kept_out, torch.int32, "kept_out")
     ws = workspace.numel() * workspace.element_size()
-    return _check(_lib.rkv_select_compact_shared(ctypes.byref(cfg), len(k_layers), batch, cap,
-                                                 _ptr_array(k_layers), _ptr_array(v_layers),
+    return _check(_lib.rkv_select_compact_shared(ctypes.byref(cfg), n_layers, batch, cap,
+                                                 kp, vp,
                                                  _ptr(budgets), _ptr(cur_len), _ptr(z_sum),
                                                  _ptr(kept_out), _ptr(workspace), ws,
                                                  _stream(stream)),
@@ -335,11 +343,10 @@ def rkv_compress_step_paged(cfg, k_pools, v_pools, q_layers, cur_len, workspace,
     receive the pages each compressed sequence gives back.  kept_out /
     scores_out as in rkv_compress_step with cap = max_blocks * page_rows.
     """
-    k_pools, v_pools, q_layers = list(k_pools), list(v_pools), list(q_layers)
-    num_pages = k_pools[0].shape[0]
+    kp, n_layers, (num_pages, _, _, _) = _layers(k_pools, "k")
+    vp, _, _ = _layers(v_pools, "v")
+    qp, _, _ = _layers(q_layers, "q")
     batch, max_blocks = block_table.shape
-    for t in k_pools + v_pools + q_layers:
-        _dtype(t, torch.bfloat16, "k/v/q")
     for t, n in ((cur_len, "cur_len"), (budgets, "budgets"), (block_table, "block_table"),
                  (freed_pages, "freed_pages"), (n_freed, "n_freed"), (kept_out, "kept_out")):
         _dtype(t, torch.int32, n)
@@ -351,9 +358,8 @@ def rkv_compress_step_paged(cfg, k_pools, v_pools, q_layers, cur_len, workspace,
         opts.main_begin = events[0].cuda_event
         opts.main_end = events[1].cuda_event
     ws = workspace.numel() * workspace.element_size()
-    return _check(_lib.rkv_compress_step_paged(ctypes.byref(cfg), len(k_pools), batch,
-                                               ctypes.byref(pg), _ptr_array(k_pools),
-                                               _ptr_array(v_pools), _ptr_array(q_layers),
+    return _check(_lib.rkv_compress_step_paged(ctypes.byref(cfg), n_layers, batch,
+                                               ctypes.byref(pg), kp, vp, qp,
                                                _ptr(budgets), _ptr(lambdas), _ptr(cur_len),
                                                ctypes.byref(opts), _ptr(workspace), ws,
                                                _stream(stream)),

@@ -574,10 +574,9 @@ rkv_status rkv_compress_step(const rkv_config *cfg, int32_t n_layers, int32_t ba
     p.status = status;
     p.r_ext = red_max ? r_ext : nullptr;
 
-    cudaError_t e = cudaMemsetAsync(ws, 0, kStatusBytes, strm);
-    if (e == cudaSuccess)
-        e = launch_plan(batch, budgets, cfg->budget, cfg->buffer, cfg->window, cap, cur_len, n_eff,
-                        status, strm);
+    // the plan kernel clears the status words first
+    cudaError_t e = launch_plan(batch, budgets, cfg->budget, cfg->buffer, cfg->window, cap, cur_len,
+                                n_eff, status, strm);
     if (red_max && e == cudaSuccess)   // raw r of every candidate: the tcgen05 similarity kernel
         e = launch_gram_layers(cfg, n_layers, batch, cap,
                                const_cast<const rkv_bf16 *const *>(k_layers), n_eff, r_ext, status,
@@ -730,10 +729,9 @@ rkv_status rkv_score_shared(const rkv_config *cfg, int32_t n_layers, int32_t bat
     float *r_ext = reinterpret_cast<float *>(ws + kStatusBytes + align256(static_cast<size_t>(batch) * 4));
     float *z_heads = reinterpret_cast<float *>(ws + base);
     const bool red_max = cfg->redundancy_mode == RKV_RED_MAX;
-    cudaError_t e = cudaMemsetAsync(ws, 0, kStatusBytes, strm);
-    if (e == cudaSuccess)
-        e = launch_plan(batch, budgets, cfg->budget, cfg->buffer, cfg->window, cap,
-                        const_cast<int32_t *>(cur_len), n_eff, status, strm, false);
+    // the plan kernel clears the status words first
+    cudaError_t e = launch_plan(batch, budgets, cfg->budget, cfg->buffer, cfg->window, cap,
+                                const_cast<int32_t *>(cur_len), n_eff, status, strm, false);
     if (red_max && e == cudaSuccess)
         e = launch_gram_layers(cfg, n_layers, batch, cap, k_layers, n_eff, r_ext, status, strm);
     if (e == cudaSuccess)
@@ -770,10 +768,9 @@ rkv_status rkv_select_compact_shared(const rkv_config *cfg, int32_t n_layers, in
     uint32_t *status = reinterpret_cast<uint32_t *>(ws);
     int32_t *n_eff = reinterpret_cast<int32_t *>(ws + kStatusBytes);
     const size_t units = static_cast<size_t>(n_layers) * batch * cfg->n_kv_heads;
-    cudaError_t e = cudaMemsetAsync(ws, 0, kStatusBytes, strm);
-    if (e == cudaSuccess)
-        e = launch_plan(batch, budgets, cfg->budget, cfg->buffer, cfg->window, cap, cur_len, n_eff,
-                        status, strm, true);
+    // the plan kernel clears the status words first
+    cudaError_t e = launch_plan(batch, budgets, cfg->budget, cfg->buffer, cfg->window, cap, cur_len,
+                                n_eff, status, strm, true);
     SharedParams sp;
     std::memset(&sp, 0, sizeof(sp));
     sp.batch = batch;
@@ -838,10 +835,9 @@ rkv_status rkv_compress_step_paged(const rkv_config *cfg, int32_t n_layers, int3
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     uint32_t *status = reinterpret_cast<uint32_t *>(ws);
     int32_t *n_eff = reinterpret_cast<int32_t *>(ws + kStatusBytes);
-    cudaError_t e = cudaMemsetAsync(ws, 0, kStatusBytes, strm);
-    if (e == cudaSuccess)
-        e = launch_plan(batch, budgets, cfg->budget, cfg->buffer, cfg->window, cap, cur_len, n_eff,
-                        status, strm, true);
+    // the plan kernel clears the status words first
+    cudaError_t e = launch_plan(batch, budgets, cfg->budget, cfg->buffer, cfg->window, cap, cur_len,
+                                n_eff, status, strm, true);
     if (e == cudaSuccess)
         e = launch_freed_pages(batch, budgets, cfg->budget, n_eff, pg->block_table, pg->max_blocks,
                                P, pg->freed_pages, pg->n_freed, strm);

@@ -56,34 +56,35 @@ namespace cg = cooperative_groups;
 namespace rkv {
 
 // ----------------------------------------------------------------------------
-// Plan: which sequences are due; snapshot their length; set cur_len = budget.
+// Plan: clear the status words; which sequences are due; snapshot their length;
+// set cur_len = budget.  One CTA, so the clearing precedes every flag it records.
 // ----------------------------------------------------------------------------
-__global__ void rkv_plan_kernel(int batch, const int32_t *__restrict__ budgets,
-                                int32_t budget_cfg, int32_t buffer, int32_t window,
-                                int32_t cap, int32_t *__restrict__ cur_len,
-                                int32_t *__restrict__ n_eff, uint32_t *__restrict__ status,
-                                int update) {
-    const int b = blockIdx.x * blockDim.x + threadIdx.x;
-    if (b >= batch) return;
-    const int32_t bud = budgets ? budgets[b] : budget_cfg;
-    const int32_t n = cur_len[b];
-    // Compression is active only when budget and buffer are both positive.
-    bool due = bud > 0 && buffer > 0 && n >= bud + buffer;
-    if (due && (bud < window || n > cap)) {
-        record_flag(status, kDevFlagBadSeq);
-        due = false;
+__global__ void __launch_bounds__(256) rkv_plan_kernel(int batch, const int32_t *__restrict__ budgets,
+                                                       int32_t budget_cfg, int32_t buffer, int32_t window,
+                                                       int32_t cap, int32_t *__restrict__ cur_len,
+                                                       int32_t *__restrict__ n_eff,
+                                                       uint32_t *__restrict__ status, int update) {
+    for (int i = threadIdx.x; i < static_cast<int>(kStatusBytes / 4); i += blockDim.x) status[i] = 0u;
+    __syncthreads();
+    for (int b = threadIdx.x; b < batch; b += blockDim.x) {
+        const int32_t bud = budgets ? budgets[b] : budget_cfg;
+        const int32_t n = cur_len[b];
+        // Compression is active only when budget and buffer are both positive.
+        bool due = bud > 0 && buffer > 0 && n >= bud + buffer;
+        if (due && (bud < window || n > cap)) {
+            record_flag(status, kDevFlagBadSeq);
+            due = false;
+        }
+        n_eff[b] = due ? n : 0;
+        if (due && update) cur_len[b] = bud;
     }
-    n_eff[b] = due ? n : 0;
-    if (due && update) cur_len[b] = bud;
 }
 
 cudaError_t launch_plan(int batch, const int32_t *budgets, int32_t budget_cfg, int32_t buffer,
                         int32_t window, int32_t cap, int32_t *cur_len, int32_t *n_eff,
                         uint32_t *status, cudaStream_t stream, bool update) {
-    const int threads = 128;
-    const int blocks = (batch + threads - 1) / threads;
-    rkv_plan_kernel<<<blocks, threads, 0, stream>>>(batch, budgets, budget_cfg, buffer, window,
-                                                    cap, cur_len, n_eff, status, update ? 1 : 0);
+    rkv_plan_kernel<<<1, 256, 0, stream>>>(batch, budgets, budget_cfg, buffer, window, cap,
+                                           cur_len, n_eff, status, update ? 1 : 0);
     return cudaGetLastError();
 }
 

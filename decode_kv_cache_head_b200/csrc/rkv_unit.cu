@@ -27,10 +27,10 @@
 //     r_i = (khat_i . S - khat_i . khat_i) / (N - 1) (MEAN) or r_i from the
 //     similarity kernel (MAX).
 //   then the normalisers, the joint scores, the radix select and the
-//   destinations of the kept rows, and the in-place compaction in ascending
-//   chunks of 64 rows (every source row of a chunk is read before any row of
-//   it is written; later chunks only read rows above the current chunk, so the
-//   next chunk's reads overlap this chunk's writes).
+//   destinations of the kept rows, and the in-place compaction of K, then of V,
+//   in ascending chunks of 128 rows (every source row of a chunk is read before
+//   any row of it is written; later chunks only read rows above the current
+//   chunk, so the next chunk's reads overlap this chunk's writes).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -52,7 +52,7 @@ namespace {
 constexpr int kTileRows = 128;
 constexpr uint32_t kStageBytes = 32768u;
 constexpr uint32_t kHalfBytes = 16384u;
-constexpr int kChunkRows = 64;           // compaction chunk (two in flight)
+constexpr int kChunkRows = 128;          // compaction chunk of one tensor (two in flight)
 constexpr float kRescaleLog2 = 8.0f;     // online softmax: rescale past 2^8
 
 // Merges (m2, s2) into (m, s): s = sum of 2^(x - m) over the values seen.
@@ -760,12 +760,11 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
         for (int k = 1; k < NW; ++k) first = min(first, sRedU[k]);
         // Software-pipelined: chunk c + 1 is read before chunk c is written.  Its
         // rows lie above every destination of chunk c, and every read of chunk c
-        // precedes the barrier before chunk c's writes.  The two cache layouts are
-        // compiled separately so the contiguous one carries no page lookups.
-        auto compaction = [&](auto paged_c) {
+        // precedes the barrier before chunk c's writes.  K is moved first, while the
+        // rows the second pass just read are still in L2, then V.  The two cache
+        // layouts are compiled separately so the contiguous one carries no page lookups.
+        auto compaction = [&](auto paged_c, uint16_t *buf) {
             constexpr bool PG = decltype(paged_c)::value;
-            uint16_t *kb = p.k[l];
-            uint16_t *vb = p.v[l];
             auto row_of = [&](int r) -> int64_t {
                 if constexpr (PG)
                     return ((static_cast<int64_t>(sBT[r >> psh]) * p.n_kv + h) << psh) + (r & (P - 1));
@@ -773,52 +772,51 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
                     return krow0 + r;
             };
             constexpr int PER = kChunkRows * 16 / NT;   // 16-byte pieces per thread per chunk
-            auto load = [&](int c0, uint4 (&kx)[PER], uint4 (&vx)[PER], int (&dd)[PER]) {
+            auto load = [&](int c0, uint4 (&x)[PER], int (&dd)[PER]) {
 #pragma unroll
                 for (int k = 0; k < PER; ++k) {
                     const int idx = tid + k * NT;
                     const int row = c0 + (idx >> 4), pc = idx & 15;
                     const int d = row < N ? sDst[row] : -1;
                     dd[k] = (d >= 0 && d != row) ? d : -1;
-                    if (dd[k] >= 0) {
-                        const int64_t src = row_of(row) * kHeadDim;
-                        kx[k] = __ldcg(reinterpret_cast<const uint4 *>(kb + src) + pc);
-                        vx[k] = __ldcg(reinterpret_cast<const uint4 *>(vb + src) + pc);
-                    }
+                    if (dd[k] >= 0) x[k] = __ldcg(reinterpret_cast<const uint4 *>(buf + row_of(row) * kHeadDim) + pc);
                 }
             };
-            auto store = [&](const uint4 (&kx)[PER], const uint4 (&vx)[PER], const int (&dd)[PER]) {
+            auto store = [&](const uint4 (&x)[PER], const int (&dd)[PER]) {
 #pragma unroll
                 for (int k = 0; k < PER; ++k) {
                     if (dd[k] >= 0) {
                         const int pc = (tid + k * NT) & 15;
-                        const int64_t dst = row_of(dd[k]) * kHeadDim;
-                        reinterpret_cast<uint4 *>(kb + dst)[pc] = kx[k];
-                        reinterpret_cast<uint4 *>(vb + dst)[pc] = vx[k];
+                        reinterpret_cast<uint4 *>(buf + row_of(dd[k]) * kHeadDim)[pc] = x[k];
                     }
                 }
             };
-            uint4 ka[PER], va[PER], kc[PER], vc[PER];
+            uint4 xa[PER], xc[PER];
             int da[PER], dc[PER];
             int c0 = static_cast<int>(first);
-            if (c0 < N) load(c0, ka, va, da);
+            if (c0 < N) load(c0, xa, da);
             while (c0 < N) {
                 const int c1 = c0 + kChunkRows;
-                if (c1 < N) load(c1, kc, vc, dc);
+                if (c1 < N) load(c1, xc, dc);
                 __syncthreads();
-                store(ka, va, da);
+                store(xa, da);
                 if (c1 >= N) break;
                 const int c2 = c1 + kChunkRows;
-                if (c2 < N) load(c2, ka, va, da);
+                if (c2 < N) load(c2, xa, da);
                 __syncthreads();
-                store(kc, vc, dc);
+                store(xc, dc);
                 c0 = c2;
             }
         };
-        if (paged)
-            compaction(std::true_type{});
-        else
-            compaction(std::false_type{});
+        uint16_t *kb = p.k[l];
+        uint16_t *vb = p.v[l];
+        if (paged) {
+            compaction(std::true_type{}, kb);
+            compaction(std::true_type{}, vb);
+        } else {
+            compaction(std::false_type{}, kb);
+            compaction(std::false_type{}, vb);
+        }
     }
 
     __syncthreads();
