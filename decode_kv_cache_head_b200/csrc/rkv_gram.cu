@@ -53,6 +53,24 @@ struct GramSmem {
     uint32_t tmem;
 };
 
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// max(best, c[0..31]) as a tree of three-input maxima.
+__device__ __forceinline__ float max_of_32(float best, const float (&c)[32]) {
+    float t[11];
+#pragma unroll
+    for (int q = 0; q < 10; ++q) t[q] = fmax3(c[3 * q], c[3 * q + 1], c[3 * q + 2]);
+    t[10] = fmaxf(c[30], c[31]);
+    const float u0 = fmax3(t[0], t[1], t[2]), u1 = fmax3(t[3], t[4], t[5]);
+    const float u2 = fmax3(t[6], t[7], t[8]), u3 = fmax3(t[9], t[10], best);
+    return fmax3(u0, u1, fmaxf(u2, u3));
+}
+
 __device__ __forceinline__ void named_sync_epilogue() {
     asm volatile("bar.sync 1, 256;" ::: "memory");
 }
@@ -183,8 +201,7 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
                     c[4 * q] = a.x; c[4 * q + 1] = a.y; c[4 * q + 2] = bb.x; c[4 * q + 3] = bb.y;
                 }
                 if (clean) {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) best = fmaxf(best, c[e]);
+                    best = max_of_32(best, c);
                 } else {
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
