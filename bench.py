@@ -80,10 +80,20 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
-def kernel_source_digest():
+# The sources each timed kernel is compiled from (its file and the headers it includes).
+KERNEL_SOURCES = {
+    "rkv_unit_kernel": ("rkv_unit.cu", "rkv_block.cuh", "rkv_internal.h", "rkv_post.cuh",
+                        "rkv_ptx.cuh"),
+    "rkv_step_kernel": ("rkv_step.cu", "rkv_block.cuh", "rkv_internal.h", "rkv_post.cuh",
+                        "rkv_ptx.cuh"),
+}
+
+
+def kernel_source_digest(kernel):
+    """sha256 (16 hex digits) of the kernel's own sources."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "decode_kv_cache_head_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(KERNEL_SOURCES[kernel]):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
@@ -102,7 +112,7 @@ def profiled_traffic(kernel, workload, units_per_launch):
             if ":" in line and not line.startswith("#"):
                 k, v = line.split(":", 1)
                 kv[k.strip()] = v.strip()
-    if kv.get("kernel_source_sha256_16") != kernel_source_digest():
+    if kv.get("kernel_source_sha256_16") != kernel_source_digest(kernel):
         return None
     try:
         per_unit = float(kv["dram_bytes_per_unit"])
@@ -407,7 +417,7 @@ def run_rkv(args, w, red_mode):
                 "frac": achieved / peak, "traffic": profiled_traffic(kernel_name, w.name, units),
                 "kernel": kernel_name, "kernel_us_per_launch": kern_ms * 1e3,
                 "algorithmic_bytes_per_launch": alg_bytes, "peak_source": peak_kind,
-                "kernel_source_sha256_16": kernel_source_digest(),
+                "kernel_source_sha256_16": kernel_source_digest(kernel_name),
                 "cluster_size": shape[0], "rows_per_cta": shape[1], "smem_per_cta": shape[2]}
 
     cpu = None
