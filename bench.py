@@ -53,7 +53,7 @@ def parse_args():
     ap.add_argument("--impl", default="rkv", choices=["rkv", "reference"])
     ap.add_argument("--workload", default="llama3_8b_step", choices=sorted(WORKLOADS))
     ap.add_argument("--redundancy", default="mean", choices=["mean", "max"])
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cluster-size", type=int, default=0,
                     help="CTAs per unit: 0 = the library's choice, 1 = one CTA per unit, "
@@ -377,39 +377,67 @@ def run_rkv(args, w, red_mode):
     ms_per_step = elapsed_ms / args.steps
     value = world * token_heads / (ms_per_step / 1e3)
 
-    # end to end through host buffers: H2D of the inputs, the step, D2H of the result
+    # end to end through host buffers: every step copies its inputs host -> device, runs
+    # the step and copies its result device -> host.  Consecutive steps overlap: two
+    # device buffer sets, the copies in on one stream and out on another, so the H2D of
+    # step i + 1 and the D2H of step i - 1 run while step i computes (the two copy
+    # directions use the link at the same time).
     e2e = None
-    # the end-to-end leg pins two host copies of the caches: only for caches of a few GB
+    # the end-to-end leg pins host copies of the caches: only for caches of a few GB
     if args.e2e_steps > 0 and rep_bytes <= 4 * 1024 ** 3:
         hK, hV, hQ = K0.cpu().pin_memory(), V0.cpu().pin_memory(), Q.cpu().pin_memory()
         hc = cur0.cpu().pin_memory()
         oK, oV, oc = torch.empty_like(hK).pin_memory(), torch.empty_like(hV).pin_memory(), \
             torch.empty_like(hc).pin_memory()
-        dK, dV, dQ, dc = torch.empty_like(K0), torch.empty_like(V0), torch.empty_like(Q), \
-            torch.empty_like(cur0)
+        sets = [(torch.empty_like(K0), torch.empty_like(V0), torch.empty_like(Q),
+                 torch.empty_like(cur0)) for _ in range(2)]
+        s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_step = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+        used = [False, False]
 
-        def e2e_step():
-            dK.copy_(hK, non_blocking=True); dV.copy_(hV, non_blocking=True)
-            dQ.copy_(hQ, non_blocking=True); dc.copy_(hc, non_blocking=True)
+        def e2e_step(i):
+            k = i % 2
+            dK, dV, dQ, dc = sets[k]
+            with torch.cuda.stream(s_in):
+                if used[k]:
+                    s_in.wait_event(ev_out[k])      # this set's previous result is out
+                dK.copy_(hK, non_blocking=True); dV.copy_(hV, non_blocking=True)
+                dQ.copy_(hQ, non_blocking=True); dc.copy_(hc, non_blocking=True)
+                ev_in[k].record(s_in)
+            stream.wait_event(ev_in[k])
             rkv.rkv_compress_step(cfg, dK, dV, dQ, dc, ws, budgets=budgets,
                                   cluster_size=args.cluster_size, stream=stream)
-            oK.copy_(dK, non_blocking=True); oV.copy_(dV, non_blocking=True)
-            oc.copy_(dc, non_blocking=True)
+            ev_step[k].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_step[k])
+                oK.copy_(dK, non_blocking=True); oV.copy_(dV, non_blocking=True)
+                oc.copy_(dc, non_blocking=True)
+                ev_out[k].record(s_out)
+            used[k] = True
 
-        e2e_step()
+        for i in range(2):
+            e2e_step(i)
         torch.cuda.synchronize()
         rdist.barrier(dev)
+        torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
+        s_in.wait_event(a)
+        for i in range(args.e2e_steps):
+            e2e_step(i)
+        for k in range(2):
+            stream.wait_event(ev_out[k])
         b.record(stream)
         torch.cuda.synchronize()
+        assert rkv.rkv_workspace_status(ws) == 0
         e_ms = rdist.max_over_ranks([a.elapsed_time(b) / args.e2e_steps], dev)[0]
         h2d = sum(t.numel() * t.element_size() for t in (hK, hV, hQ, hc))
         d2h = sum(t.numel() * t.element_size() for t in (oK, oV, oc))
         e2e = {"value": world * token_heads / (e_ms / 1e3), "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms,
+               "overlap": "copies of consecutive steps overlap (two buffer sets, copy streams)"}
 
     peak, peak_kind = measured_peaks()
     achieved = alg_bytes / (kern_ms / 1e3) / 1e9
