@@ -43,8 +43,8 @@ __global__ void __launch_bounds__(256) rkv_gather_kernel(
     }
     const int64_t so = h * head_stride + static_cast<int64_t>(s) * kHeadDim + c * 8;
     const int64_t d = h * head_stride + static_cast<int64_t>(t) * kHeadDim + c * 8;
-    *reinterpret_cast<uint4 *>(k_dst + d) = __ldg(reinterpret_cast<const uint4 *>(k_src + so));
-    *reinterpret_cast<uint4 *>(v_dst + d) = __ldg(reinterpret_cast<const uint4 *>(v_src + so));
+    __stcs(reinterpret_cast<uint4 *>(k_dst + d), __ldg(reinterpret_cast<const uint4 *>(k_src + so)));
+    __stcs(reinterpret_cast<uint4 *>(v_dst + d), __ldg(reinterpret_cast<const uint4 *>(v_src + so)));
 }
 
 __global__ void __launch_bounds__(kThreads, 1) rkv_compact_inplace_kernel(
@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(kThreads, 1) rkv_compact_inplace_kernel(
         if (s < 0 || s >= n_tokens || s == t) continue;
         const uint4 x = *reinterpret_cast<const uint4 *>(stage + i * 512 + c * 16);
         uint16_t *dst = (c < 16 ? kh : vh) + static_cast<int64_t>(t) * kHeadDim + (c & 15) * 8;
-        *reinterpret_cast<uint4 *>(dst) = x;
+        __stcs(reinterpret_cast<uint4 *>(dst), x);
     }
 }
 

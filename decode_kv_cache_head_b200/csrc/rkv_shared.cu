@@ -161,8 +161,8 @@ __global__ void __launch_bounds__(kSelThreads) rkv_shared_compact_kernel(const S
         for (int k = 0; k < PER; ++k) {
             if (dd[k] >= 0) {
                 const int pc = (tid + k * NT) & 15;
-                reinterpret_cast<uint4 *>(kb + static_cast<int64_t>(dd[k]) * kHeadDim)[pc] = kx[k];
-                reinterpret_cast<uint4 *>(vb + static_cast<int64_t>(dd[k]) * kHeadDim)[pc] = vx[k];
+                __stcs(reinterpret_cast<uint4 *>(kb + static_cast<int64_t>(dd[k]) * kHeadDim) + pc, kx[k]);
+                __stcs(reinterpret_cast<uint4 *>(vb + static_cast<int64_t>(dd[k]) * kHeadDim) + pc, vx[k]);
             }
         }
     }

@@ -613,8 +613,8 @@ __global__ void __launch_bounds__(kStepThreads, 2) rkv_step_kernel(const __grid_
                 const uint4 kx = *reinterpret_cast<const uint4 *>(sK + (c >> 3) * p.rp * 128 +
                                                                   sw128_offset(row, c & 7));
                 const uint4 vx = *reinterpret_cast<const uint4 *>(sV + row * 256 + c * 16);
-                *reinterpret_cast<uint4 *>(kdst + static_cast<int64_t>(d) * kHeadDim + c * 8) = kx;
-                *reinterpret_cast<uint4 *>(vdst + static_cast<int64_t>(d) * kHeadDim + c * 8) = vx;
+                __stcs(reinterpret_cast<uint4 *>(kdst + static_cast<int64_t>(d) * kHeadDim + c * 8), kx);
+                __stcs(reinterpret_cast<uint4 *>(vdst + static_cast<int64_t>(d) * kHeadDim + c * 8), vx);
             }
         }
     }

@@ -782,12 +782,14 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
                     if (dd[k] >= 0) x[k] = __ldcg(reinterpret_cast<const uint4 *>(buf + row_of(row) * kHeadDim) + pc);
                 }
             };
+            // streaming (evict-first) stores: the moved rows are not read again by this
+            // step, so they leave L2 early instead of displacing the rows still to be read
             auto store = [&](const uint4 (&x)[PER], const int (&dd)[PER]) {
 #pragma unroll
                 for (int k = 0; k < PER; ++k) {
                     if (dd[k] >= 0) {
                         const int pc = (tid + k * NT) & 15;
-                        reinterpret_cast<uint4 *>(buf + row_of(dd[k]) * kHeadDim)[pc] = x[k];
+                        __stcs(reinterpret_cast<uint4 *>(buf + row_of(dd[k]) * kHeadDim) + pc, x[k]);
                     }
                 }
             };
