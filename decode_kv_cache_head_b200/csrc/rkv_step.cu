@@ -64,6 +64,8 @@ __global__ void __launch_bounds__(256) rkv_plan_kernel(int batch, const int32_t 
                                                        int32_t cap, int32_t *__restrict__ cur_len,
                                                        int32_t *__restrict__ n_eff,
                                                        uint32_t *__restrict__ status, int update) {
+    // the kernel that follows may be scheduled now; it waits for this one to finish
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     for (int i = threadIdx.x; i < static_cast<int>(kStatusBytes / 4); i += blockDim.x) status[i] = 0u;
     __syncthreads();
     for (int b = threadIdx.x; b < batch; b += blockDim.x) {

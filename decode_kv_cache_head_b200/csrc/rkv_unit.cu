@@ -123,6 +123,9 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
     const int l = unit / (p.n_kv * p.batch);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wg = warp >> 2;
 
+    // launched as a programmatic dependent of the plan kernel: nothing it wrote (or that
+    // ran before it) is read before this wait
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int N = p.n_eff[b];
     if (N <= 0) return;   // not due
 
@@ -834,8 +837,19 @@ static cudaError_t launch_unit_t(const UnitParams &p, int n_units, size_t smem, 
     static std::atomic<int> granted{0};
     const cudaError_t e = ensure_smem_attr(kern, smem, granted);
     if (e != cudaSuccess) return e;
-    kern<<<static_cast<unsigned>(n_units), kUnitThreads, smem, stream>>>(p);
-    return cudaGetLastError();
+    // programmatic dependent launch: the CTAs may be scheduled while the preceding
+    // kernel (the plan) finishes, and wait for it on the device
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(n_units), 1, 1);
+    cfg.blockDim = dim3(kUnitThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
 cudaError_t launch_unit(const UnitParams &p, int n_units, int nqp, size_t smem, cudaStream_t stream) {
