@@ -80,6 +80,17 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def measured_bf16_tflops():
+    """Dense bf16 tensor peak: the measured burst figure (kernels of a few hundred
+    microseconds, timed inside short steps), else the fallback."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured (burst)"
+    return 1590.0, "fallback (burst)"
+
+
 # The sources each timed kernel is compiled from (its file and the headers it includes).
 KERNEL_SOURCES = {
     "rkv_unit_kernel": ("rkv_unit.cu", "rkv_block.cuh", "rkv_internal.h", "rkv_post.cuh",
@@ -290,10 +301,10 @@ def run_rkv(args, w, red_mode):
     kernel_name = "rkv_unit_kernel" if shape[0] == 1 else "rkv_step_kernel"
     stream = torch.cuda.current_stream()
 
-    def step(Kr, Vr, cr, events=None, kept=None):
+    def step(Kr, Vr, cr, events=None, kept=None, sim_events=None):
         rkv.rkv_compress_step(cfg, Kr, Vr, Q, cr, ws, budgets=budgets, kept_out=kept,
                               cluster_size=args.cluster_size,
-                              events=events, stream=stream)
+                              events=events, stream=stream, sim_events=sim_events)
 
     # exact moved-row count (rows whose destination differs from their source)
     kept = torch.full((L, B, H, cap), -1, dtype=torch.int32, device=dev)
@@ -323,9 +334,12 @@ def run_rkv(args, w, red_mode):
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
+    # MAX redundancy: the similarity kernel is timed too (it is the longer kernel there)
+    ev_sim = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)] if red_mode == 1 else None
     st = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
-    for a, b in ev:        # materialise the events before handing them to the library
+    for a, b in ev + (ev_sim or []):   # materialise the events before handing them to the library
         a.record(stream); b.record(stream)
 
     def restore(r):
@@ -345,7 +359,8 @@ def run_rkv(args, w, red_mode):
             if not fits:
                 restore(reps[0])
                 st[i][0].record(stream)
-            step(*reps[args.warmup + i if fits else 0], events=ev[i] if kernel_events else None)
+            step(*reps[args.warmup + i if fits else 0], events=ev[i] if kernel_events else None,
+                 sim_events=ev_sim[i] if (kernel_events and ev_sim) else None)
             if not fits:
                 st[i][1].record(stream)
         t_stop.record(stream)
@@ -447,6 +462,24 @@ def run_rkv(args, w, red_mode):
                 "algorithmic_bytes_per_launch": alg_bytes, "peak_source": peak_kind,
                 "kernel_source_sha256_16": kernel_source_digest(kernel_name),
                 "cluster_size": shape[0], "rows_per_cta": shape[1], "smem_per_cta": shape[2]}
+    roofline_unit = None
+    if ev_sim:
+        # MAX redundancy: the similarity kernel is the dominant one.  Algorithmic flops are
+        # the symmetric Gram N (N - 1) D per unit; the kernel computes every (row block,
+        # column tile) pair of 128 x 128 x 128, 2 * 128^3 flops each.
+        sim_ms = sum(a.elapsed_time(b) for a, b in ev_sim) / args.steps
+        sim_ms = rdist.max_over_ranks([sim_ms], dev)[0]
+        n_seq = [w.budget_of(b) + w.buffer for b in range(B)]
+        alg_flops = L * H * sum(n * (n - 1) * D for n in n_seq)
+        exe_flops = L * H * sum(-(-(n - w.window) // 128) * -(-n // 128) * 2 * 128 ** 3 for n in n_seq)
+        tpeak, tkind = measured_bf16_tflops()
+        t_ach = alg_flops / (sim_ms / 1e3) / 1e12
+        roofline_unit = roofline
+        roofline = {"bound": "tensor", "achieved": t_ach, "peak": tpeak, "unit": "TFLOP/s",
+                    "frac": t_ach / tpeak, "traffic": None, "kernel": "rkv_gram_max_kernel",
+                    "kernel_us_per_launch": sim_ms * 1e3, "algorithmic_flops_per_launch": alg_flops,
+                    "executed_flops_per_launch": exe_flops,
+                    "executed_tflops": exe_flops / (sim_ms / 1e3) / 1e12, "peak_source": tkind}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -470,6 +503,7 @@ def run_rkv(args, w, red_mode):
         "data": "synthetic", "config": workload_config(w, red_mode, args),
         "e2e": e2e, "gpu_launches": args.steps * (1 + n_main_launches),
         "roofline": roofline, "cpu_baseline": cpu, "clocks": clocks,
+        **({"roofline_unit_kernel": roofline_unit} if roofline_unit else {}),
         "token_heads_per_step_per_gpu": token_heads,
     }
     print(json.dumps(line), flush=True)

@@ -66,6 +66,8 @@ class rkv_step_options(ctypes.Structure):
         ("main_begin", ctypes.c_void_p),
         ("main_end", ctypes.c_void_p),
         ("cluster_size", ctypes.c_int32),
+        ("sim_begin", ctypes.c_void_p),
+        ("sim_end", ctypes.c_void_p),
     ]
 
 
@@ -250,7 +252,7 @@ def _layers(x, name: str):
 
 def rkv_compress_step(cfg, k_layers, v_layers, q_layers, cur_len, workspace, budgets=None,
                       lambdas=None, kept_out=None, scores_out=None, events=None,
-                      cluster_size=0, stream=None):
+                      cluster_size=0, stream=None, sim_events=None):
     """The whole step over all layers of a batch, in place.
 
     k_layers / v_layers: sequences of [batch, Hkv, cap, 128] bf16 tensors (one
@@ -259,7 +261,8 @@ def rkv_compress_step(cfg, k_layers, v_layers, q_layers, cur_len, workspace, bud
     budgets [batch] int32 / lambdas [batch] fp32 or None; kept_out
     [n_layers, batch, Hkv, cap] int32 and scores_out [n_layers, batch, Hkv, 4,
     cap] fp32 optional; events: (begin, end) torch.cuda.Event recorded around
-    the main kernel, or None.
+    the main kernel, or None; sim_events: the same around the similarity kernel
+    (MAX redundancy).
     """
     kp, n_layers, (batch, _, cap, _) = _layers(k_layers, "k")
     vp, _, _ = _layers(v_layers, "v")
@@ -271,6 +274,9 @@ def rkv_compress_step(cfg, k_layers, v_layers, q_layers, cur_len, workspace, bud
     if events is not None:
         opts.main_begin = events[0].cuda_event
         opts.main_end = events[1].cuda_event
+    if sim_events is not None:
+        opts.sim_begin = sim_events[0].cuda_event
+        opts.sim_end = sim_events[1].cuda_event
     ws = workspace.numel() * workspace.element_size()
     return _check(_lib.rkv_compress_step(ctypes.byref(cfg), n_layers, batch, cap,
                                          kp, vp, qp, _ptr(budgets), _ptr(lambdas),

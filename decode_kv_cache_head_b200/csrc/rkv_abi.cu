@@ -226,9 +226,12 @@ cudaError_t launch_unit_layers(const rkv_config *cfg, int32_t n_layers, int32_t 
 }
 
 // MAX mode: raw r of every candidate of every due unit, by the similarity kernel.
+// sim_begin / sim_end (or null): recorded before the first and after the last launch
+// of the similarity kernel.
 cudaError_t launch_gram_layers(const rkv_config *cfg, int32_t n_layers, int32_t batch, int32_t cap,
                                const rkv_bf16 *const *k_layers, const int32_t *n_eff, float *r_ext,
-                               uint32_t *status, cudaStream_t strm) {
+                               uint32_t *status, cudaStream_t strm, cudaEvent_t sim_begin = nullptr,
+                               cudaEvent_t sim_end = nullptr) {
     GramParams *gp = new GramParams();
     std::memset(gp, 0, sizeof(*gp));
     gp->batch = batch;
@@ -252,7 +255,9 @@ cudaError_t launch_gram_layers(const rkv_config *cfg, int32_t n_layers, int32_t 
                                 static_cast<uint64_t>(batch) * cfg->n_kv_heads * cap, 128))
                 e = cudaErrorInvalidValue;
         }
-        if (e == cudaSuccess) e = launch_gram_max(*gp, nl * batch * cfg->n_kv_heads, strm);
+        if (e == cudaSuccess)
+            e = launch_gram_max(*gp, nl * batch * cfg->n_kv_heads, strm, l0 == 0 ? sim_begin : nullptr,
+                                l0 + nl >= n_layers ? sim_end : nullptr);
     }
     delete gp;
     return e;
@@ -580,7 +585,8 @@ rkv_status rkv_compress_step(const rkv_config *cfg, int32_t n_layers, int32_t ba
     if (red_max && e == cudaSuccess)   // raw r of every candidate: the tcgen05 similarity kernel
         e = launch_gram_layers(cfg, n_layers, batch, cap,
                                const_cast<const rkv_bf16 *const *>(k_layers), n_eff, r_ext, status,
-                               strm);
+                               strm, opts ? reinterpret_cast<cudaEvent_t>(opts->sim_begin) : nullptr,
+                               opts ? reinterpret_cast<cudaEvent_t>(opts->sim_end) : nullptr);
     if (e == cudaSuccess && opts && opts->main_begin)
         e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->main_begin), strm);
     if (unit_path && e == cudaSuccess)

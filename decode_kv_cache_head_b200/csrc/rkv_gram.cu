@@ -262,7 +262,8 @@ __global__ void __launch_bounds__(256) rkv_inv_norm_kernel(const __grid_constant
 
 size_t gram_smem_bytes() { return sizeof(GramSmem) + 1024; }
 
-cudaError_t launch_gram_max(const GramParams &p, int n_units, cudaStream_t stream) {
+cudaError_t launch_gram_max(const GramParams &p, int n_units, cudaStream_t stream,
+                            cudaEvent_t before_gram, cudaEvent_t after_gram) {
     const size_t smem = gram_smem_bytes();
     static std::atomic<int> granted{0};
     cudaError_t e = ensure_smem_attr(rkv_gram_max_kernel, smem, granted);
@@ -270,9 +271,12 @@ cudaError_t launch_gram_max(const GramParams &p, int n_units, cudaStream_t strea
     const int nchunk = (p.cap + 63) / 64;
     rkv_inv_norm_kernel<<<static_cast<unsigned>(n_units * nchunk), 256, 0, stream>>>(p, nchunk);
     e = cudaGetLastError();
+    if (e == cudaSuccess && before_gram) e = cudaEventRecord(before_gram, stream);
     if (e != cudaSuccess) return e;
     rkv_gram_max_kernel<<<n_units * p.nblk, kGramThreads, smem, stream>>>(p);
-    return cudaGetLastError();
+    e = cudaGetLastError();
+    if (e == cudaSuccess && after_gram) e = cudaEventRecord(after_gram, stream);
+    return e;
 }
 
 }  // namespace rkv

@@ -241,7 +241,10 @@ struct alignas(64) GramParams {
     float *inv;              // [units][cap] 1 / max(||k||, 1e-12), written by the first pass
     uint32_t *status;
 };
-cudaError_t launch_gram_max(const GramParams &p, int n_units, cudaStream_t stream);
+// before_gram / after_gram (or null): recorded around the similarity kernel itself
+// (after the inverse-norm pass).
+cudaError_t launch_gram_max(const GramParams &p, int n_units, cudaStream_t stream,
+                            cudaEvent_t before_gram = nullptr, cudaEvent_t after_gram = nullptr);
 
 struct AppendParams {
     uint16_t *k[kMaxLayersPerLaunch];

@@ -109,6 +109,9 @@ typedef struct {
     int32_t cluster_size;    /* CTAs per unit: 0 = automatic, 1 = one CTA per unit (K
                                 streamed twice through shared memory), else a cluster of
                                 2, 4, 8 or 16 CTAs that holds the unit's K on chip */
+    rkv_event_t sim_begin;   /* MAX redundancy, if not NULL: recorded on `stream` just before
+                                the first launch of the similarity kernel */
+    rkv_event_t sim_end;     /* MAX redundancy, if not NULL: recorded just after its last */
 } rkv_step_options;
 
 /* Human-readable name of a status code (static storage). */
