@@ -35,6 +35,8 @@ constexpr int kChunkRows = 128;
 // Every entry of z_sum is written: the head sum for candidates of due
 // sequences, 0 elsewhere (so that an all-reduce over ranks sees defined data).
 __global__ void __launch_bounds__(256) rkv_head_sum_kernel(const SharedParams p) {
+    // a programmatic dependent of the scoring kernel: wait for it before reading
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int nch = (p.cap + 255) / 256;
     const int lb = blockIdx.x / nch;                 // layer * batch + sequence
     const int b = lb % p.batch;
@@ -104,6 +106,8 @@ __device__ __forceinline__ void shared_select_body(const SharedParams &p, int lb
 // above it (destinations never exceed their source).
 __global__ void __launch_bounds__(kSelThreads) rkv_shared_compact_kernel(const SharedParams p) {
     constexpr int NT = kSelThreads;
+    // a programmatic dependent of the kernel before it: wait for it before reading
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     extern __shared__ uint32_t sel_smem[];
     const int unit = blockIdx.x;                 // (layer, sequence, head)
     const int h = unit % p.n_kv;
@@ -168,10 +172,27 @@ __global__ void __launch_bounds__(kSelThreads) rkv_shared_compact_kernel(const S
     }
 }
 
+// Launches `kern` as a programmatic dependent of the kernel before it on `stream`: its
+// CTAs may be scheduled while that kernel finishes, and wait for it on the device.
+template <class Kern>
+static cudaError_t launch_dependent(Kern kern, unsigned blocks, unsigned threads, size_t smem,
+                                    cudaStream_t stream, const SharedParams &p) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(blocks, 1, 1);
+    cfg.blockDim = dim3(threads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
 cudaError_t launch_head_sum(const SharedParams &p, int n_lb, cudaStream_t stream) {
     const unsigned blocks = static_cast<unsigned>(n_lb) * static_cast<unsigned>((p.cap + 255) / 256);
-    rkv_head_sum_kernel<<<blocks, 256, 0, stream>>>(p);
-    return cudaGetLastError();
+    return launch_dependent(rkv_head_sum_kernel, blocks, 256u, 0, stream, p);
 }
 
 size_t shared_select_smem(int cap) { return (1024u + 64u + 2u * static_cast<size_t>(cap)) * 4u; }
@@ -181,8 +202,8 @@ cudaError_t launch_shared_compact(const SharedParams &p, int n_units, cudaStream
     static std::atomic<int> granted{0};
     const cudaError_t e = ensure_smem_attr(rkv_shared_compact_kernel, smem, granted);
     if (e != cudaSuccess) return e;
-    rkv_shared_compact_kernel<<<static_cast<unsigned>(n_units), kSelThreads, smem, stream>>>(p);
-    return cudaGetLastError();
+    return launch_dependent(rkv_shared_compact_kernel, static_cast<unsigned>(n_units),
+                            static_cast<unsigned>(kSelThreads), smem, stream, p);
 }
 
 }  // namespace rkv
