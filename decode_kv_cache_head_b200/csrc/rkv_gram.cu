@@ -81,6 +81,8 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
     extern __shared__ uint8_t smem_raw[];
     GramSmem &S = *reinterpret_cast<GramSmem *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    // a programmatic dependent of the inverse-norm pass: wait for it before reading
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int unit = blockIdx.x / p.nblk, bi = blockIdx.x % p.nblk;
     const int h = unit % p.n_kv;
@@ -231,6 +233,8 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
 // (16 lanes x 8 columns), 64 rows per CTA.
 __global__ void __launch_bounds__(256) rkv_inv_norm_kernel(const __grid_constant__ GramParams p,
                                                            int nchunk) {
+    // a programmatic dependent of the plan kernel: wait for it before reading
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int unit = blockIdx.x / nchunk, chunk = blockIdx.x % nchunk;
     const int h = unit % p.n_kv;
     const int b = (unit / p.n_kv) % p.batch;
@@ -269,12 +273,24 @@ cudaError_t launch_gram_max(const GramParams &p, int n_units, cudaStream_t strea
     cudaError_t e = ensure_smem_attr(rkv_gram_max_kernel, smem, granted);
     if (e != cudaSuccess) return e;
     const int nchunk = (p.cap + 63) / 64;
-    rkv_inv_norm_kernel<<<static_cast<unsigned>(n_units * nchunk), 256, 0, stream>>>(p, nchunk);
-    e = cudaGetLastError();
+    // both launched as programmatic dependents of the kernel before them: their CTAs may
+    // be scheduled while it finishes, and wait for it on the device
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(n_units * nchunk), 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, rkv_inv_norm_kernel, p, nchunk);
     if (e == cudaSuccess && before_gram) e = cudaEventRecord(before_gram, stream);
     if (e != cudaSuccess) return e;
-    rkv_gram_max_kernel<<<n_units * p.nblk, kGramThreads, smem, stream>>>(p);
-    e = cudaGetLastError();
+    cfg.gridDim = dim3(static_cast<unsigned>(n_units * p.nblk), 1, 1);
+    cfg.blockDim = dim3(kGramThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    e = cudaLaunchKernelEx(&cfg, rkv_gram_max_kernel, p);
     if (e == cudaSuccess && after_gram) e = cudaEventRecord(after_gram, stream);
     return e;
 }
