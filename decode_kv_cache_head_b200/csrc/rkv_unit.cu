@@ -229,10 +229,12 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
         tma_last = g;
         const int tt = g < T ? g : g - T;
         uint8_t *stg = sStage + (g & 1) * kStageBytes;
+        // K tiles are kept in L2 (evict last): pass 2 and the compaction read them again
+        const uint64_t pol = policy_evict_last();
         if (!paged) {
             const int32_t y = static_cast<int32_t>(krow0 + tt * kTileRows);
-            tma_load_2d(stg, mk, &full[g & 1], 0, y);
-            tma_load_2d(stg + kHalfBytes, mk, &full[g & 1], 64, y);
+            tma_load_2d_hint(stg, mk, &full[g & 1], 0, y, pol);
+            tma_load_2d_hint(stg + kHalfBytes, mk, &full[g & 1], 64, y, pol);
         } else {
             // one box per page; pages past the sequence's last read as zeros (a row
             // coordinate below the pool)
@@ -240,8 +242,8 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
             for (int j = 0; j < kTileRows / P; ++j) {
                 const int pg = tt * (kTileRows / P) + j;
                 const int32_t y = pg < npg ? static_cast<int32_t>(prow(pg * P)) : -P;
-                tma_load_2d(stg + j * P * 128, mk, &full[g & 1], 0, y);
-                tma_load_2d(stg + kHalfBytes + j * P * 128, mk, &full[g & 1], 64, y);
+                tma_load_2d_hint(stg + j * P * 128, mk, &full[g & 1], 0, y, pol);
+                tma_load_2d_hint(stg + kHalfBytes + j * P * 128, mk, &full[g & 1], 64, y, pol);
             }
         }
     };
