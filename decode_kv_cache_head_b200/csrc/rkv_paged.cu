@@ -18,6 +18,8 @@ __global__ void rkv_freed_pages_kernel(int batch, const int32_t *__restrict__ bu
                                        const int32_t *__restrict__ block_table, int max_blocks,
                                        int page_rows, int32_t *__restrict__ freed,
                                        int32_t *__restrict__ n_freed) {
+    // a programmatic dependent of the step kernel: wait for it before reading or writing
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int b = blockIdx.x * blockDim.x + threadIdx.x;
     if (b >= batch) return;
     const int N = n_eff[b];
@@ -37,9 +39,19 @@ cudaError_t launch_freed_pages(int batch, const int32_t *budgets, int32_t budget
                                const int32_t *n_eff, const int32_t *block_table, int max_blocks,
                                int page_rows, int32_t *freed, int32_t *n_freed,
                                cudaStream_t stream) {
-    rkv_freed_pages_kernel<<<(batch + 127) / 128, 128, 0, stream>>>(
-        batch, budgets, budget_cfg, n_eff, block_table, max_blocks, page_rows, freed, n_freed);
-    return cudaGetLastError();
+    // launched as a programmatic dependent of the kernel before it: its CTAs may be
+    // scheduled while that kernel finishes, and wait for it on the device
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>((batch + 127) / 128), 1, 1);
+    cfg.blockDim = dim3(128, 1, 1);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, rkv_freed_pages_kernel, batch, budgets, budget_cfg, n_eff,
+                              block_table, max_blocks, page_rows, freed, n_freed);
 }
 
 }  // namespace rkv
