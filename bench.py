@@ -2,11 +2,14 @@
 
 One step = one rkv_compress_step call over every layer, sequence and KV head
 of the workload (plan kernel + fused per-unit kernel), on a cache that is due
-for compression.  The step compacts the cache in place, so every warm-up and
-timed step gets its own pristine replica of the inputs, materialised in HBM
-before timing; each replica (K+V, 151 MB for the Llama3-8B-shaped step) is
-larger than the 126 MB L2, and a 256 MB buffer is written after the replicas
-are made, so every step starts from a cold L2.
+for compression.  The default workload is the largest single-GPU one, the
+ragged batch (64 sequences x 32 layers x 8 KV heads, budgets 512..2048 + 128,
+lambda cycling 0 / 0.1 / 1 over the sequences).  The step compacts the cache
+in place, so every warm-up and timed step starts from a pristine copy of the
+inputs in HBM: its own replica when the replicas fit in memory, else one
+working copy restored (outside the per-step events) before every step.  Every
+replica is larger than the 126 MB L2, and a 256 MB buffer is written before
+each timed region (and after each restore), so steps start from a cold L2.
 
 Metric: cached tokens compressed per second (sum over compressed units of
 their cached length N), and microseconds per step.
@@ -20,6 +23,7 @@ no collective on the data path); the time is the max over ranks.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import hashlib
 import json
@@ -37,7 +41,7 @@ if ROOT not in sys.path:
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from rkv_synth import WORKLOADS, bf16_bits, make_inputs  # noqa: E402
+from rkv_synth import WORKLOADS, bf16_bits, make_inputs, pack_ragged  # noqa: E402
 
 METRIC = "cached tokens compressed/sec (all layers×heads); µs per compress step"
 UNIT = "tokens/s"
@@ -51,9 +55,14 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="rkv", choices=["rkv", "reference"])
-    ap.add_argument("--workload", default="llama3_8b_step", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="ragged_batch", choices=sorted(WORKLOADS))
     ap.add_argument("--redundancy", default="mean", choices=["mean", "max"])
-    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--e2e-steps", type=int, default=6)
+    ap.add_argument("--layers", type=int, default=0,
+                    help="run the workload with this many layers instead of its own (a smaller "
+                         "case of the same shape, for profiler captures); 0 = the workload's")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the lambda sweep and the single-layer graph-replay figure")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cluster-size", type=int, default=0,
                     help="CTAs per unit: 0 = the library's choice, 1 = one CTA per unit, "
@@ -63,6 +72,10 @@ def parse_args():
                          "(layer, sequence) across the KV heads (rkv_score_shared, all-reduce "
                          "over ranks, rkv_select_compact_shared); paged: rkv_compress_step_paged")
     ap.add_argument("--page-rows", type=int, default=16)
+    ap.add_argument("--layout", default="auto", choices=["auto", "uniform", "ragged"],
+                    help="cache layout of the step: uniform [batch][Hkv][cap] caches "
+                         "(rkv_compress_step) or per-sequence capacities in one pool per layer "
+                         "(rkv_compress_step_ragged); auto = ragged when budgets differ")
     ap.add_argument("--loop", action="store_true",
                     help="run the whole decode loop of the workload (append + compress steps)")
     ap.add_argument("--generated", type=int, default=16384,
@@ -207,23 +220,31 @@ def dist_setup(args):
 
 
 # ----------------------------------------------------------------------------- reference arm
-def oracle_sample(w, red_mode):
-    """Inputs for the oracle arm: the first layer of the workload (all its units)."""
+ORACLE_SAMPLE_UNITS = 64        # units of layer 0 one oracle step computes (all threads)
+ORACLE_SAMPLE_UNITS_1T = 8      # the same, single-threaded
+
+
+def oracle_sample(w, red_mode, max_units):
+    """Inputs for the oracle: up to max_units (sequence, KV head) units of layer 0 of
+    the workload, taken at an even stride over the batch so that every budget of a
+    ragged batch is represented."""
     x = make_inputs(w, layers=[0])
     G = w.n_q_heads // w.n_kv_heads
     qb, kb = bf16_bits(x["Q"]), bf16_bits(x["K"])
-    units = [(b, h) for b in range(w.batch) for h in range(w.n_kv_heads)]
+    allu = [(b, h) for b in range(w.batch) for h in range(w.n_kv_heads)]
+    stride = max(1, -(-len(allu) // max_units))
+    units = allu[::stride][:max_units]
     q = np.stack([qb[0, b, h * G:(h + 1) * G] for (b, h) in units])
     k = np.stack([kb[0, b, h] for (b, h) in units])
     N = np.array([int(x["cur_len"][b]) for (b, _) in units], dtype=np.int32)
     bud = np.array([w.budget_of(b) for (b, _) in units], dtype=np.int32)
-    lam = np.full(len(units), w.mix_lambda)
+    lam = np.array([lambda_of(w, b) for (b, _) in units], dtype=np.float64)
     return q, k, N, bud, lam
 
 
-def time_oracle(w, red_mode, reps, threads):
+def time_oracle(w, red_mode, reps, threads, max_units):
     import oracle
-    q, k, N, bud, lam = oracle_sample(w, red_mode)
+    q, k, N, bud, lam = oracle_sample(w, red_mode, max_units)
     oracle.build()
     times = []
     for _ in range(reps):
@@ -234,44 +255,142 @@ def time_oracle(w, red_mode, reps, threads):
     return tokens, times, len(N)
 
 
+def oracle_sample_text(w, units, tokens, threads):
+    return (f"{units} (sequence, KV head) units of layer 0 of {w.name} at an even stride over "
+            f"the batch, {tokens} cached tokens per run; C oracle, fp64, "
+            + ("OpenMP over units" if threads > 1 else "one thread"))
+
+
 def run_reference(args, w, red_mode):
     world, rank, _ = dist_setup(args)
     if rank != 0:
         return
     threads = os.cpu_count() or 1
-    tokens, wt, units = time_oracle(w, red_mode, args.warmup, threads) if args.warmup else (0, [], 0)
-    tokens, times, units = time_oracle(w, red_mode, args.steps, threads)
+    if args.warmup:
+        time_oracle(w, red_mode, args.warmup, threads, ORACLE_SAMPLE_UNITS)
+    tokens, times, units = time_oracle(w, red_mode, args.steps, threads, ORACLE_SAMPLE_UNITS)
     per = sum(times) / len(times)
     value = tokens / per
-    sample = (f"layer 0 of {w.name} ({units} units, {tokens} cached tokens) per step; "
-              f"C oracle, fp64, OpenMP over units")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": workload_config(w, red_mode, args),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                         "sample": sample},
+                         "sample": oracle_sample_text(w, units, tokens, threads) + " per step"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
+def lambda_of(w, b):
+    """mix_lambda of sequence b: the ragged batch cycles 0 / 0.1 / 1 over its sequences
+    (the two ablation extremes and the pages' value); other workloads use w.mix_lambda."""
+    if w.name == "ragged_batch":
+        return RAGGED_LAMBDAS[b % 3]
+    return w.mix_lambda
+
+
+RAGGED_LAMBDAS = (0.0, 0.1, 1.0)
+
+
 def workload_config(w, red_mode, args):
+    lam = (f"per sequence, cycling {list(RAGGED_LAMBDAS)}" if w.name == "ragged_batch"
+           else w.mix_lambda)
     return {"workload": w.name, "n_layers": w.n_layers, "batch": w.batch,
             "n_kv_heads": w.n_kv_heads, "n_q_heads": w.n_q_heads, "head_dim": w.head_dim,
             "budget": list(w.budgets) if len(w.budgets) > 1 else w.budgets[0],
-            "buffer": w.buffer, "window": w.window, "mix_lambda": w.mix_lambda,
+            "buffer": w.buffer, "window": w.window, "mix_lambda": lam,
             "redundancy": "max" if red_mode else "mean", "gqa_pool": "max",
             "cached_len": w.n_tokens()[0] if len(set(w.n_tokens())) == 1 else "ragged",
             "near_duplicate_frac": list(w.dup_frac) if len(w.dup_frac) > 1 else w.dup_frac[0],
             "l2": "pristine in-HBM caches every step (a fresh replica, or the working copy "
                   "restored outside the per-step events when replicas do not fit; K+V larger "
-                  "than L2) and a 256 MB L2 flush before the timed region",
+                  "than L2) and a 256 MB L2 flush before the timed region and after every restore",
+            "layout": ("per-sequence capacities: one pool per layer, each sequence's block "
+                       "budget + buffer rows per KV head (rkv_compress_step_ragged)"
+                       if use_ragged_layout(args, w) else
+                       "uniform [batch][Hkv][cap] caches (rkv_compress_step)"),
             "parallelism": f"dp{args.gpus} (independent sequences per rank)"}
 
 
+def algorithmic_bytes(n_tok, budgets, n_layers, n_kv, G, window, moved):
+    """HBM bytes the step must move, per the step's byte count: per unit the scoring
+    reads K once (N rows of 256 B) and the G * w query rows, the select reads two
+    fp32 scores per candidate and writes one int32 per kept row, and every kept row
+    whose destination differs from its source is read and written once for each of
+    K and V (4 x 256 B).  `moved` counts those rows exactly over the whole launch."""
+    per_seq = [256 * (n + G * window) + 8 * (n - window) + 4 * bud
+               for n, bud in zip(n_tok, budgets)]
+    return n_layers * n_kv * sum(per_seq) + 1024 * moved
+
+
+ALG_BYTES_DEFINITION = ("per unit 256*(N + G*w) (K read once, window queries) + 8*(N - w) + "
+                        "4*budget (select) + 1024 per kept row that moves (K and V read and "
+                        "written), moved rows counted exactly")
+
+
 # ----------------------------------------------------------------------------- rkv arm
+def graph_replay_single_layer(rkv, dev, stream, reps=50):
+    """The single-layer step (8 units, N = 1152) as a captured CUDA graph of
+    (reset cur_len, rkv_compress_step), replayed `reps` times with events around each
+    replay; the same two calls issued eagerly for comparison.  Every replay compresses
+    the cache again from N = 1152 rows, so each does the full step's work."""
+    w1 = WORKLOADS["single_layer"]
+    x = make_inputs(w1, device=str(dev))
+    K, V, Q, cur0 = x["K"], x["V"], x["Q"], x["cur_len"].to(dev)
+    cur = cur0.clone()
+    L, B, H, cap, _ = K.shape
+    cfg = rkv.make_config(w1.budget_of(0), w1.buffer, w1.window, 128, w1.n_kv_heads,
+                          w1.n_q_heads, w1.mix_lambda)
+    ws = torch.zeros(rkv.rkv_workspace_size(cfg, L, B, cap), dtype=torch.uint8, device=dev)
+
+    def body(s):
+        cur.copy_(cur0)
+        rkv.rkv_compress_step(cfg, K, V, Q, cur, ws, stream=s)
+
+    for _ in range(3):
+        body(stream)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(stream)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            body(side)
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+
+    def timed(fn):
+        out = []
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            out.append(a.elapsed_time(b) * 1e3)
+        return statistics.median(out)
+
+    g_us = timed(graph.replay)
+    e_us = timed(lambda: body(stream))
+    assert rkv.rkv_workspace_status(ws) == 0
+    del graph
+    return {"workload": "single_layer", "graph_replay_us_median": g_us,
+            "eager_us_median": e_us, "replays": reps,
+            "what": "CUDA graph of (cur_len reset, rkv_compress_step) on 1 layer x 8 KV heads, "
+                    "N = 1152; events around each replay"}
+
+
+def use_ragged_layout(args, w):
+    if args.layout == "auto":
+        return len(set(w.budget_of(b) for b in range(w.batch))) > 1
+    return args.layout == "ragged"
+
+
 def run_rkv(args, w, red_mode):
     world, rank, local = dist_setup(args)
     torch.cuda.set_device(local)
@@ -287,24 +406,52 @@ def run_rkv(args, w, red_mode):
 
     seed = rdist.rank_seed(w.seed, rank)
     x = make_inputs(w, device=str(dev), seed=seed)
-    K0, V0, Q, cur0 = x["K"], x["V"], x["Q"], x["cur_len"].to(dev)
-    L, B, H, cap, D = K0.shape
+    L, B, H, cap, D = x["K"].shape
+    Q, cur0 = x["Q"], x["cur_len"].to(dev)
+    G = w.n_q_heads // w.n_kv_heads
+    ragged = use_ragged_layout(args, w)
+    caps = [w.budget_of(b) + w.buffer for b in range(B)]
+    if ragged:
+        # one pool per layer, every sequence's block exactly budget + buffer rows per head
+        K0, V0 = pack_ragged(x["K"], caps), pack_ragged(x["V"], caps)
+        rows, pool_rows = rkv.ragged_rows(caps, H)
+        seq_row = torch.tensor(rows, dtype=torch.int64, device=dev)
+        seq_cap = torch.tensor(caps, dtype=torch.int32, device=dev)
+        cap = max(caps)
+    else:
+        K0, V0 = x["K"], x["V"]
+    del x
     cfg = rkv.make_config(w.budget_of(0), w.buffer, w.window, 128, w.n_kv_heads, w.n_q_heads,
                           w.mix_lambda, redundancy_mode=red_mode)
     budgets = None
     if len(w.budgets) > 1:
         budgets = torch.tensor([w.budget_of(b) for b in range(B)], dtype=torch.int32, device=dev)
+    lambdas = None
+    if w.name == "ragged_batch":
+        lambdas = torch.tensor([lambda_of(w, b) for b in range(B)], dtype=torch.float32,
+                               device=dev)
     ws = torch.zeros(rkv.rkv_workspace_size(cfg, L, B, cap), dtype=torch.uint8, device=dev)
     shape = rkv.rkv_query_step_shape(cfg, L * B * H, cap)
-    if args.cluster_size:
-        shape = (args.cluster_size, cap if args.cluster_size == 1 else shape[1], shape[2])
+    if args.cluster_size or ragged:
+        cs = args.cluster_size or 1
+        shape = (cs, cap if cs == 1 else shape[1], shape[2])
     kernel_name = "rkv_unit_kernel" if shape[0] == 1 else "rkv_step_kernel"
     stream = torch.cuda.current_stream()
 
-    def step(Kr, Vr, cr, events=None, kept=None, sim_events=None):
-        rkv.rkv_compress_step(cfg, Kr, Vr, Q, cr, ws, budgets=budgets, kept_out=kept,
-                              cluster_size=args.cluster_size,
-                              events=events, stream=stream, sim_events=sim_events)
+    def call(cfg_, Kr, Vr, Qr, cr, lambdas_, events=None, kept=None, sim_events=None, strm=None):
+        if ragged:
+            rkv.rkv_compress_step_ragged(cfg_, Kr, Vr, Qr, cr, ws, seq_row, seq_cap, cap,
+                                         budgets=budgets, lambdas=lambdas_, kept_out=kept,
+                                         events=events, sim_events=sim_events,
+                                         cluster_size=args.cluster_size, stream=strm or stream)
+        else:
+            rkv.rkv_compress_step(cfg_, Kr, Vr, Qr, cr, ws, budgets=budgets, lambdas=lambdas_,
+                                  kept_out=kept, cluster_size=args.cluster_size,
+                                  events=events, stream=strm or stream, sim_events=sim_events)
+
+    def step(Kr, Vr, cr, events=None, kept=None, sim_events=None, cfg_=None, lambdas_=lambdas):
+        call(cfg_ or cfg, Kr, Vr, Q, cr, lambdas_, events=events, kept=kept,
+             sim_events=sim_events)
 
     # exact moved-row count (rows whose destination differs from their source)
     kept = torch.full((L, B, H, cap), -1, dtype=torch.int32, device=dev)
@@ -312,17 +459,17 @@ def run_rkv(args, w, red_mode):
     step(Kt, Vt, ct, kept=kept)
     torch.cuda.synchronize()
     assert rkv.rkv_workspace_status(ws) == 0
-    kept_h = kept.cpu().numpy()
-    n_tok = np.array([w.budget_of(b) + w.buffer for b in range(B)])
     moved = 0
     for b in range(B):
-        kb = kept_h[:, b, :, :w.budget_of(b)]
-        moved += int((kb != np.arange(w.budget_of(b))[None, None, :]).sum())
+        bud = w.budget_of(b)
+        kb = kept[:, b, :, :bud]
+        moved += int((kb != torch.arange(bud, device=dev, dtype=torch.int32)).sum().item())
     del Kt, Vt, ct, kept
     units = L * B * H
-    token_heads = int(L * H * n_tok.sum())
-    G = w.n_q_heads // w.n_kv_heads
-    alg_bytes = 256 * (L * H * int(n_tok.sum()) + units * G * w.window + 3 * moved)
+    n_tok = [w.budget_of(b) + w.buffer for b in range(B)]
+    token_heads = int(L * H * sum(n_tok))
+    alg_bytes = algorithmic_bytes(n_tok, [w.budget_of(b) for b in range(B)], L, H, G, w.window,
+                                  moved)
 
     # replicas: one pristine copy per warm-up and timed step when they fit in memory
     # (restored between the two timed passes); otherwise one working copy restored
@@ -344,23 +491,25 @@ def run_rkv(args, w, red_mode):
 
     def restore(r):
         r[0].copy_(K0); r[1].copy_(V0); r[2].copy_(cur0)
+        flush.fill_(1.0)
 
     t_start, t_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
-    def timed_pass(kernel_events):
-        """K steps over pristine caches after an L2 flush; returns the elapsed ms.
+    def timed_pass(kernel_events, n_steps=None, **kw):
+        """n_steps over pristine caches after an L2 flush; returns the elapsed ms.
         kernel_events: the library records ev[i] around the main kernel of step i."""
+        n_steps = n_steps or args.steps
         flush.fill_(1.0)
         torch.cuda.synchronize()
         rdist.barrier(dev)
         torch.cuda.synchronize()
         t_start.record(stream)
-        for i in range(args.steps):
+        for i in range(n_steps):
             if not fits:
                 restore(reps[0])
                 st[i][0].record(stream)
             step(*reps[args.warmup + i if fits else 0], events=ev[i] if kernel_events else None,
-                 sim_events=ev_sim[i] if (kernel_events and ev_sim) else None)
+                 sim_events=ev_sim[i] if (kernel_events and ev_sim) else None, **kw)
             if not fits:
                 st[i][1].record(stream)
         t_stop.record(stream)
@@ -369,7 +518,12 @@ def run_rkv(args, w, red_mode):
         assert rkv.rkv_workspace_status(ws) == 0
         if fits:
             return t_start.elapsed_time(t_stop)
-        return sum(a.elapsed_time(b) for a, b in st)
+        return sum(a.elapsed_time(b) for a, b in st[:n_steps])
+
+    def restore_all():
+        if fits:
+            for r in reps[args.warmup:]:
+                restore(r)
 
     sampler = ClockSampler(local)
     sampler.start()
@@ -381,16 +535,32 @@ def run_rkv(args, w, red_mode):
     elapsed_ms = timed_pass(False)
     # the main kernel's duration: the same steps again on restored caches, with
     # events around the kernel (they cost the step a few microseconds)
-    if fits:
-        for r in reps[args.warmup:]:
-            restore(r)
+    restore_all()
     timed_pass(True)
     clocks = sampler.stop()
     kern_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
     elapsed_ms, kern_ms = rdist.max_over_ranks([elapsed_ms, kern_ms], dev)
-    del reps
     ms_per_step = elapsed_ms / args.steps
     value = world * token_heads / (ms_per_step / 1e3)
+
+    # the ragged batch is also timed with one scalar lambda per call: the two ablation
+    # extremes and the pages' value
+    lambda_sweep = None
+    if w.name == "ragged_batch" and not args.no_extras:
+        lambda_sweep = {}
+        n_sw = min(args.steps, 10)
+        for lam in RAGGED_LAMBDAS:
+            c_l = rkv.make_config(w.budget_of(0), w.buffer, w.window, 128, w.n_kv_heads,
+                                  w.n_q_heads, lam, redundancy_mode=red_mode)
+            restore_all()
+            ms = timed_pass(False, n_steps=n_sw, cfg_=c_l, lambdas_=None)
+            lambda_sweep[str(lam)] = rdist.max_over_ranks([ms], dev)[0] / n_sw * 1e3
+        lambda_sweep = {"us_per_step": lambda_sweep, "steps": n_sw}
+    del reps
+
+    graph1 = None
+    if rank == 0 and world == 1 and not args.no_extras:
+        graph1 = graph_replay_single_layer(rkv, dev, stream)
 
     # end to end through host buffers: every step copies its inputs host -> device, runs
     # the step and copies its result device -> host.  Consecutive steps overlap: two
@@ -398,12 +568,24 @@ def run_rkv(args, w, red_mode):
     # step i + 1 and the D2H of step i - 1 run while step i computes (the two copy
     # directions use the link at the same time).
     e2e = None
-    # the end-to-end leg pins host copies of the caches: only for caches of a few GB
-    if args.e2e_steps > 0 and rep_bytes <= 4 * 1024 ** 3:
-        hK, hV, hQ = K0.cpu().pin_memory(), V0.cpu().pin_memory(), Q.cpu().pin_memory()
-        hc = cur0.cpu().pin_memory()
-        oK, oV, oc = torch.empty_like(hK).pin_memory(), torch.empty_like(hV).pin_memory(), \
-            torch.empty_like(hc).pin_memory()
+    host_need = 2.5 * rep_bytes          # pinned inputs + pinned outputs, with headroom
+    try:
+        import psutil
+        host_free = psutil.virtual_memory().available
+    except Exception:
+        host_free = float("inf")
+    if args.e2e_steps > 0 and host_need > host_free:
+        e2e = {"skipped": f"host RAM: {host_need / 1e9:.1f} GB of pinned buffers needed, "
+                          f"{host_free / 1e9:.1f} GB available"}
+    elif args.e2e_steps > 0:
+        def pinned_copy(t):
+            h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+            h.copy_(t)
+            return h
+        hK, hV, hQ, hc = pinned_copy(K0), pinned_copy(V0), pinned_copy(Q), pinned_copy(cur0)
+        oK = torch.empty(K0.shape, dtype=K0.dtype, pin_memory=True)
+        oV = torch.empty(V0.shape, dtype=V0.dtype, pin_memory=True)
+        oc = torch.empty(cur0.shape, dtype=cur0.dtype, pin_memory=True)
         sets = [(torch.empty_like(K0), torch.empty_like(V0), torch.empty_like(Q),
                  torch.empty_like(cur0)) for _ in range(2)]
         s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
@@ -422,8 +604,7 @@ def run_rkv(args, w, red_mode):
                 dQ.copy_(hQ, non_blocking=True); dc.copy_(hc, non_blocking=True)
                 ev_in[k].record(s_in)
             stream.wait_event(ev_in[k])
-            rkv.rkv_compress_step(cfg, dK, dV, dQ, dc, ws, budgets=budgets,
-                                  cluster_size=args.cluster_size, stream=stream)
+            call(cfg, dK, dV, dQ, dc, lambdas)
             ev_step[k].record(stream)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_step[k])
@@ -452,26 +633,29 @@ def run_rkv(args, w, red_mode):
         d2h = sum(t.numel() * t.element_size() for t in (oK, oV, oc))
         e2e = {"value": world * token_heads / (e_ms / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms,
+               "steps": args.e2e_steps,
                "overlap": "copies of consecutive steps overlap (two buffer sets, copy streams)"}
+        del sets, hK, hV, oK, oV
 
     peak, peak_kind = measured_peaks()
     achieved = alg_bytes / (kern_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "traffic": profiled_traffic(kernel_name, w.name, units),
                 "kernel": kernel_name, "kernel_us_per_launch": kern_ms * 1e3,
-                "algorithmic_bytes_per_launch": alg_bytes, "peak_source": peak_kind,
+                "algorithmic_bytes_per_launch": alg_bytes,
+                "algorithmic_bytes_definition": ALG_BYTES_DEFINITION,
+                "moved_rows": moved, "kept_rows": L * H * sum(w.budget_of(b) for b in range(B)),
+                "peak_source": peak_kind,
                 "kernel_source_sha256_16": kernel_source_digest(kernel_name),
                 "cluster_size": shape[0], "rows_per_cta": shape[1], "smem_per_cta": shape[2]}
     roofline_unit = None
     if ev_sim:
         # MAX redundancy: the similarity kernel is the dominant one.  Algorithmic flops are
-        # the symmetric Gram N (N - 1) D per unit; the kernel computes every (row block,
-        # column tile) pair of 128 x 128 x 128, 2 * 128^3 flops each.
+        # the symmetric Gram N (N - 1) D per unit.
         sim_ms = sum(a.elapsed_time(b) for a, b in ev_sim) / args.steps
         sim_ms = rdist.max_over_ranks([sim_ms], dev)[0]
-        n_seq = [w.budget_of(b) + w.buffer for b in range(B)]
-        alg_flops = L * H * sum(n * (n - 1) * D for n in n_seq)
-        exe_flops = L * H * sum(-(-(n - w.window) // 128) * -(-n // 128) * 2 * 128 ** 3 for n in n_seq)
+        alg_flops = L * H * sum(n * (n - 1) * D for n in n_tok)
+        exe_flops = L * H * sum(gram_executed_flops(n, w.window) for n in n_tok)
         tpeak, tkind = measured_bf16_tflops()
         t_ach = alg_flops / (sim_ms / 1e3) / 1e12
         roofline_unit = roofline
@@ -481,32 +665,50 @@ def run_rkv(args, w, red_mode):
                     "executed_flops_per_launch": exe_flops,
                     "executed_tflops": exe_flops / (sim_ms / 1e3) / 1e12, "peak_source": tkind}
 
-    cpu = None
+    cpu = cpu1 = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         threads = os.cpu_count() or 1
-        tokens, times, nu = time_oracle(w, red_mode, 3, threads)
+        tokens, times, nu = time_oracle(w, red_mode, 3, threads, ORACLE_SAMPLE_UNITS)
         per = sorted(times)[1]
         cpu = {"value": tokens / per, "unit": UNIT, "cores": threads, "kind": "oracle",
-               "sample": f"layer 0 of {w.name}: {nu} units, {tokens} cached tokens per run, "
-                         f"median of 3 runs, C oracle fp64 with OpenMP over units"}
+               "sample": oracle_sample_text(w, nu, tokens, threads) + ", median of 3 runs"}
+        tokens, times, nu = time_oracle(w, red_mode, 1, 1, ORACLE_SAMPLE_UNITS_1T)
+        cpu1 = {"value": tokens / times[0], "unit": UNIT, "cores": 1, "kind": "oracle",
+                "sample": oracle_sample_text(w, nu, tokens, 1) + ", one run"}
 
     if world > 1:
         torch.distributed.destroy_process_group()
     if rank != 0:
         return
-    # per 32-layer chunk: the step kernel, plus the inverse-norm and similarity kernels in MAX mode
-    n_main_launches = ((L + 31) // 32) * (3 if red_mode else 1)
+    # per 32-layer chunk: the step kernel, plus the similarity kernel(s) in MAX mode
+    n_main_launches = ((L + 31) // 32) * (1 + gram_launches_per_chunk() if red_mode else 1)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "us_per_step": ms_per_step * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic", "config": workload_config(w, red_mode, args),
         "e2e": e2e, "gpu_launches": args.steps * (1 + n_main_launches),
-        "roofline": roofline, "cpu_baseline": cpu, "clocks": clocks,
+        "roofline": roofline, "cpu_baseline": cpu, "cpu_baseline_single_thread": cpu1,
+        "clocks": clocks,
         **({"roofline_unit_kernel": roofline_unit} if roofline_unit else {}),
+        **({"lambda_sweep": lambda_sweep} if lambda_sweep else {}),
+        **({"single_layer_graph": graph1} if graph1 else {}),
         "token_heads_per_step_per_gpu": token_heads,
     }
     print(json.dumps(line), flush=True)
+
+
+def gram_launches_per_chunk():
+    """Kernels the MAX-mode redundancy launches per 32-layer chunk (the similarity
+    kernel computes the inverse norms itself)."""
+    return 1
+
+
+def gram_executed_flops(n, window):
+    """Flops the similarity kernel executes for one unit of n cached rows: the tile
+    pairs (I, J >= I) of 128 x 128 x 128 (the symmetric half, diagonal tiles whole)."""
+    t = -(-n // 128)
+    return t * (t + 1) // 2 * 2 * 128 ** 3
 
 
 # ----------------------------------------------------------------------------- decode loop
@@ -593,6 +795,7 @@ def run_loop(args, w, red_mode):
         "us_per_step": 1e3 * total_ms / len(step_ms), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": dict(workload_config(w, red_mode, args), mode="decode_loop",
+                       layout="uniform [batch][Hkv][cap] caches",
                        generated_tokens=args.generated),
         "loop": {"compress_steps": len(step_ms), "total_compress_ms": total_ms,
                  "step_us_median": 1e3 * statistics.median(step_ms),
@@ -700,13 +903,15 @@ def run_mode(args, w, red_mode):
             "scaling": "strong" if tp else "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": dict(workload_config(w, red_mode, args), mode=args.mode, **extra,
+                           layout=("paged pools" if args.mode == "paged"
+                                   else "uniform [batch][Hkv][cap] caches"),
                            **({"parallelism": f"tp{world} (KV heads split over ranks)"}
                               if tp else {})),
             # shared: plan, scoring kernels, head sum, plan, select+compact per 32-layer chunk;
-            # paged: plan, freed pages, step kernel per chunk
+            # paged: plan, freed pages, step kernel per chunk (+ the similarity kernel in MAX)
             "gpu_launches": args.steps * (
-                3 + ((L + 31) // 32) * (2 + (2 if red_mode else 0)) if args.mode == "shared"
-                else 2 + (L + 31) // 32),
+                3 + ((L + 31) // 32) * (2 + (1 if red_mode else 0)) if args.mode == "shared"
+                else 2 + ((L + 31) // 32) * (2 if red_mode else 1)),
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
@@ -718,6 +923,8 @@ def run_mode(args, w, red_mode):
 def main():
     args = parse_args()
     w = WORKLOADS[args.workload]
+    if args.layers:
+        w = dataclasses.replace(w, n_layers=args.layers)
     red_mode = 1 if args.redundancy == "max" else 0
     if args.impl == "reference":
         run_reference(args, w, red_mode)

@@ -23,6 +23,7 @@ __all__ = [
     "rkv_compress_step", "rkv_append_kv",
     "rkv_workspace_size_shared", "rkv_score_shared", "rkv_select_compact_shared",
     "rkv_paged_kv", "rkv_compress_step_paged",
+    "rkv_ragged_kv", "rkv_compress_step_ragged", "ragged_rows",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -56,6 +57,15 @@ class rkv_paged_kv(ctypes.Structure):
         ("num_pages", ctypes.c_int32),
         ("freed_pages", ctypes.c_void_p),
         ("n_freed", ctypes.c_void_p),
+    ]
+
+
+class rkv_ragged_kv(ctypes.Structure):
+    _fields_ = [
+        ("seq_row", ctypes.c_void_p),
+        ("seq_cap", ctypes.c_void_p),
+        ("pool_rows", ctypes.c_int64),
+        ("max_cap", ctypes.c_int32),
     ]
 
 
@@ -100,6 +110,9 @@ def _load() -> ctypes.CDLL:
         "rkv_compress_step_paged": (ctypes.c_int, [CFG, I32, I32, ctypes.POINTER(rkv_paged_kv), P,
                                                    P, P, P, P, P, ctypes.POINTER(rkv_step_options),
                                                    P, SZ, P]),
+        "rkv_compress_step_ragged": (ctypes.c_int, [CFG, I32, I32, ctypes.POINTER(rkv_ragged_kv),
+                                                    P, P, P, P, P, P,
+                                                    ctypes.POINTER(rkv_step_options), P, SZ, P]),
         "rkv_score_shared": (ctypes.c_int, [CFG, I32, I32, I32, P, P, P, P, P, P, P, SZ, P]),
         "rkv_select_compact_shared": (ctypes.c_int, [CFG, I32, I32, I32, P, P, P, P, P, P, P, SZ,
                                                      P]),
@@ -370,3 +383,49 @@ def rkv_compress_step_paged(cfg, k_pools, v_pools, q_layers, cur_len, workspace,
                                                ctypes.byref(opts), _ptr(workspace), ws,
                                                _stream(stream)),
                   "rkv_compress_step_paged", allow_disabled=True)
+
+
+def ragged_rows(caps, n_kv_heads: int):
+    """First pool row of every sequence when the blocks [n_kv_heads][cap_b][128]
+    are packed back to back in batch order, and the pool's row count."""
+    rows, r = [], 0
+    for c in caps:
+        rows.append(r)
+        r += int(n_kv_heads) * int(c)
+    return rows, r
+
+
+def rkv_compress_step_ragged(cfg, k_pools, v_pools, q_layers, cur_len, workspace, seq_row,
+                             seq_cap, max_cap, budgets=None, lambdas=None, kept_out=None,
+                             scores_out=None, events=None, sim_events=None, cluster_size=0,
+                             stream=None):
+    """The step on caches with per-sequence capacities, in place.
+
+    k_pools / v_pools: per layer [pool_rows, 128] bf16 (or one [n_layers,
+    pool_rows, 128] tensor); sequence b's [Hkv][seq_cap[b]][128] block starts at
+    pool row seq_row[b] (seq_row [batch] int64, seq_cap [batch] int32, on the
+    device); max_cap >= every seq_cap.  q_layers, cur_len, budgets, lambdas as in
+    rkv_compress_step; kept_out [n_layers, batch, Hkv, max_cap] int32 and
+    scores_out [n_layers, batch, Hkv, 4, max_cap] fp32 optional.
+    """
+    kp, n_layers, (pool_rows, _) = _layers(k_pools, "k")
+    vp, _, _ = _layers(v_pools, "v")
+    qp, _, (batch, _, _, _) = _layers(q_layers, "q")
+    _dtype(seq_row, torch.int64, "seq_row"); _dtype(seq_cap, torch.int32, "seq_cap")
+    _dtype(cur_len, torch.int32, "cur_len"); _dtype(budgets, torch.int32, "budgets")
+    _dtype(lambdas, torch.float32, "lambdas"); _dtype(kept_out, torch.int32, "kept_out")
+    _dtype(scores_out, torch.float32, "scores_out")
+    rg = rkv_ragged_kv(_ptr(seq_row), _ptr(seq_cap), int(pool_rows), int(max_cap))
+    opts = rkv_step_options(_ptr(kept_out), _ptr(scores_out), None, None, int(cluster_size))
+    if events is not None:
+        opts.main_begin = events[0].cuda_event
+        opts.main_end = events[1].cuda_event
+    if sim_events is not None:
+        opts.sim_begin = sim_events[0].cuda_event
+        opts.sim_end = sim_events[1].cuda_event
+    ws = workspace.numel() * workspace.element_size()
+    return _check(_lib.rkv_compress_step_ragged(ctypes.byref(cfg), n_layers, int(batch),
+                                                ctypes.byref(rg), kp, vp, qp, _ptr(budgets),
+                                                _ptr(lambdas), _ptr(cur_len), ctypes.byref(opts),
+                                                _ptr(workspace), ws, _stream(stream)),
+                  "rkv_compress_step_ragged", allow_disabled=True)

@@ -1,6 +1,11 @@
-"""Builds librkv.so (all CUDA sources of the package) for sm_100a, in-tree."""
+"""Builds librkv.so (all CUDA sources of the package) for sm_100a, in-tree.
+
+Each .cu file is compiled to its own object in parallel (objects under
+``_build/``, rebuilt when the file or any header is newer), then linked.
+"""
 from __future__ import annotations
 
+import concurrent.futures as cf
 import glob
 import os
 import subprocess
@@ -9,6 +14,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "librkv.so")
+OBJ_DIR = os.path.join(ROOT, "_build", "librkv")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -17,32 +23,67 @@ NVCC_FLAGS = [
     "--expt-relaxed-constexpr",
     "-Xptxas", "-v",
 ]
+LINK_LIBS: list = []
 
 
 def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
+def _headers():
+    hs = glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h"))
+    hs.append(os.path.join(ROOT, "include", "rkv.h"))
+    return hs
+
+
 def _stale() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h"))
-    deps.append(os.path.join(ROOT, "include", "rkv.h"))
-    return any(os.path.getmtime(d) > t for d in deps)
+    return any(os.path.getmtime(d) > t for d in sources() + _headers())
+
+
+def _obj_of(src: str) -> str:
+    return os.path.join(OBJ_DIR, os.path.basename(src)[:-3] + ".o")
+
+
+def _compile(nvcc: str, src: str, newest_header: float, force: bool):
+    obj = _obj_of(src)
+    if (not force and os.path.exists(obj) and
+            os.path.getmtime(obj) >= max(os.path.getmtime(src), newest_header)):
+        return obj, ""
+    tmp = obj + f".tmp{os.getpid()}"
+    cmd = [nvcc, *NVCC_FLAGS, "-c", "-o", tmp, src, "-I", os.path.join(ROOT, "include")]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if res.returncode != 0:
+        raise RuntimeError(f"nvcc failed on {os.path.basename(src)}:\n" + res.stdout + res.stderr)
+    os.replace(tmp, obj)
+    return obj, res.stderr
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and not _stale():
         return LIB
     nvcc = os.environ.get("NVCC", "nvcc")
+    os.makedirs(OBJ_DIR, exist_ok=True)
+    newest = max(os.path.getmtime(h) for h in _headers())
+    srcs = sources()
+    logs = []
+    with cf.ThreadPoolExecutor(max_workers=min(len(srcs), os.cpu_count() or 4)) as ex:
+        futs = [ex.submit(_compile, nvcc, s, newest, force) for s in srcs]
+        objs = []
+        for f in futs:
+            obj, log = f.result()
+            objs.append(obj)
+            logs.append(log)
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc, *NVCC_FLAGS, "-shared", "-o", tmp, *sources(), "-I", os.path.join(ROOT, "include")]
+    cmd = [nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs,
+           *LINK_LIBS]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
-        raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
+        raise RuntimeError("nvcc link failed:\n" + res.stdout + res.stderr)
     if verbose:
-        print(res.stderr)
+        print("".join(logs))
     os.replace(tmp, LIB)
     return LIB
 

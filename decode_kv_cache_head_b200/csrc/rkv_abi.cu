@@ -172,7 +172,8 @@ cudaError_t launch_unit_layers(const rkv_config *cfg, int32_t n_layers, int32_t 
                                const float *lambdas, const int32_t *n_eff, const float *r_ext,
                                int32_t *kept_out, float *scores_out, float *z_heads,
                                uint32_t *status, const UnitShape &us, int nqp, cudaStream_t strm,
-                               const PagedArgs &pg = PagedArgs{nullptr, 0, 0, 0}) {
+                               const PagedArgs &pg = PagedArgs{nullptr, 0, 0, 0},
+                               const RaggedLayout &rg = RaggedLayout{}) {
     UnitParams *up = new UnitParams();
     std::memset(up, 0, sizeof(*up));
     up->batch = batch;
@@ -198,10 +199,13 @@ cudaError_t launch_unit_layers(const rkv_config *cfg, int32_t n_layers, int32_t 
     up->block_table = pg.block_table;
     up->max_blocks = pg.max_blocks;
     up->page_rows = pg.page_rows;
+    up->seq_row = rg.seq_row;
+    up->seq_cap = rg.seq_cap;
     up->status = status;
     const uint64_t k_rows = pg.block_table
                                 ? static_cast<uint64_t>(pg.num_pages) * cfg->n_kv_heads * pg.page_rows
-                                : static_cast<uint64_t>(batch) * cfg->n_kv_heads * cap;
+                            : rg.seq_row ? static_cast<uint64_t>(rg.pool_rows)
+                                         : static_cast<uint64_t>(batch) * cfg->n_kv_heads * cap;
     const uint32_t k_box = pg.block_table ? static_cast<uint32_t>(pg.page_rows) : 128u;
     cudaError_t e = cudaSuccess;
     for (int l0 = 0; e == cudaSuccess && l0 < n_layers; l0 += kMaxLayersPerLaunch) {
@@ -231,30 +235,34 @@ cudaError_t launch_unit_layers(const rkv_config *cfg, int32_t n_layers, int32_t 
 cudaError_t launch_gram_layers(const rkv_config *cfg, int32_t n_layers, int32_t batch, int32_t cap,
                                const rkv_bf16 *const *k_layers, const int32_t *n_eff, float *r_ext,
                                uint32_t *status, cudaStream_t strm, cudaEvent_t sim_begin = nullptr,
-                               cudaEvent_t sim_end = nullptr) {
+                               cudaEvent_t sim_end = nullptr,
+                               const RaggedLayout &rg = RaggedLayout{},
+                               const PagedArgs &pg = PagedArgs{nullptr, 0, 0, 0}) {
     GramParams *gp = new GramParams();
     std::memset(gp, 0, sizeof(*gp));
     gp->batch = batch;
     gp->n_kv = cfg->n_kv_heads;
     gp->window = cfg->window;
     gp->cap = cap;
-    gp->nblk = (cap - cfg->window + 127) / 128;
     gp->n_eff = n_eff;
+    gp->seq_row = rg.seq_row;
+    gp->seq_cap = rg.seq_cap;
+    gp->block_table = pg.block_table;
+    gp->max_blocks = pg.max_blocks;
+    gp->page_rows = pg.page_rows;
     gp->r_out = r_ext;
-    gp->inv = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(r_ext) +
-                                        align256(static_cast<size_t>(n_layers) * batch *
-                                                 cfg->n_kv_heads * cap * 4));
     gp->status = status;
+    const uint64_t k_rows = pg.block_table
+                                ? static_cast<uint64_t>(pg.num_pages) * cfg->n_kv_heads * pg.page_rows
+                            : rg.seq_row ? static_cast<uint64_t>(rg.pool_rows)
+                                         : static_cast<uint64_t>(batch) * cfg->n_kv_heads * cap;
+    const uint32_t k_box = pg.block_table ? static_cast<uint32_t>(pg.page_rows) : 128u;
     cudaError_t e = cudaSuccess;
     for (int l0 = 0; e == cudaSuccess && l0 < n_layers; l0 += kMaxLayersPerLaunch) {
         const int nl = (n_layers - l0 < kMaxLayersPerLaunch) ? n_layers - l0 : kMaxLayersPerLaunch;
         gp->layer_base = l0;
-        for (int i = 0; i < nl && e == cudaSuccess; ++i) {
-            gp->k[i] = k_layers[l0 + i];
-            if (!encode_rows128(&gp->tmap[i], k_layers[l0 + i],
-                                static_cast<uint64_t>(batch) * cfg->n_kv_heads * cap, 128))
-                e = cudaErrorInvalidValue;
-        }
+        for (int i = 0; i < nl && e == cudaSuccess; ++i)
+            if (!encode_rows128(&gp->tmap[i], k_layers[l0 + i], k_rows, k_box)) e = cudaErrorInvalidValue;
         if (e == cudaSuccess)
             e = launch_gram_max(*gp, nl * batch * cfg->n_kv_heads, strm, l0 == 0 ? sim_begin : nullptr,
                                 l0 + nl >= n_layers ? sim_end : nullptr);
@@ -270,8 +278,8 @@ size_t ws_bytes_shared(const rkv_config *cfg, int32_t n_layers, int32_t batch, i
 size_t ws_bytes_for(const rkv_config *cfg, int32_t n_layers, int32_t batch, int32_t cap) {
     size_t n = kStatusBytes;
     n += align256(static_cast<size_t>(batch) * 4);
-    if (cfg->redundancy_mode == RKV_RED_MAX)   // r, then the inverse norms, per unit
-        n += 2 * align256(static_cast<size_t>(n_layers) * batch * cfg->n_kv_heads * cap * 4);
+    if (cfg->redundancy_mode == RKV_RED_MAX)   // r per unit, from the similarity kernel
+        n += align256(static_cast<size_t>(n_layers) * batch * cfg->n_kv_heads * cap * 4);
     return n;
 }
 
@@ -310,6 +318,7 @@ rkv_status run_per_head_scores(const rkv_config *cfg, const rkv_bf16 *q, const r
     const Shape s = choose_shape(cap, nqp, 0);
     if (s.cs == 0) return RKV_ERR_UNSUPPORTED;
     const bool red_max = cfg->redundancy_mode == RKV_RED_MAX && (r || R);
+    if (red_max && cap > gram_max_rows()) return RKV_ERR_UNSUPPORTED;
     StepParams *pp = new StepParams();
     StepParams &p = *pp;
     std::memset(&p, 0, sizeof(p));
@@ -337,12 +346,8 @@ rkv_status run_per_head_scores(const rkv_config *cfg, const rkv_bf16 *q, const r
         gp->n_kv = cfg->n_kv_heads;
         gp->window = cfg->window;
         gp->cap = cap;
-        gp->nblk = (cap - cfg->window + 127) / 128;
         gp->n_tokens_fixed = n_tokens;
         gp->r_out = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + kStatusBytes + 256);
-        gp->inv = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(gp->r_out) +
-                                            align256(static_cast<size_t>(cfg->n_kv_heads) * cap * 4));
-        gp->k[0] = k;
         gp->status = static_cast<uint32_t *>(ws);
         p.r_ext = gp->r_out;
     }
@@ -426,6 +431,7 @@ rkv_status rkv_score_importance(const rkv_config *cfg, const rkv_bf16 *q, const 
                                 int64_t k_head_stride, int32_t n_tokens, float *I,
                                 float *inv_norm, void *workspace, size_t ws_bytes,
                                 rkv_stream_t stream) {
+    NvtxRange nvtx_range("rkv_score_importance");
     rkv_status st = check_cfg(cfg);
     if (st != RKV_OK) return st;
     if (!q || !k || !I) return RKV_ERR_NULL;
@@ -444,6 +450,7 @@ rkv_status rkv_score_importance(const rkv_config *cfg, const rkv_bf16 *q, const 
 rkv_status rkv_score_redundancy(const rkv_config *cfg, const rkv_bf16 *k, int64_t k_head_stride,
                                 int32_t n_tokens, float *r, float *R, void *workspace,
                                 size_t ws_bytes, rkv_stream_t stream) {
+    NvtxRange nvtx_range("rkv_score_redundancy");
     rkv_status st = check_cfg(cfg);
     if (st != RKV_OK) return st;
     if (!workspace) return RKV_ERR_WORKSPACE;
@@ -462,6 +469,7 @@ rkv_status rkv_score_redundancy(const rkv_config *cfg, const rkv_bf16 *k, int64_
 rkv_status rkv_select_topk(const rkv_config *cfg, const float *I, const float *R,
                            int32_t n_tokens, int32_t *kept, float *Z, void *workspace,
                            size_t ws_bytes, rkv_stream_t stream) {
+    NvtxRange nvtx_range("rkv_select_topk");
     rkv_status st = check_cfg(cfg);
     if (st != RKV_OK) return st;
     if (cfg->budget <= 0 || cfg->buffer <= 0) return RKV_STATUS_DISABLED;
@@ -490,6 +498,7 @@ rkv_status rkv_compact_kv(const rkv_config *cfg, const rkv_bf16 *k_src, const rk
                           const int32_t *kept, rkv_bf16 *k_dst, rkv_bf16 *v_dst,
                           int64_t head_stride, int32_t n_tokens, void *workspace,
                           size_t ws_bytes, rkv_stream_t stream) {
+    NvtxRange nvtx_range("rkv_compact_kv");
     rkv_status st = check_cfg(cfg);
     if (st != RKV_OK) return st;
     if (cfg->budget <= 0 || cfg->buffer <= 0) return RKV_STATUS_DISABLED;
@@ -529,6 +538,7 @@ rkv_status rkv_compress_step(const rkv_config *cfg, int32_t n_layers, int32_t ba
                              const float *lambdas, int32_t *cur_len,
                              const rkv_step_options *opts, void *workspace, size_t ws_bytes,
                              rkv_stream_t stream) {
+    NvtxRange nvtx_range("rkv_compress_step");
     rkv_status st = check_cfg(cfg);
     if (st != RKV_OK) return st;
     if (cfg->buffer <= 0 || (!budgets && cfg->budget <= 0)) return RKV_STATUS_DISABLED;
@@ -558,6 +568,7 @@ rkv_status rkv_compress_step(const rkv_config *cfg, int32_t n_layers, int32_t ba
     if (unit_path && !us.ok) return RKV_ERR_UNSUPPORTED;
     const Shape s = unit_path ? Shape{} : choose_shape(cap, nqp, cs_req);
     if (!unit_path && s.cs == 0) return RKV_ERR_UNSUPPORTED;
+    if (cfg->redundancy_mode == RKV_RED_MAX && cap > gram_max_rows()) return RKV_ERR_UNSUPPORTED;
 
     cudaStream_t strm = reinterpret_cast<cudaStream_t>(stream);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -623,6 +634,7 @@ rkv_status rkv_append_kv(const rkv_config *cfg, int32_t n_layers, int32_t batch,
                          const rkv_bf16 *const *k_new_layers, const rkv_bf16 *const *v_new_layers,
                          int32_t n_new, int32_t *cur_len, void *workspace, size_t ws_bytes,
                          rkv_stream_t stream) {
+    NvtxRange nvtx_range("rkv_append_kv");
     rkv_status st = check_cfg(cfg);
     if (st != RKV_OK) return st;
     if (!k_layers || !v_layers || !k_new_layers || !v_new_layers || !cur_len) return RKV_ERR_NULL;
@@ -697,6 +709,7 @@ rkv_status check_shared_args(const rkv_config *cfg, int32_t n_layers, int32_t ba
         return RKV_ERR_UNSUPPORTED;
     const int nqp = nqp_of((cfg->n_q_heads / cfg->n_kv_heads) * cfg->window);
     if (!unit_shape(cap, nqp).ok) return RKV_ERR_UNSUPPORTED;
+    if (cfg->redundancy_mode == RKV_RED_MAX && cap > gram_max_rows()) return RKV_ERR_UNSUPPORTED;
     const size_t layer_bytes = static_cast<size_t>(batch) * cfg->n_kv_heads * cap * kHeadDim * 2;
     for (int l = 0; l < n_layers; ++l) {
         if (!k_layers[l] || (v_layers && !v_layers[l]) || (q_layers && !q_layers[l]))
@@ -721,6 +734,7 @@ rkv_status rkv_score_shared(const rkv_config *cfg, int32_t n_layers, int32_t bat
                             const rkv_bf16 *const *k_layers, const rkv_bf16 *const *q_layers,
                             const int32_t *budgets, const float *lambdas, const int32_t *cur_len,
                             float *z_sum, void *workspace, size_t ws_bytes, rkv_stream_t stream) {
+    NvtxRange nvtx_range("rkv_score_shared");
     if (!q_layers) return check_cfg(cfg) != RKV_OK ? check_cfg(cfg) : RKV_ERR_NULL;
     rkv_status st = check_shared_args(cfg, n_layers, batch, cap, k_layers, nullptr, q_layers,
                                       budgets, cur_len, z_sum, workspace, ws_bytes);
@@ -763,6 +777,7 @@ rkv_status rkv_select_compact_shared(const rkv_config *cfg, int32_t n_layers, in
                                      rkv_bf16 *const *v_layers, const int32_t *budgets,
                                      int32_t *cur_len, const float *z_sum, int32_t *kept_out,
                                      void *workspace, size_t ws_bytes, rkv_stream_t stream) {
+    NvtxRange nvtx_range("rkv_select_compact_shared");
     if (!v_layers) return check_cfg(cfg) != RKV_OK ? check_cfg(cfg) : RKV_ERR_NULL;
     rkv_status st = check_shared_args(cfg, n_layers, batch, cap,
                                       const_cast<const rkv_bf16 *const *>(k_layers),
@@ -807,6 +822,7 @@ rkv_status rkv_compress_step_paged(const rkv_config *cfg, int32_t n_layers, int3
                                    const int32_t *budgets, const float *lambdas, int32_t *cur_len,
                                    const rkv_step_options *opts, void *workspace, size_t ws_bytes,
                                    rkv_stream_t stream) {
+    NvtxRange nvtx_range("rkv_compress_step_paged");
     rkv_status st = check_cfg(cfg);
     if (st != RKV_OK) return st;
     if (cfg->buffer <= 0 || (!budgets && cfg->budget <= 0)) return RKV_STATUS_DISABLED;
@@ -816,7 +832,6 @@ rkv_status rkv_compress_step_paged(const rkv_config *cfg, int32_t n_layers, int3
     const int P = pg->page_rows;
     if (P != 16 && P != 32 && P != 64 && P != 128) return RKV_ERR_UNSUPPORTED;
     if (n_layers < 1 || batch < 1 || pg->max_blocks < 1 || pg->num_pages < 1) return RKV_ERR_INVALID;
-    if (cfg->redundancy_mode != RKV_RED_MEAN) return RKV_ERR_UNSUPPORTED;
     if (opts && opts->cluster_size != 0 && opts->cluster_size != 1) return RKV_ERR_UNSUPPORTED;
     const int64_t cap64 = static_cast<int64_t>(pg->max_blocks) * P;
     if (cap64 > kUnitMaxPages * static_cast<int64_t>(P) ||
@@ -837,13 +852,24 @@ rkv_status rkv_compress_step_paged(const rkv_config *cfg, int32_t n_layers, int3
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return RKV_ERR_ALIGN;
     if (ws_bytes < ws_bytes_for(cfg, n_layers, batch, cap)) return RKV_ERR_WORKSPACE;
 
+    if (cfg->redundancy_mode == RKV_RED_MAX && cap > gram_max_rows()) return RKV_ERR_UNSUPPORTED;
+
     cudaStream_t strm = reinterpret_cast<cudaStream_t>(stream);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     uint32_t *status = reinterpret_cast<uint32_t *>(ws);
     int32_t *n_eff = reinterpret_cast<int32_t *>(ws + kStatusBytes);
+    float *r_ext = reinterpret_cast<float *>(ws + kStatusBytes + align256(static_cast<size_t>(batch) * 4));
+    const bool red_max = cfg->redundancy_mode == RKV_RED_MAX;
+    const PagedArgs pa{pg->block_table, pg->max_blocks, P, pg->num_pages};
     // the plan kernel clears the status words first
     cudaError_t e = launch_plan(batch, budgets, cfg->budget, cfg->buffer, cfg->window, cap, cur_len,
                                 n_eff, status, strm, true);
+    if (red_max && e == cudaSuccess)   // raw r of every candidate, through the block table
+        e = launch_gram_layers(cfg, n_layers, batch, cap,
+                               const_cast<const rkv_bf16 *const *>(k_pools), n_eff, r_ext, status,
+                               strm, opts ? reinterpret_cast<cudaEvent_t>(opts->sim_begin) : nullptr,
+                               opts ? reinterpret_cast<cudaEvent_t>(opts->sim_end) : nullptr,
+                               RaggedLayout{}, pa);
     if (e == cudaSuccess)
         e = launch_freed_pages(batch, budgets, cfg->budget, n_eff, pg->block_table, pg->max_blocks,
                                P, pg->freed_pages, pg->n_freed, strm);
@@ -852,9 +878,77 @@ rkv_status rkv_compress_step_paged(const rkv_config *cfg, int32_t n_layers, int3
     if (e == cudaSuccess)
         e = launch_unit_layers(cfg, n_layers, batch, cap,
                                const_cast<const rkv_bf16 *const *>(k_pools), v_pools, q_layers,
-                               budgets, lambdas, n_eff, nullptr, opts ? opts->kept_out : nullptr,
-                               opts ? opts->scores_out : nullptr, nullptr, status, us, nqp, strm,
-                               PagedArgs{pg->block_table, pg->max_blocks, P, pg->num_pages});
+                               budgets, lambdas, n_eff, red_max ? r_ext : nullptr,
+                               opts ? opts->kept_out : nullptr,
+                               opts ? opts->scores_out : nullptr, nullptr, status, us, nqp, strm, pa);
+    if (e == cudaSuccess && opts && opts->main_end)
+        e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->main_end), strm);
+    return cuda_status(e);
+}
+
+rkv_status rkv_compress_step_ragged(const rkv_config *cfg, int32_t n_layers, int32_t batch,
+                                    const rkv_ragged_kv *rg, rkv_bf16 *const *k_pools,
+                                    rkv_bf16 *const *v_pools, const rkv_bf16 *const *q_layers,
+                                    const int32_t *budgets, const float *lambdas,
+                                    int32_t *cur_len, const rkv_step_options *opts,
+                                    void *workspace, size_t ws_bytes, rkv_stream_t stream) {
+    NvtxRange nvtx_range("rkv_compress_step_ragged");
+    rkv_status st = check_cfg(cfg);
+    if (st != RKV_OK) return st;
+    if (cfg->buffer <= 0 || (!budgets && cfg->budget <= 0)) return RKV_STATUS_DISABLED;
+    if (!rg || !k_pools || !v_pools || !q_layers || !cur_len) return RKV_ERR_NULL;
+    if (!rg->seq_row || !rg->seq_cap) return RKV_ERR_NULL;
+    if (!workspace) return RKV_ERR_WORKSPACE;
+    if (n_layers < 1 || batch < 1 || rg->max_cap < 2 || rg->pool_rows < 1) return RKV_ERR_INVALID;
+    if (rg->pool_rows > INT32_MAX || static_cast<int64_t>(batch) * cfg->n_q_heads * cfg->window > INT32_MAX)
+        return RKV_ERR_UNSUPPORTED;
+    const int cap = rg->max_cap;
+    if (!budgets && (cfg->budget < cfg->window || cfg->budget >= cap)) return RKV_ERR_INVALID;
+    if (opts && opts->cluster_size != 0 && opts->cluster_size != 1) return RKV_ERR_UNSUPPORTED;
+    const int nqp = nqp_of((cfg->n_q_heads / cfg->n_kv_heads) * cfg->window);
+    const UnitShape us = unit_shape(cap, nqp);
+    if (!us.ok) return RKV_ERR_UNSUPPORTED;
+    if ((reinterpret_cast<uintptr_t>(rg->seq_row) & 7u) || (reinterpret_cast<uintptr_t>(rg->seq_cap) & 3u))
+        return RKV_ERR_ALIGN;
+    const size_t pool_bytes = static_cast<size_t>(rg->pool_rows) * kHeadDim * 2;
+    for (int l = 0; l < n_layers; ++l) {
+        if (!k_pools[l] || !v_pools[l] || !q_layers[l]) return RKV_ERR_NULL;
+        if (!aligned16(k_pools[l]) || !aligned16(v_pools[l]) || !aligned16(q_layers[l]))
+            return RKV_ERR_ALIGN;
+        if (overlap(k_pools[l], pool_bytes, v_pools[l], pool_bytes)) return RKV_ERR_ALIAS;
+    }
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return RKV_ERR_ALIGN;
+    if (ws_bytes < ws_bytes_for(cfg, n_layers, batch, cap)) return RKV_ERR_WORKSPACE;
+    if (cfg->redundancy_mode == RKV_RED_MAX && cap > gram_max_rows()) return RKV_ERR_UNSUPPORTED;
+
+    cudaStream_t strm = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    uint32_t *status = reinterpret_cast<uint32_t *>(ws);
+    int32_t *n_eff = reinterpret_cast<int32_t *>(ws + kStatusBytes);
+    float *r_ext = reinterpret_cast<float *>(ws + kStatusBytes + align256(static_cast<size_t>(batch) * 4));
+    const bool red_max = cfg->redundancy_mode == RKV_RED_MAX;
+    RaggedLayout lay;
+    lay.seq_row = rg->seq_row;
+    lay.seq_cap = rg->seq_cap;
+    lay.pool_rows = rg->pool_rows;
+    lay.n_kv = cfg->n_kv_heads;
+    // the plan kernel clears the status words first, then checks every due sequence's
+    // block against the pool
+    cudaError_t e = launch_plan(batch, budgets, cfg->budget, cfg->buffer, cfg->window, cap, cur_len,
+                                n_eff, status, strm, true, lay);
+    if (red_max && e == cudaSuccess)
+        e = launch_gram_layers(cfg, n_layers, batch, cap,
+                               const_cast<const rkv_bf16 *const *>(k_pools), n_eff, r_ext, status,
+                               strm, opts ? reinterpret_cast<cudaEvent_t>(opts->sim_begin) : nullptr,
+                               opts ? reinterpret_cast<cudaEvent_t>(opts->sim_end) : nullptr, lay);
+    if (e == cudaSuccess && opts && opts->main_begin)
+        e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->main_begin), strm);
+    if (e == cudaSuccess)
+        e = launch_unit_layers(cfg, n_layers, batch, cap,
+                               const_cast<const rkv_bf16 *const *>(k_pools), v_pools, q_layers,
+                               budgets, lambdas, n_eff, red_max ? r_ext : nullptr,
+                               opts ? opts->kept_out : nullptr, opts ? opts->scores_out : nullptr,
+                               nullptr, status, us, nqp, strm, PagedArgs{nullptr, 0, 0, 0}, lay);
     if (e == cudaSuccess && opts && opts->main_end)
         e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->main_end), strm);
     return cuda_status(e);

@@ -6,26 +6,36 @@
 // other keys is the near-duplicate reading of "cosine similarity to identify
 // and prune near-duplicates" (sourcepulse summary, "How It Works").
 //
-// One CTA per (unit, block of 128 candidate rows).  The Gram tiles
-// K_I . K_J^T are computed by tcgen05 UMMA (bf16 in, fp32 accumulate) into
-// TMEM and folded to row maxima on chip; the N x N matrix never reaches HBM.
-// A first pass (rkv_inv_norm_kernel) writes 1 / max(||k_j||, 1e-12) of every
-// row once, so the row blocks of a unit do not each recompute the norms of
-// every column tile.
-// Warp roles (320 threads):
-//   warps 0-7  epilogue: per row max_j acc_ij * inv_j from TMEM; warps w and
-//              w + 4 read the same 32 TMEM lanes (rows) and split the tile's
-//              128 columns;
-//   warp 8     producer: TMA of the row block once, then 128-row column tiles
-//              into a two-stage ring;
-//   warp 9     MMA issuer: 8 UMMAs (K = 128) per column tile into one of two
-//              TMEM accumulators (128 columns each).
+// With a_ij = k_i . k_j (bf16 products, fp32 accumulate on tcgen05) and
+// inv_i = 1 / max(||k_i||, 1e-12):  r_i = inv_i * u_i,  u_i = max_{j != i} a_ij inv_j.
+// The Gram matrix is symmetric, so only the tile pairs (I, J >= I) of 128 x 128
+// are computed: the accumulator of pair (I, J) gives u of the rows of tile I
+// (row maxima of a_ij inv_j) and u of the rows of tile J (column maxima of
+// a_ij inv_i).  The N x N matrix never leaves the chip, and the inverse norms
+// are computed here from the tiles already in shared memory: K is read once
+// from HBM (the tiles a unit reuses come from L2).
+//
+// Persistent CTAs (one per SM) walk the units; per unit the row tiles go from
+// last to first, so that when row I runs, the inverse norms of every tile
+// J >= I are known (tile J was the A operand of an earlier row).  Warp roles
+// (320 threads, one CTA per SM):
+//   warps 0-7  epilogue: inverse norms of each row tile; per pair, the
+//              accumulator read with tcgen05.ld 16x256b (each thread holds 4
+//              rows x 16 columns), row and column maxima folded in registers,
+//              across 4 and 8 lanes by shuffles, then merged into per-row
+//              order-preserving keys in shared memory with atomicMax;
+//   warp 8     producer: TMA of the row tile (double-buffered A) and of the
+//              column tiles (three-stage B ring);
+//   warp 9     MMA issuer: 8 UMMAs (K = 128) per pair into one of four TMEM
+//              accumulators (128 columns each); the diagonal pair uses the A
+//              tile as both operands.
 // Hand-offs are mbarriers; every wait is bounded and a timeout is recorded in
-// the status word.
+// the status word (the CTA then drains what it issued and stops).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 
 #include "rkv_block.cuh"
@@ -37,21 +47,32 @@ namespace rkv {
 namespace {
 
 constexpr int kGramThreads = 320;
-constexpr int kStages = 2;
-constexpr uint32_t kTileBytes = 128u * 256u;      // 128 rows x 128 bf16
-constexpr uint32_t kTmemCols = 256;               // two 128-column accumulators
+constexpr int kEpiThreads = 256;
+constexpr int kBStages = 3;
+constexpr int kAcc = 4;                            // TMEM accumulators of 128 columns
+constexpr uint32_t kTileBytes = 128u * 256u;       // 128 rows x 128 bf16
+constexpr uint32_t kHalfBytes = kTileBytes / 2;
+constexpr uint32_t kTmemCols = 128u * kAcc;
 
-struct GramSmem {
-    uint8_t a[kTileBytes];                 // row block (two 64-column halves)
-    uint8_t b[kStages][kTileBytes];        // column tiles
-    float inv_b[2][128];                   // inverse norms of the column tile in each accumulator
-    float inv_a[128];
-    float part[128];                       // row maxima of the second column half
-    uint64_t bar_a;
-    uint64_t full[kStages], empty[kStages];
-    uint64_t tfull[2], tempty[2];
-    uint32_t tmem;
+struct GramLayout {
+    uint32_t a, b, key, inv, pages, bars, total;
 };
+
+// Offsets from a 1024-byte-aligned base; key and inv hold one entry per row of
+// the largest unit (rounded up to whole tiles).
+__host__ __device__ inline GramLayout gram_layout(int cap) {
+    GramLayout L;
+    const uint32_t kc = static_cast<uint32_t>((cap + 127) / 128) * 128u;
+    uint32_t o = 0;
+    L.a = o;     o += 2u * kTileBytes;
+    L.b = o;     o += kBStages * kTileBytes;
+    L.key = o;   o += 4u * kc;
+    L.inv = o;   o += 4u * kc;
+    L.pages = o; o += 4u * kUnitMaxPages;
+    L.bars = o;  o += 256u;
+    L.total = o + 1024u;
+    return L;
+}
 
 // max(a, b, c) in one instruction.
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -60,166 +81,379 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return r;
 }
 
-// max(best, c[0..31]) as a tree of three-input maxima.
-__device__ __forceinline__ float max_of_32(float best, const float (&c)[32]) {
-    float t[11];
-#pragma unroll
-    for (int q = 0; q < 10; ++q) t[q] = fmax3(c[3 * q], c[3 * q + 1], c[3 * q + 2]);
-    t[10] = fmaxf(c[30], c[31]);
-    const float u0 = fmax3(t[0], t[1], t[2]), u1 = fmax3(t[3], t[4], t[5]);
-    const float u2 = fmax3(t[6], t[7], t[8]), u3 = fmax3(t[9], t[10], best);
-    return fmax3(u0, u1, fmaxf(u2, u3));
+// Order-preserving unsigned key of a float (larger float, larger key); 0 is
+// below every key of a float, so a cleared array means "no value yet".
+__device__ __forceinline__ uint32_t ord_key(float f) {
+    const uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-__device__ __forceinline__ void named_sync_epilogue() {
-    asm volatile("bar.sync 1, 256;" ::: "memory");
+__device__ __forceinline__ float key_value(uint32_t k) {
+    if (k == 0u) return -INFINITY;
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+// 16 TMEM lanes x 64 fp32 columns (16x256b, 8 repetitions): thread t gets, for
+// repetition k, lane (t / 4) columns 8k + 2 (t % 4) + {0, 1} in r[4k], r[4k+1]
+// and lane (t / 4) + 8 the same columns in r[4k+2], r[4k+3].
+__device__ __forceinline__ void tmem_ld_16x256b_x8(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x8.b32"
+        " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15,"
+        " %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void reg_tie32(uint32_t (&r)[32]) {
+#pragma unroll
+    for (int i = 0; i < 32; i += 8)
+        asm volatile("" : "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]),
+                     "+r"(r[i + 4]), "+r"(r[i + 5]), "+r"(r[i + 6]), "+r"(r[i + 7])::"memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// The unit a persistent CTA handles k-th, its cache length and its rows.
+struct UnitInfo {
+    int N, M, T, b, h, l;
+    int64_t unit_g, krow0;
+};
+
+__device__ __forceinline__ UnitInfo unit_info(const GramParams &p, int unit) {
+    UnitInfo u;
+    u.h = unit % p.n_kv;
+    u.b = (unit / p.n_kv) % p.batch;
+    u.l = unit / (p.n_kv * p.batch);
+    u.N = p.n_tokens_fixed > 0 ? p.n_tokens_fixed : p.n_eff[u.b];
+    u.M = u.N - p.window;
+    u.T = (u.N + 127) / 128;
+    u.unit_g = (static_cast<int64_t>(p.layer_base + u.l) * p.batch + u.b) * p.n_kv + u.h;
+    u.krow0 = unit_first_row(p.seq_row, p.seq_cap, u.b, u.h, p.n_kv, p.cap);
+    return u;
 }
 
 }  // namespace
 
-__global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __grid_constant__ GramParams p) {
+__global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __grid_constant__ GramParams p,
+                                                                      int n_units) {
     extern __shared__ uint8_t smem_raw[];
-    GramSmem &S = *reinterpret_cast<GramSmem *>(
+    uint8_t *base = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    // a programmatic dependent of the inverse-norm pass: wait for it before reading
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const GramLayout Lg = gram_layout(p.cap);
+    uint8_t *sA = base + Lg.a;
+    uint8_t *sB = base + Lg.b;
+    uint32_t *sKey = reinterpret_cast<uint32_t *>(base + Lg.key);
+    float *sInv = reinterpret_cast<float *>(base + Lg.inv);
+    int32_t *sPages = reinterpret_cast<int32_t *>(base + Lg.pages);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(base + Lg.bars);
+    uint64_t *afull = bars, *aempty = bars + 2, *bfull = bars + 4, *bempty = bars + 4 + kBStages;
+    uint64_t *tfull = bars + 4 + 2 * kBStages, *tempty = tfull + kAcc;
+    uint32_t *sTmem = reinterpret_cast<uint32_t *>(tempty + kAcc);
+
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int unit = blockIdx.x / p.nblk, bi = blockIdx.x % p.nblk;
-    const int h = unit % p.n_kv;
-    const int b = (unit / p.n_kv) % p.batch;
-    const int l = unit / (p.n_kv * p.batch);
-    const int N = p.n_tokens_fixed > 0 ? p.n_tokens_fixed : p.n_eff[b];
-    const int M = N - p.window;
-    const int i0 = bi * 128;
-    if (N <= 0 || i0 >= M) return;
-    const int n_tiles = (N + 127) / 128;
-    const int64_t krow0 = (static_cast<int64_t>(b) * p.n_kv + h) * p.cap;
-    const int64_t unit_g = (static_cast<int64_t>(p.layer_base + l) * p.batch + b) * p.n_kv + h;
-    const CUtensorMap *map = &p.tmap[l];
+    const int kc = (p.cap + 127) / 128 * 128;
+    const bool paged = p.block_table != nullptr;
+    const int psh = paged ? 31 - __clz(p.page_rows) : 7;
+    const int P = 1 << psh;
 
     if (warp == 0) {
-        tmem_alloc(&S.tmem, kTmemCols);
+        tmem_alloc(sTmem, kTmemCols);
         tmem_relinquish();
     }
-    if (tid == 0) {
-        mbar_init(&S.bar_a, 1);
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(&S.full[s], 1);
-            mbar_init(&S.empty[s], 1);   // the MMA is done reading the tile
+    if (tid == 32) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&afull[i], 1);
+            mbar_init(&aempty[i], 2);        // the row's last UMMA + the epilogue's norm pass
         }
-        for (int t = 0; t < 2; ++t) {
-            mbar_init(&S.tfull[t], 1);
-            mbar_init(&S.tempty[t], 1);
+        for (int s = 0; s < kBStages; ++s) {
+            mbar_init(&bfull[s], 1);
+            mbar_init(&bempty[s], 1);
+        }
+        for (int t = 0; t < kAcc; ++t) {
+            mbar_init(&tfull[t], 1);
+            mbar_init(&tempty[t], 8);        // one arrival per epilogue warp
         }
         fence_mbar_init();
     }
+    for (int i = tid; i < kc; i += kGramThreads) sKey[i] = 0u;
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem_base = S.tmem;
-    bool ok = true;
+    const uint32_t tmem_base = *sTmem;
+    // a programmatic dependent of the plan kernel: nothing it wrote is read before this
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
+    bool ok = true;
     if (warp == 8) {
-        // ---------------- producer
-        if (lane == 0) {
-            mbar_arrive_expect_tx(&S.bar_a, kTileBytes);
-            tma_load_2d(S.a, map, &S.bar_a, 0, static_cast<int32_t>(krow0 + i0));
-            tma_load_2d(S.a + 16384, map, &S.bar_a, 64, static_cast<int32_t>(krow0 + i0));
-            for (int jt = 0; jt < n_tiles && ok; ++jt) {
-                const int s = jt % kStages;
-                if (jt >= kStages && !mbar_wait(&S.empty[s], ((jt / kStages) - 1) & 1)) {
-                    ok = false;
-                    break;
-                }
-                mbar_arrive_expect_tx(&S.full[s], kTileBytes);
-                const int32_t y = static_cast<int32_t>(krow0 + jt * 128);
-                tma_load_2d(S.b[s], map, &S.full[s], 0, y);
-                tma_load_2d(S.b[s] + 16384, map, &S.full[s], 64, y);
+        // ---------------- producer: per unit, row tiles T-1 .. 0 into A, column tiles into B
+        uint32_t na = 0, nb = 0;
+        for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x) {
+            const UnitInfo u = unit_info(p, unit);
+            if (u.N <= 0 || u.M <= 0) continue;
+            const CUtensorMap *map = &p.tmap[u.l];
+            if (paged) {
+                __syncwarp();
+                for (int j = lane; j < (u.N + P - 1) / P; j += 32)
+                    sPages[j] = p.block_table[static_cast<int64_t>(u.b) * p.max_blocks + j];
+                __syncwarp();
             }
+            const int npg = (u.N + P - 1) / P;
+            auto load_tile = [&](uint8_t *dst, uint64_t *bar, int t) {
+                if (!paged) {
+                    const int32_t y = static_cast<int32_t>(u.krow0 + t * 128);
+                    tma_load_2d(dst, map, bar, 0, y);
+                    tma_load_2d(dst + kHalfBytes, map, bar, 64, y);
+                } else {
+                    // one box per page; pages past the sequence's last read as zeros
+                    for (int j = 0; j < 128 / P; ++j) {
+                        const int pg = t * (128 / P) + j;
+                        const int32_t y = pg < npg
+                                              ? static_cast<int32_t>(((static_cast<int64_t>(sPages[pg]) * p.n_kv + u.h) << psh))
+                                              : -P;
+                        tma_load_2d(dst + j * P * 128, map, bar, 0, y);
+                        tma_load_2d(dst + kHalfBytes + j * P * 128, map, bar, 64, y);
+                    }
+                }
+            };
+            for (int I = u.T - 1; I >= 0 && ok; --I) {
+                if (lane == 0) {
+                    const uint32_t a = na & 1u;
+                    if (na >= 2 && !mbar_wait(&aempty[a], ((na >> 1) - 1) & 1u)) ok = false;
+                    if (ok) {
+                        mbar_arrive_expect_tx(&afull[a], kTileBytes);
+                        load_tile(sA + a * kTileBytes, &afull[a], I);
+                    }
+                    ++na;
+                    for (int J = I + 1; J < u.T && ok; ++J) {
+                        const uint32_t s = nb % kBStages;
+                        if (nb >= kBStages && !mbar_wait(&bempty[s], ((nb / kBStages) - 1) & 1u)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&bfull[s], kTileBytes);
+                        load_tile(sB + s * kTileBytes, &bfull[s], J);
+                        ++nb;
+                    }
+                }
+                ok = __shfl_sync(kFull, ok ? 1 : 0, 0) != 0;
+            }
+        }
+        if (!ok && lane == 0) {
+            // drain (bounded): the copies still in flight land before shared memory goes
+            for (uint32_t i = na >= 2 ? na - 2 : 0; i < na; ++i)
+                (void)mbar_wait(&afull[i & 1u], (i >> 1) & 1u);
+            for (uint32_t i = nb >= kBStages ? nb - kBStages : 0; i < nb; ++i)
+                (void)mbar_wait(&bfull[i % kBStages], (i / kBStages) & 1u);
         }
     } else if (warp == 9) {
         // ---------------- MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
-            if (!mbar_wait(&S.bar_a, 0)) ok = false;
-            tc_fence_after();
-            const uint32_t a_base = smem_u32(S.a);
-            for (int jt = 0; jt < n_tiles && ok; ++jt) {
-                const int s = jt % kStages, t = jt & 1;
-                if (!mbar_wait(&S.full[s], (jt / kStages) & 1)) { ok = false; break; }
-                if (jt >= 2 && !mbar_wait(&S.tempty[t], ((jt >> 1) - 1) & 1)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t b_base = smem_u32(S.b[s]);
+            uint32_t na = 0, nb = 0, np = 0;
+            for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x) {
+                const UnitInfo u = unit_info(p, unit);
+                if (u.N <= 0 || u.M <= 0) continue;
+                for (int I = u.T - 1; I >= 0 && ok; --I) {
+                    const uint32_t a = na & 1u;
+                    if (!mbar_wait(&afull[a], (na >> 1) & 1u)) { ok = false; break; }
+                    ++na;
+                    const uint32_t a_base = smem_u32(sA + a * kTileBytes);
+                    for (int J = I; J < u.T && ok; ++J) {
+                        const uint32_t t = np % kAcc;
+                        if (np >= kAcc && !mbar_wait(&tempty[t], ((np / kAcc) - 1) & 1u)) { ok = false; break; }
+                        uint32_t b_base = a_base, s = 0;
+                        if (J > I) {
+                            s = nb % kBStages;
+                            if (!mbar_wait(&bfull[s], (nb / kBStages) & 1u)) { ok = false; break; }
+                            b_base = smem_u32(sB + s * kTileBytes);
+                        }
+                        tc_fence_after();
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t off = (ks >> 2) * 16384u + (ks & 3) * 32u;
-                    umma_bf16(tmem_base + t * 128u, desc_kmajor_sw128(a_base + off),
-                              desc_kmajor_sw128(b_base + off), idesc, ks > 0 ? 1u : 0u);
+                        for (int ks = 0; ks < 8; ++ks) {
+                            const uint32_t off = (ks >> 2) * kHalfBytes + (ks & 3) * 32u;
+                            umma_bf16(tmem_base + t * 128u, desc_kmajor_sw128(a_base + off),
+                                      desc_kmajor_sw128(b_base + off), idesc, ks > 0 ? 1u : 0u);
+                        }
+                        umma_commit(&tfull[t]);
+                        ++np;
+                        if (J > I) {
+                            umma_commit(&bempty[s]);
+                            ++nb;
+                        }
+                    }
+                    if (ok) umma_commit(&aempty[a]);
                 }
-                umma_commit(&S.tfull[t]);
-                umma_commit(&S.empty[s]);
             }
+            // drain (bounded): every UMMA issued so far completes before TMEM is freed
+            if (!ok && np > 0) (void)mbar_wait(&tfull[(np - 1) % kAcc], ((np - 1) / kAcc) & 1u);
         }
     } else {
-        // ---------------- epilogue warps 0-7: row i0 + (tid & 127), column half tid >> 7
-        const int lrow = tid & 127, chalf = tid >> 7;
-        const int i = i0 + lrow;
-        const float *inv_g = p.inv + unit_g * p.cap;
-        if (tid < 128) {
-            S.inv_a[tid] = (i0 + tid < N) ? inv_g[i0 + tid] : 0.f;
-            S.inv_b[0][tid] = (tid < N) ? inv_g[tid] : 0.f;
-        }
-        named_sync_epilogue();
-        float best = -INFINITY;
-        for (int jt = 0; jt < n_tiles; ++jt) {
-            const int t = jt & 1;
-            // the next tile's inverse norms: loaded now, stored after this tile's epilogue
-            float nxt = 0.f;
-            if (tid < 128 && jt + 1 < n_tiles && (jt + 1) * 128 + tid < N) nxt = inv_g[(jt + 1) * 128 + tid];
-            if (ok && !mbar_wait(&S.tfull[t], (jt >> 1) & 1)) ok = false;
-            tc_fence_after();
-            const int j0 = jt * 128 + chalf * 64;
-            const bool clean = (jt * 128 + 128 <= N) && (jt != bi);
-            const uint32_t taddr = tmem_base + ((32u * (warp & 3)) << 16) + t * 128u + chalf * 64u;
-            const float *invt = &S.inv_b[t][chalf * 64];
+        // ---------------- epilogue warps 0-7: quadrant qd of TMEM lanes, column half ch
+        const int qd = warp & 3, ch = warp >> 2;
+        const int g = lane >> 2, q = lane & 3;
+        // this thread's 4 tile rows 32 qd + g + 8 r (r = 0, 1: the first 16-lane slab,
+        // r = 2, 3: the second) and the row it keeps after the 4-lane fold (r = q)
+        auto row_of = [&](int r) { return 32 * qd + g + 8 * r; };
+        const int myrow = row_of(q);
+        // norms: two threads per row, 64 columns each
+        const int nrow = (lane & 7) + 8 * (lane >> 4), nhalf = (lane >> 3) & 1;
+        const int row_t = 16 * warp + nrow;
+        uint32_t na = 0, np = 0;
+        for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x) {
+            const UnitInfo u = unit_info(p, unit);
+            if (u.N <= 0 || u.M <= 0) continue;
+            for (int I = u.T - 1; I >= 0 && ok; --I) {
+                const uint32_t a = na & 1u;
+                if (!mbar_wait(&afull[a], (na >> 1) & 1u)) { ok = false; break; }
+                ++na;
+                {
+                    // 1 / max(||k_i||, 1e-12) of the row tile's rows (0 past N)
+                    const uint8_t *hp = sA + a * kTileBytes + nhalf * kHalfBytes + row_t * 128;
+                    float2 ss2 = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int c0 = 0; c0 < 64; c0 += 32) {
-                // 32 columns in flight per wait
-                uint32_t r0[16], r1[16];
-                tmem_ld16_nowait(taddr + c0, r0);
-                tmem_ld16_nowait(taddr + c0 + 16, r1);
-                tmem_wait_ld();
-                reg_tie16(r0);
-                reg_tie16(r1);
-                float c[32];
-                const float4 *iv4 = reinterpret_cast<const float4 *>(invt + c0);
+                    for (int c = 0; c < 8; ++c) {
+                        const uint4 raw = *reinterpret_cast<const uint4 *>(hp + ((c ^ (row_t & 7)) << 4));
+                        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const float4 iv = iv4[q];
-                    const uint32_t *rr = q < 4 ? &r0[4 * q] : &r1[4 * (q - 4)];
-                    const float2 a = __fmul2_rn(make_float2(__uint_as_float(rr[0]), __uint_as_float(rr[1])),
-                                                make_float2(iv.x, iv.y));
-                    const float2 bb = __fmul2_rn(make_float2(__uint_as_float(rr[2]), __uint_as_float(rr[3])),
-                                                 make_float2(iv.z, iv.w));
-                    c[4 * q] = a.x; c[4 * q + 1] = a.y; c[4 * q + 2] = bb.x; c[4 * q + 3] = bb.y;
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f = __bfloat1622float2(h2[e]);
+                            ss2 = __ffma2_rn(f, f, ss2);
+                        }
+                    }
+                    const float ssh = ss2.x + ss2.y;
+                    const float ss = ssh + __shfl_xor_sync(kFull, ssh, 8);
+                    const int i = I * 128 + row_t;
+                    if (nhalf == 0) sInv[i] = i < u.N ? 1.0f / fmaxf(sqrtf(ss), 1e-12f) : 0.f;
                 }
-                if (clean) {
-                    best = max_of_32(best, c);
-                } else {
+                epi_sync();
+                if (tid == 0) mbar_arrive(&aempty[a]);   // the epilogue is done reading A
+                float inv_r[4];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int j = j0 + c0 + e;
-                        best = (j < N && j != i) ? fmaxf(best, c[e]) : best;
+                for (int r = 0; r < 4; ++r) inv_r[r] = sInv[I * 128 + row_of(r)];
+                float rrun = -INFINITY;
+                for (int J = I; J < u.T && ok; ++J) {
+                    const uint32_t t = np % kAcc;
+                    if (!mbar_wait(&tfull[t], (np / kAcc) & 1u)) { ok = false; break; }
+                    ++np;
+                    tc_fence_after();
+                    uint32_t v0[32], v1[32];   // slab 0 (rows 0, 1), slab 1 (rows 2, 3)
+                    const uint32_t tcol = tmem_base + t * 128u + 64u * ch;
+                    tmem_ld_16x256b_x8(tcol + ((32u * qd) << 16), v0);
+                    tmem_ld_16x256b_x8(tcol + ((32u * qd + 16u) << 16), v1);
+                    tmem_wait_ld();
+                    reg_tie32(v0);
+                    reg_tie32(v1);
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&tempty[t]);   // the accumulator may be reused
+                    // a(row r, column k, e): slab r >> 1, register 4k + 2 (r & 1) + e
+                    auto av = [&](int r, int k, int e) -> float {
+                        const uint32_t x = (r < 2) ? v0[4 * k + 2 * (r & 1) + e] : v1[4 * k + 2 * (r & 1) + e];
+                        return __uint_as_float(x);
+                    };
+                    const int c0 = J * 128 + 64 * ch + 2 * q;    // unit row of column (k = 0, e = 0)
+                    float inv_c[16];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const float2 iv = *reinterpret_cast<const float2 *>(&sInv[c0 + 8 * k]);
+                        inv_c[2 * k] = iv.x;
+                        inv_c[2 * k + 1] = iv.y;
+                    }
+                    // ---- rows of tile I: max over this pair's columns of a_ij inv_j
+                    const bool diag = J == I, tail = (J + 1) * 128 > u.N;
+                    float rm[4];
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        float x[16];
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            const float2 pr = __fmul2_rn(make_float2(av(r, k, 0), av(r, k, 1)),
+                                                         make_float2(inv_c[2 * k], inv_c[2 * k + 1]));
+                            x[2 * k] = pr.x;
+                            x[2 * k + 1] = pr.y;
+                        }
+                        if (diag || tail) {
+                            const int ri = I * 128 + row_of(r);
+#pragma unroll
+                            for (int k = 0; k < 8; ++k)
+#pragma unroll
+                                for (int e = 0; e < 2; ++e) {
+                                    const int cj = c0 + 8 * k + e;
+                                    if (cj == ri || cj >= u.N) x[2 * k + e] = -INFINITY;
+                                }
+                        }
+                        const float m0 = fmax3(x[0], x[1], x[2]), m1 = fmax3(x[3], x[4], x[5]);
+                        const float m2 = fmax3(x[6], x[7], x[8]), m3 = fmax3(x[9], x[10], x[11]);
+                        const float m4 = fmax3(x[12], x[13], x[14]);
+                        rm[r] = fmax3(fmax3(m0, m1, m2), fmax3(m3, m4, x[15]), -INFINITY);
+                    }
+                    // fold across the 4 lanes of a row group: lane q keeps row q
+                    {
+                        const bool up = (q & 2) != 0;
+                        const float s0 = up ? rm[0] : rm[2], s1 = up ? rm[1] : rm[3];
+                        float k0 = up ? rm[2] : rm[0], k1 = up ? rm[3] : rm[1];
+                        k0 = fmaxf(k0, __shfl_xor_sync(kFull, s0, 2));
+                        k1 = fmaxf(k1, __shfl_xor_sync(kFull, s1, 2));
+                        const bool up1 = (q & 1) != 0;
+                        const float s2 = up1 ? k0 : k1;
+                        float kk = up1 ? k1 : k0;
+                        kk = fmaxf(kk, __shfl_xor_sync(kFull, s2, 1));
+                        rrun = fmaxf(rrun, kk);
+                    }
+                    if (!diag) {
+                        // ---- rows of tile J (columns here): max over tile I's rows of a_ij inv_i
+                        float cm[16];
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                const float2 pa = __fmul2_rn(make_float2(av(0, k, e), av(1, k, e)),
+                                                             make_float2(inv_r[0], inv_r[1]));
+                                const float2 pb = __fmul2_rn(make_float2(av(2, k, e), av(3, k, e)),
+                                                             make_float2(inv_r[2], inv_r[3]));
+                                cm[2 * k + e] = fmax3(fmaxf(pa.x, pa.y), pb.x, pb.y);
+                            }
+                        // fold across the 8 lanes of a column group: lane g keeps columns
+                        // 2g, 2g + 1 of its 16 (k = g)
+#pragma unroll
+                        for (int lvl = 0; lvl < 3; ++lvl) {
+                            const int half = 8 >> lvl;              // values kept after this round
+                            const int bit = 4 >> lvl;               // lane bit (of g) exchanged
+                            const bool upper = (g & bit) != 0;
+#pragma unroll
+                            for (int i = 0; i < half; ++i) {
+                                const float send = upper ? cm[i] : cm[i + half];
+                                const float keep = upper ? cm[i + half] : cm[i];
+                                cm[i] = fmaxf(keep, __shfl_xor_sync(kFull, send, bit * 4));
+                            }
+                        }
+                        const int cj = c0 + 8 * g;
+                        atomicMax(&sKey[cj], ord_key(cm[0]));
+                        atomicMax(&sKey[cj + 1], ord_key(cm[1]));
                     }
                 }
+                if (!ok) break;
+                atomicMax(&sKey[I * 128 + myrow], ord_key(rrun));
             }
-            if (tid < 128 && jt + 1 < n_tiles) S.inv_b[t ^ 1][tid] = nxt;   // read last in tile jt - 1
-            tc_fence_before();
-            named_sync_epilogue();
-            if (tid == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&S.tempty[t])) : "memory");
+            if (!ok) break;
+            // every key of the unit is final: r = inv_i * u_i; then clear for the next unit
+            epi_sync();
+            float *ro = p.r_out + u.unit_g * p.cap;
+            for (int i = tid; i < u.T * 128; i += kEpiThreads) {
+                if (i < u.M) ro[i] = key_value(sKey[i]) * sInv[i];
+                sKey[i] = 0u;
+            }
+            epi_sync();
         }
-        if (chalf == 1) S.part[lrow] = best;
-        named_sync_epilogue();
-        if (chalf == 0 && i < M) p.r_out[unit_g * p.cap + i] = fmaxf(best, S.part[lrow]) * S.inv_a[lrow];
     }
     if (!ok) record_flag(p.status, kDevFlagTimeout);
     __syncthreads();
@@ -229,68 +463,43 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
     }
 }
 
-// 1 / max(||k_j||, 1e-12) of every row of every due unit: half a warp per row
-// (16 lanes x 8 columns), 64 rows per CTA.
-__global__ void __launch_bounds__(256) rkv_inv_norm_kernel(const __grid_constant__ GramParams p,
-                                                           int nchunk) {
-    // a programmatic dependent of the plan kernel: wait for it before reading
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    const int unit = blockIdx.x / nchunk, chunk = blockIdx.x % nchunk;
-    const int h = unit % p.n_kv;
-    const int b = (unit / p.n_kv) % p.batch;
-    const int l = unit / (p.n_kv * p.batch);
-    const int N = p.n_tokens_fixed > 0 ? p.n_tokens_fixed : p.n_eff[b];
-    if (N <= 0 || chunk * 64 >= N) return;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, half = lane >> 4, sub = lane & 15;
-    const int64_t krow0 = (static_cast<int64_t>(b) * p.n_kv + h) * p.cap;
-    const int64_t unit_g = (static_cast<int64_t>(p.layer_base + l) * p.batch + b) * p.n_kv + h;
-#pragma unroll
-    for (int it = 0; it < 4; ++it) {
-        const int row = chunk * 64 + warp * 8 + it * 2 + half;
-        float2 ss2 = make_float2(0.f, 0.f);
-        if (row < N) {
-            const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(p.k[l] + (krow0 + row) * kHeadDim) + sub);
-            const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 f = __bfloat1622float2(h2[e]);
-                ss2 = __ffma2_rn(f, f, ss2);
-            }
-        }
-        float ss = ss2.x + ss2.y;
-#pragma unroll
-        for (int off = 8; off >= 1; off >>= 1) ss += __shfl_xor_sync(kFull, ss, off);
-        if (row < N && sub == 0) p.inv[unit_g * p.cap + row] = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
-    }
-}
+size_t gram_smem_bytes(int cap) { return gram_layout(cap).total; }
 
-size_t gram_smem_bytes() { return sizeof(GramSmem) + 1024; }
+int gram_max_rows() {
+    // rows whose keys and inverse norms still fit next to the tiles
+    int cap = kUnitMaxRows;
+    while (cap > 128 && gram_layout(cap).total > 232448u) cap -= 128;
+    return cap;
+}
 
 cudaError_t launch_gram_max(const GramParams &p, int n_units, cudaStream_t stream,
                             cudaEvent_t before_gram, cudaEvent_t after_gram) {
-    const size_t smem = gram_smem_bytes();
+    const size_t smem = gram_smem_bytes(p.cap);
     static std::atomic<int> granted{0};
     cudaError_t e = ensure_smem_attr(rkv_gram_max_kernel, smem, granted);
     if (e != cudaSuccess) return e;
-    const int nchunk = (p.cap + 63) / 64;
-    // both launched as programmatic dependents of the kernel before them: their CTAs may
-    // be scheduled while it finishes, and wait for it on the device
+    static int n_sm = 0;
+    if (n_sm == 0) {
+        int dev = 0, v = 0;
+        e = cudaGetDevice(&dev);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        n_sm = v;
+    }
+    // launched as a programmatic dependent of the kernel before it: the CTAs may be
+    // scheduled while it finishes, and wait for it on the device
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(n_units * nchunk), 1, 1);
-    cfg.blockDim = dim3(256, 1, 1);
+    cfg.gridDim = dim3(static_cast<unsigned>(n_units < n_sm ? n_units : n_sm), 1, 1);
+    cfg.blockDim = dim3(kGramThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, rkv_inv_norm_kernel, p, nchunk);
-    if (e == cudaSuccess && before_gram) e = cudaEventRecord(before_gram, stream);
-    if (e != cudaSuccess) return e;
-    cfg.gridDim = dim3(static_cast<unsigned>(n_units * p.nblk), 1, 1);
-    cfg.blockDim = dim3(kGramThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    e = cudaLaunchKernelEx(&cfg, rkv_gram_max_kernel, p);
+    if (before_gram) e = cudaEventRecord(before_gram, stream);
+    if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, rkv_gram_max_kernel, p, n_units);
     if (e == cudaSuccess && after_gram) e = cudaEventRecord(after_gram, stream);
     return e;
 }

@@ -4,6 +4,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <atomic>
 #include <cstddef>
 #include <cstdint>
@@ -11,6 +12,16 @@
 #include "../../include/rkv.h"
 
 namespace rkv {
+
+// An NVTX range around one entry point (host side): profilers that record NVTX
+// show each call of the library as a named span over the kernels it enqueues.
+// Header-only NVTX: without an attached tool a push / pop costs a few ns.
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 constexpr int kHeadDim = 128;
 constexpr int kMaxLayersPerLaunch = 32;
@@ -122,10 +133,29 @@ inline cudaError_t ensure_smem_attr(K kernel, size_t bytes, std::atomic<int> &gr
     return e;
 }
 
+// Caches with per-sequence capacities: each layer's K (and V) is one pool of
+// pool_rows rows of 128 bf16, and sequence b's [Hkv][seq_cap[b]] block starts at
+// row seq_row[b].  seq_row == null: the uniform [batch][Hkv][cap] layout.
+struct RaggedLayout {
+    const int64_t *seq_row = nullptr;   // device [batch]
+    const int32_t *seq_cap = nullptr;   // device [batch]
+    int64_t pool_rows = 0;
+    int32_t n_kv = 0;
+};
+
+// First row of unit (b, h) in its layer's 2-D [rows, 128] view.
+__device__ __forceinline__ int64_t unit_first_row(const int64_t *seq_row, const int32_t *seq_cap,
+                                                  int b, int h, int n_kv, int cap) {
+    return seq_row ? seq_row[b] + static_cast<int64_t>(h) * seq_cap[b]
+                   : (static_cast<int64_t>(b) * n_kv + h) * cap;
+}
+
 // Launchers (defined in the .cu files); all return cudaSuccess or the launch error.
+// cap: the uniform capacity, or with a ragged layout the largest seq_cap allowed.
 cudaError_t launch_plan(int batch, const int32_t *budgets, int32_t budget_cfg, int32_t buffer,
                         int32_t window, int32_t cap, int32_t *cur_len, int32_t *n_eff,
-                        uint32_t *status, cudaStream_t stream, bool update = true);
+                        uint32_t *status, cudaStream_t stream, bool update = true,
+                        const RaggedLayout &rg = RaggedLayout{});
 cudaError_t launch_step(const StepParams &p, int n_units, int nqp, size_t smem,
                         cudaStream_t stream);
 size_t step_smem_bytes(int rp, int rmax, int cap, int nqp, int cs);
@@ -164,6 +194,9 @@ struct alignas(64) UnitParams {
     // one page; logical row i of sequence b is in page block_table[b][i / page_rows]
     const int32_t *block_table;   // [batch][max_blocks] or null (contiguous caches)
     int32_t max_blocks, page_rows;
+    // per-sequence capacities (null: uniform [batch][Hkv][cap]; cap is then the largest)
+    const int64_t *seq_row;
+    const int32_t *seq_cap;
     uint32_t *status;
 };
 
@@ -172,27 +205,28 @@ constexpr int kUnitMaxPages = 512;     // pages of one sequence staged in shared
 constexpr int kUnitMaxRows = 7680;     // keys + destinations + histograms fit the 64 KB ring
 
 struct UnitLayout {
-    uint32_t stage, b, bs, inv, self, ia, ib, r, scr, s, colm, colf, vis, red, bt, bars, total;
+    uint32_t stage, b, bs, ss, ihat, r, scr, s, colm, colf, vis, red, bt, bars, total;
 };
 
 // Offsets from a 1024-byte-aligned base.  Lifetimes share bytes: the two 32 KB
 // ring stages hold, after the last tile, the select keys, the destinations and
 // the histograms; the B operand of the S UMMA (pass 1) shares bytes with the
-// pass-2 arrays Ihat halves and r (the last S UMMA completes between the passes).
+// pass-2 arrays Ihat and r (the last S UMMA completes between the passes).  Per
+// row only ||k||^2 crosses from pass 1 to pass 2 (the inverse norm is recomputed
+// from it), and the two warpgroups' importance partials meet in one array, so
+// that caches of up to about 2500 rows still fit two CTAs on an SM.
 __host__ __device__ inline UnitLayout make_unit_layout(int nmax, int nqp) {
     UnitLayout L;
     uint32_t o = 0;
     L.stage = o;  o += 2u * 32768u;
     L.b = o;      o += 2u * (nqp + 16u) * 128u;        // queries + split S, two swizzled halves
     const uint32_t arr = align_up(static_cast<uint32_t>(nmax) * 4u, 16);
-    L.inv = o;    o += arr;
-    L.self = o;   o += arr;
+    L.ss = o;     o += arr;
     o = align_up(o, 1024);
     L.bs = o;                                          // pass 1: inv split, 2 x 4 KB
-    L.ia = o;                                          // pass 2: Ihat halves and r
-    L.ib = o + arr;
-    L.r = o + 2u * arr;
-    o += (3u * arr > 8192u) ? 3u * arr : 8192u;
+    L.ihat = o;                                        // pass 2: Ihat and r
+    L.r = o + arr;
+    o += (2u * arr > 8192u) ? 2u * arr : 8192u;
     L.scr = o;    o += 2048u;                          // column (max, sum) per warp
     L.s = o;      o += 512u;
     L.colm = o;   o += 256u;
@@ -232,19 +266,21 @@ cudaError_t launch_freed_pages(int batch, const int32_t *budgets, int32_t budget
 
 // MAX-mode similarity kernel: raw r of every candidate of every due unit.
 struct alignas(64) GramParams {
-    CUtensorMap tmap[kMaxLayersPerLaunch];   // [B*Hkv*cap rows, 128] bf16, box 64 x 128, SW128
-    const uint16_t *k[kMaxLayersPerLaunch];  // the same caches, for the inverse-norm pass
-    int32_t layer_base, batch, n_kv, window, cap, nblk;
+    CUtensorMap tmap[kMaxLayersPerLaunch];   // [rows, 128] bf16, box 64 x 128 (paged: 64 x page_rows), SW128
+    int32_t layer_base, batch, n_kv, window, cap;
     int32_t n_tokens_fixed;  // > 0: per-head entry point, N fixed
     const int32_t *n_eff;
+    const int64_t *seq_row;  // per-sequence capacities, as in UnitParams (or null)
+    const int32_t *seq_cap;
+    const int32_t *block_table;   // paged caches, as in UnitParams (or null)
+    int32_t max_blocks, page_rows;
     float *r_out;            // [units][cap]
-    float *inv;              // [units][cap] 1 / max(||k||, 1e-12), written by the first pass
     uint32_t *status;
 };
-// before_gram / after_gram (or null): recorded around the similarity kernel itself
-// (after the inverse-norm pass).
+// before_gram / after_gram (or null): recorded around the similarity kernel.
 cudaError_t launch_gram_max(const GramParams &p, int n_units, cudaStream_t stream,
                             cudaEvent_t before_gram = nullptr, cudaEvent_t after_gram = nullptr);
+int gram_max_rows();   // longest unit the similarity kernel holds
 
 struct AppendParams {
     uint16_t *k[kMaxLayersPerLaunch];
@@ -257,6 +293,5 @@ struct AppendParams {
 };
 cudaError_t launch_append(const AppendParams &p, int n_layers, cudaStream_t stream);
 cudaError_t launch_bump(int batch, int n_new, int cap, int32_t *cur_len, cudaStream_t stream);
-size_t gram_smem_bytes();
 
 }  // namespace rkv

@@ -32,7 +32,7 @@ std::mutex g_mutex;
 void *g_scratch_addr[kMaxDevices] = {};
 
 // Device address of the scratch array on the current device, looked up once per
-// device (with that device current) and cached.
+// device (with that device current) and cached for the life of the process.
 rkv_status scratch_address(void **out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) return RKV_ERR_CUDA;
@@ -64,10 +64,20 @@ extern "C" rkv_status rkv_compress_step_noalloc(const rkv_config *cfg, int32_t n
     if (need == 0)   // invalid config: let the step report exactly what is wrong
         return rkv_compress_step(cfg, n_layers, batch, cap, k_layers, v_layers, q_layers, budgets,
                                  lambdas, cur_len, opts, nullptr, 0, stream);
+    // MAX redundancy keeps r of every unit in the workspace: far beyond the scratch
+    if (cfg->redundancy_mode == RKV_RED_MAX) return RKV_ERR_UNSUPPORTED;
     if (batch > RKV_NOALLOC_MAX_BATCH || need > kScratchBytes) return RKV_ERR_UNSUPPORTED;
     void *scratch = nullptr;
     const rkv_status st = scratch_address(&scratch);
     if (st != RKV_OK) return st;
     return rkv_compress_step(cfg, n_layers, batch, cap, k_layers, v_layers, q_layers, budgets,
                              lambdas, cur_len, opts, scratch, kScratchBytes, stream);
+}
+
+extern "C" rkv_status rkv_noalloc_status(rkv_stream_t stream) {
+    void *scratch = nullptr;
+    const rkv_status st = scratch_address(&scratch);
+    if (st != RKV_OK) return st;
+    // the status word sits at the start of the scratch, as in a workspace
+    return rkv_workspace_status(scratch, stream);
 }

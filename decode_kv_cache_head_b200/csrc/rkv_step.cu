@@ -63,7 +63,8 @@ __global__ void __launch_bounds__(256) rkv_plan_kernel(int batch, const int32_t 
                                                        int32_t budget_cfg, int32_t buffer, int32_t window,
                                                        int32_t cap, int32_t *__restrict__ cur_len,
                                                        int32_t *__restrict__ n_eff,
-                                                       uint32_t *__restrict__ status, int update) {
+                                                       uint32_t *__restrict__ status, int update,
+                                                       RaggedLayout rg) {
     // the kernel that follows may be scheduled now; it waits for this one to finish
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     for (int i = threadIdx.x; i < static_cast<int>(kStatusBytes / 4); i += blockDim.x) status[i] = 0u;
@@ -73,7 +74,16 @@ __global__ void __launch_bounds__(256) rkv_plan_kernel(int batch, const int32_t 
         const int32_t n = cur_len[b];
         // Compression is active only when budget and buffer are both positive.
         bool due = bud > 0 && buffer > 0 && n >= bud + buffer;
-        if (due && (bud < window || n > cap)) {
+        // the sequence's capacity: its own block of a ragged pool, else the uniform one
+        int32_t c = cap;
+        bool bad_block = false;
+        if (due && rg.seq_row) {
+            c = rg.seq_cap[b];
+            const int64_t r0 = rg.seq_row[b];
+            bad_block = c < 2 || c > cap || r0 < 0 ||
+                        r0 + static_cast<int64_t>(rg.n_kv) * c > rg.pool_rows;
+        }
+        if (due && (bud < window || n > c || bad_block)) {
             record_flag(status, kDevFlagBadSeq);
             due = false;
         }
@@ -84,9 +94,10 @@ __global__ void __launch_bounds__(256) rkv_plan_kernel(int batch, const int32_t 
 
 cudaError_t launch_plan(int batch, const int32_t *budgets, int32_t budget_cfg, int32_t buffer,
                         int32_t window, int32_t cap, int32_t *cur_len, int32_t *n_eff,
-                        uint32_t *status, cudaStream_t stream, bool update) {
+                        uint32_t *status, cudaStream_t stream, bool update,
+                        const RaggedLayout &rg) {
     rkv_plan_kernel<<<1, 256, 0, stream>>>(batch, budgets, budget_cfg, buffer, window, cap,
-                                           cur_len, n_eff, status, update ? 1 : 0);
+                                           cur_len, n_eff, status, update ? 1 : 0, rg);
     return cudaGetLastError();
 }
 

@@ -139,7 +139,7 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
     const bool red_max = p.red_mode == RKV_RED_MAX;
     const bool pool_max = p.gqa_pool == RKV_GQA_MAX;
     const int T = (N + kTileRows - 1) / kTileRows;
-    const int64_t krow0 = (static_cast<int64_t>(b) * p.n_kv + h) * p.cap;
+    const int64_t krow0 = unit_first_row(p.seq_row, p.seq_cap, b, h, p.n_kv, p.cap);
     // paged caches: row r of this unit is row prow(r) of the layer's page pool
     const bool paged = p.block_table != nullptr;
     const int psh = paged ? 31 - __clz(p.page_rows) : 7;   // page_rows is a power of two
@@ -149,10 +149,8 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
     const UnitLayout L = make_unit_layout(p.nmax, NQP);
     uint8_t *sStage = base + L.stage;
     uint8_t *sB = base + L.b;
-    float *sInv = reinterpret_cast<float *>(base + L.inv);
-    float *sSelf = reinterpret_cast<float *>(base + L.self);
-    float *sIa = reinterpret_cast<float *>(base + L.ia);
-    float *sIb = reinterpret_cast<float *>(base + L.ib);
+    float *sSS = reinterpret_cast<float *>(base + L.ss);       // ||k_i||^2 (pass 1 -> pass 2)
+    float *sIhat = reinterpret_cast<float *>(base + L.ihat);   // Ihat (max or sum over heads)
     float *sR = reinterpret_cast<float *>(base + L.r);
     float *sScr = reinterpret_cast<float *>(base + L.scr);
     float *sColM = reinterpret_cast<float *>(base + L.colm);
@@ -338,10 +336,7 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
                         *reinterpret_cast<uint16_t *>(bb + sw128_offset(0, c) + e) = hi;
                         *reinterpret_cast<uint16_t *>(bb + sw128_offset(1, c) + e) = mid;
                         *reinterpret_cast<uint16_t *>(bb + sw128_offset(2, c) + e) = lo;
-                        if (in) {
-                            sInv[i] = inv;
-                            sSelf[i] = inv * inv * ss;
-                        }
+                        if (in) sSS[i] = ss;
                     }
                 }
                 if (tt == T - 1 && N < T * kTileRows) {
@@ -432,6 +427,9 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
                 sColM[q] = -m;   // negated: pass 2 adds it
                 sColF[q] = sm > 0.f ? 1.0f / sm : 0.f;
             }
+            // Ihat starts at zero: both warpgroups merge their heads into it in pass 2
+            // (the S UMMA that read these bytes is complete)
+            for (int j = tid; j < M; j += NT) sIhat[j] = 0.f;
             fence_proxy_async_smem();
             tc_fence_before();
             __syncthreads();
@@ -591,16 +589,24 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
                         tmem_wait_ld();
                         reg_tie4(d);
                         const float dot = (__uint_as_float(d[0]) + __uint_as_float(d[1])) + __uint_as_float(d[2]);
-                        if (cand) r = (sInv[i] * dot - sSelf[i]) * inv_nm1;
+                        if (cand) {
+                            // the inverse norm and khat_i . khat_i exactly as pass 1 had them
+                            const float ss = sSS[i];
+                            const float inv = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
+                            const float self = __fmul_rn(__fmul_rn(inv, inv), ss);
+                            r = (inv * dot - self) * inv_nm1;
+                        }
                     }
                 }
                 if (cand) {
-                    if (wg == 0) {
-                        sIa[i] = pool;
-                    } else {
-                        sIb[i] = pool;
-                        sR[i] = r;
-                    }
+                    // pool >= 0, so its bits order like the value: the max of the two
+                    // warpgroups' heads is an integer max; the mean pool adds two terms
+                    // (a + b == b + a, whichever lands first)
+                    if (pool_max)
+                        atomicMax(reinterpret_cast<int *>(&sIhat[i]), __float_as_int(pool));
+                    else
+                        atomicAdd(&sIhat[i], pool);
+                    if (wg == 1) sR[i] = r;
                 }
             }
         }
@@ -659,10 +665,7 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
     const float invG = 1.0f / static_cast<float>(G);
     const bool scores_only = p.z_heads != nullptr;
     post_scores_any<NT, 1>(
-        [&](int j) {
-            const float a = sIa[j], c = sIb[j];
-            return make_float2(pool_max ? fmaxf(a, c) : (a + c) * invG, sR[j]);
-        },
+        [&](int j) { return make_float2(pool_max ? sIhat[j] : sIhat[j] * invG, sR[j]); },
         sKeys, sHist, sRed, M, kk, lam, !scores_only, inv_sumI, rmax_g, inv_rsum, Tk, n_gt);
 
     if (scores_only) {
@@ -670,8 +673,7 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
         // heads (and ranks) are summed and one set is selected afterwards
         float *zo = p.z_heads + unit_g * p.cap;
         for (int row = tid; row < M; row += NT) {
-            const float a = sIa[row], c = sIb[row];
-            const float I = (pool_max ? fmaxf(a, c) : (a + c) * invG) * inv_sumI;
+            const float I = (pool_max ? sIhat[row] : sIhat[row] * invG) * inv_sumI;
             const float Rv = ex2_approx((sR[row] - rmax_g) * kLog2e) * inv_rsum;
             zo[row] = joint_score(lam, I, Rv);
         }
@@ -738,8 +740,7 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
             if (p.kept_out && d >= 0) p.kept_out[unit_g * p.cap + d] = row;
             if (p.scores_out && row < M) {
                 float *so = p.scores_out + unit_g * 4 * p.cap;
-                const float a = sIa[row], c = sIb[row];
-                const float I = (pool_max ? fmaxf(a, c) : (a + c) * invG) * inv_sumI;
+                const float I = (pool_max ? sIhat[row] : sIhat[row] * invG) * inv_sumI;
                 const float Rv = ex2_approx((sR[row] - rmax_g) * kLog2e) * inv_rsum;
                 so[row] = I;
                 so[p.cap + row] = sR[row];

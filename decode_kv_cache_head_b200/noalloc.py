@@ -22,6 +22,17 @@ _f.argtypes = [ctypes.POINTER(rkv_config), ctypes.c_int32, ctypes.c_int32, ctype
                ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(rkv_step_options),
                ctypes.c_void_p]
 
+_fs = _lib.rkv_noalloc_status
+_fs.restype = ctypes.c_int
+_fs.argtypes = [ctypes.c_void_p]
+
+
+def rkv_noalloc_status(stream=None) -> int:
+    """Device-side status of the latest allocation-free call on the current
+    device (synchronises the stream): 0, or the RKV_STATUS_DEVICE_TIMEOUT /
+    RKV_ERR_DEVICE_INPUT code."""
+    return int(_fs(_stream(stream)))
+
 
 def rkv_compress_step_noalloc(cfg, k_layers, v_layers, q_layers, cur_len, budgets=None,
                               lambdas=None, kept_out=None, scores_out=None, cluster_size=0,

@@ -266,18 +266,24 @@ RKV_API rkv_status rkv_append_kv(const rkv_config *cfg, int32_t n_layers, int32_
  * Instead of a workspace the call uses a fixed scratch array of
  * RKV_NOALLOC_SCRATCH_BYTES in the library's own device memory.  It holds a
  * status header and one int32 per sequence, so batch is limited to
- * RKV_NOALLOC_MAX_BATCH; a larger batch returns RKV_ERR_UNSUPPORTED, and so
- * does any config whose workspace would not fit.  Every GPU on which the
- * library is used keeps this array until the process exits.
+ * RKV_NOALLOC_MAX_BATCH; a larger batch returns RKV_ERR_UNSUPPORTED.  Only
+ * MEAN redundancy fits: MAX keeps r of every (layer, sequence, head) in the
+ * workspace, so redundancy_mode RKV_RED_MAX returns RKV_ERR_UNSUPPORTED.
+ * Every GPU on which the library is used keeps this array until the process
+ * exits.
  *
- * The first call on each device looks up the array's device address with
- * cudaGetSymbolAddress (that device must be current), so make that first call
- * before any stream capture.  The call allocates nothing (no cudaMalloc, no
- * cudaFree, no allocating library routine).  All calls share the one array
+ * The first call on each device (or of rkv_noalloc_status) looks up the
+ * array's device address with cudaGetSymbolAddress, with that device current,
+ * and caches it for the life of the process; make that first call before any
+ * stream capture, and do not use these two calls after cudaDeviceReset (the
+ * cached address would be stale).  The call allocates nothing (no cudaMalloc,
+ * no cudaFree, no allocating library routine).  All calls share the one array
  * and it keeps whatever the last call left in it; the call resets what must
  * start at zero itself.  Calls whose work overlaps on the GPU (two streams,
  * two host threads) race on the array: serialise them.  Other arguments,
- * results and statuses are those of rkv_compress_step.
+ * results and host-side statuses are those of rkv_compress_step; faults found
+ * on the device land in the array's status word, which rkv_noalloc_status
+ * reads back.
  */
 #define RKV_NOALLOC_MAX_BATCH 4096
 #define RKV_NOALLOC_SCRATCH_BYTES (256 + 4 * RKV_NOALLOC_MAX_BATCH)
@@ -289,6 +295,16 @@ RKV_API rkv_status rkv_compress_step_noalloc(const rkv_config *cfg, int32_t n_la
                                              const int32_t *budgets, const float *lambdas,
                                              int32_t *cur_len, const rkv_step_options *opts,
                                              rkv_stream_t stream);
+
+/*
+ * The device-side status of the latest rkv_compress_step_noalloc call on the
+ * current device, as rkv_workspace_status reports it for a workspace:
+ * synchronises `stream`, then returns RKV_OK, RKV_STATUS_DEVICE_TIMEOUT or
+ * RKV_ERR_DEVICE_INPUT (for instance a sequence whose per-sequence budget is
+ * below the window, which the step skipped).  No counterpart in the R-KV
+ * pages either.
+ */
+RKV_API rkv_status rkv_noalloc_status(rkv_stream_t stream);
 
 /*
  * Shared selection: every KV head of a (sequence, layer) keeps the same
@@ -362,8 +378,8 @@ typedef struct {
  * device pointers to the page pools; q_layers, budgets, lambdas, cur_len,
  * opts (kept_out / scores_out / events; cluster_size 0 or 1) and the
  * workspace (rkv_workspace_size with cap = max_blocks * page_rows) as in
- * rkv_compress_step.  MEAN redundancy only (MAX: RKV_ERR_UNSUPPORTED); pages
- * of different sequences must be distinct.  Caches up to 512 pages per
+ * rkv_compress_step (MAX redundancy reads its similarity tiles through the
+ * block table too); pages of different sequences must be distinct.  Caches up to 512 pages per
  * sequence and one CTA's rows (rkv_query_step_shape cluster_size 1).
  */
 RKV_API rkv_status rkv_compress_step_paged(const rkv_config *cfg, int32_t n_layers, int32_t batch,
@@ -373,6 +389,49 @@ RKV_API rkv_status rkv_compress_step_paged(const rkv_config *cfg, int32_t n_laye
                                            const int32_t *budgets, const float *lambdas,
                                            int32_t *cur_len, const rkv_step_options *opts,
                                            void *workspace, size_t ws_bytes, rkv_stream_t stream);
+
+/*
+ * Caches with per-sequence capacities.  Each layer's keys live in one pool of
+ * pool_rows rows of 128 bf16 (256 bytes), and so do its values (a second pool
+ * of the same geometry).  Sequence b owns the block of n_kv_heads *
+ * seq_cap[b] rows starting at row seq_row[b]: row i of KV head h of sequence
+ * b is pool row seq_row[b] + h * seq_cap[b] + i.  This is the
+ * [batch, kv_heads, len, head_dim] layout of rkv_compress_step with the batch
+ * split into blocks of their own size, so a sequence with a small budget
+ * holds budget + buffer rows instead of the largest sequence's (the pages'
+ * fixed buffer per sequence: atlas.scime.ai summary, "Approach"; the 90%
+ * memory saving: sourcepulse summary, "Highlighted Details").  Blocks of
+ * different sequences must not overlap; gaps between them are allowed.
+ */
+typedef struct {
+    const int64_t *seq_row;   /* device [batch]: first pool row of sequence b (8-byte aligned) */
+    const int32_t *seq_cap;   /* device [batch]: rows per KV head of sequence b's block */
+    int64_t pool_rows;        /* rows in each layer's pool (<= INT32_MAX) */
+    int32_t max_cap;          /* an upper bound of every seq_cap[b]: sizes shared memory, the
+                                 workspace (rkv_workspace_size with cap = max_cap) and the
+                                 row stride of kept_out / scores_out */
+} rkv_ragged_kv;
+
+/*
+ * The step on caches with per-sequence capacities (layout above): for every
+ * due sequence (cur_len[b] >= budget_b + buffer), for every layer and KV head,
+ * steps 1-5 over its N = cur_len[b] rows, then cur_len[b] = budget_b, exactly
+ * as rkv_compress_step.  k_pools / v_pools: host arrays [n_layers] of device
+ * pointers to the pools; q_layers, budgets, lambdas, cur_len as in
+ * rkv_compress_step; opts: kept_out / scores_out as there with cap = max_cap,
+ * events, cluster_size 0 or 1 (one CTA per unit; clusters:
+ * RKV_ERR_UNSUPPORTED).  A due sequence whose block does not fit the pool
+ * (seq_row[b] < 0, seq_row[b] + n_kv_heads * seq_cap[b] > pool_rows,
+ * seq_cap[b] > max_cap) or whose cur_len exceeds seq_cap[b] is skipped and
+ * reported through the workspace status (RKV_ERR_DEVICE_INPUT).
+ */
+RKV_API rkv_status rkv_compress_step_ragged(const rkv_config *cfg, int32_t n_layers, int32_t batch,
+                                            const rkv_ragged_kv *rg, rkv_bf16 *const *k_pools,
+                                            rkv_bf16 *const *v_pools,
+                                            const rkv_bf16 *const *q_layers,
+                                            const int32_t *budgets, const float *lambdas,
+                                            int32_t *cur_len, const rkv_step_options *opts,
+                                            void *workspace, size_t ws_bytes, rkv_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -43,6 +43,8 @@ __all__ = [
     "dup_runs",
     "make_inputs",
     "bf16_bits",
+    "pack_ragged",
+    "unpack_ragged",
 ]
 
 
@@ -236,6 +238,27 @@ def make_inputs(w: Workload, device: str = "cpu", layers: Optional[Sequence[int]
             Q[li, bi] = torch.randn((Hq, win, D), generator=g, device=device,
                                     dtype=torch.float32).to(torch.bfloat16)
     return {"K": K, "V": V, "Q": Q, "cur_len": cur_len.to(device)}
+
+
+def pack_ragged(X: torch.Tensor, caps: Sequence[int]) -> torch.Tensor:
+    """[n_layers, batch, H, cap, D] -> [n_layers, sum_b H * caps[b], D]: every
+    sequence's first caps[b] rows of each head, the sequences' blocks packed back
+    to back in batch order (the per-sequence-capacity pool layout)."""
+    L, B, H, _, D = X.shape
+    return torch.cat([X[:, b, :, :int(caps[b])].reshape(L, H * int(caps[b]), D)
+                      for b in range(B)], dim=1).contiguous()
+
+
+def unpack_ragged(P: torch.Tensor, caps: Sequence[int], n_kv: int, cap: int) -> torch.Tensor:
+    """Inverse of pack_ragged: [n_layers, rows, D] -> [n_layers, batch, H, cap, D]
+    (rows past a sequence's capacity are zero)."""
+    L, _, D = P.shape
+    out = torch.zeros((L, len(caps), n_kv, cap, D), dtype=P.dtype, device=P.device)
+    r = 0
+    for b, c in enumerate(caps):
+        out[:, b, :, :int(c)] = P[:, r:r + n_kv * int(c)].reshape(L, n_kv, int(c), D)
+        r += n_kv * int(c)
+    return out
 
 
 def bf16_bits(t: torch.Tensor) -> np.ndarray:

@@ -168,3 +168,51 @@ def test_shared_selection_host_validation():
     big = rkv.rkv_workspace_size_shared(c, 2, 1, 9000)
     assert L.rkv_select_compact_shared(cfgp, 2, 1, 9000, k, v, None, cur, z, None, ws, big,
                                        None) == -6
+
+
+def test_ragged_step_host_validation():
+    L = rkv._lib
+    c = rkv.make_config()
+    cfgp = ctypes.byref(c)
+    arr = ctypes.c_void_p * 2
+    k = arr(A, A + (1 << 34))
+    v = arr(A + (1 << 36), A + (1 << 36) + (1 << 34))
+    q = arr(A + (1 << 37), A + (1 << 37) + (1 << 20))
+    cur, ws = A + 7 * 4096, A + (1 << 38)
+    need = rkv.rkv_workspace_size(c, 2, 4, 2176)
+
+    def call(rg=None, cfg=cfgp, kk=k, vv=v, ws_=ws, ws_bytes=need, opts=None):
+        if rg is None:
+            rg = rkv.rkv_ragged_kv(A + (1 << 39), A + (1 << 39) + 4096, 4 * 8 * 2176, 2176)
+        return L.rkv_compress_step_ragged(cfg, 2, 4, ctypes.byref(rg), kk, vv, q, None, None,
+                                          cur, opts, ws_, ws_bytes, None)
+
+    assert L.rkv_compress_step_ragged(cfgp, 2, 4, None, k, v, q, None, None, cur, None, ws,
+                                      need, None) == -1
+    assert call(rkv.rkv_ragged_kv(None, A, 100, 2176)) == -1                 # no seq_row
+    assert call(rkv.rkv_ragged_kv(A + 4, A, 100000, 2176)) == -3             # seq_row not 8-aligned
+    assert call(rkv.rkv_ragged_kv(A, A, 1 << 31, 2176)) == -6                # rows past int32
+    assert call(rkv.rkv_ragged_kv(A, A, 100000, 1)) == -2                    # max_cap < 2
+    assert call(rkv.rkv_ragged_kv(A, A, 100000, 1000)) == -2                 # budget >= max_cap
+    assert call(rkv.rkv_ragged_kv(A, A, 100000, 9000)) == -6                 # one CTA cannot hold it
+    assert call(cfg=ctypes.byref(rkv.make_config(buffer=0))) == 1            # disabled
+    assert call(ws_=None) == -5
+    assert call(ws_bytes=need - 256) == -5
+    assert call(ws_=ws + 16) == -3
+    assert call(vv=arr(A + 4096, A + (1 << 36))) == -4                       # K pool overlaps V pool
+    opts = rkv.rkv_step_options(None, None, None, None, 8)
+    assert call(opts=ctypes.byref(opts)) == -6                               # clusters unsupported
+
+
+def test_ragged_layout_helpers():
+    import torch
+    from rkv_synth import pack_ragged, unpack_ragged
+    rows, total = rkv.ragged_rows([10, 3, 7], 2)
+    assert rows == [0, 20, 26] and total == 40
+    X = torch.arange(2 * 3 * 2 * 10 * 4, dtype=torch.float32).reshape(2, 3, 2, 10, 4)
+    P = pack_ragged(X, [10, 3, 7])
+    assert P.shape == (2, 40, 4)
+    assert torch.equal(P[:, 20:23], X[:, 1, 0, :3]) and torch.equal(P[:, 23:26], X[:, 1, 1, :3])
+    Y = unpack_ragged(P, [10, 3, 7], 2, 10)
+    assert torch.equal(Y[:, 0], X[:, 0])
+    assert torch.equal(Y[:, 2, :, :7], X[:, 2, :, :7]) and not Y[:, 2, :, 7:].any()
