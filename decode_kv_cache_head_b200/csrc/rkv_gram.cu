@@ -307,15 +307,23 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
         // norms: two threads per row, 64 columns each
         const int nrow = (lane & 7) + 8 * (lane >> 4), nhalf = (lane >> 3) & 1;
         const int row_t = 16 * warp + nrow;
+        // A wait that runs out makes `ok` false for the whole warp (so the warp's
+        // .sync.aligned TMEM loads never diverge); a failed warp skips the work but keeps
+        // every named barrier of the schedule, so the other epilogue warps never wait
+        // on it at a barrier without a time limit.
+        auto wait_all = [&](uint64_t *bar, uint32_t parity) {
+            const bool w = ok ? mbar_wait(bar, parity) : false;
+            ok = __all_sync(kFull, w) != 0;
+        };
         uint32_t na = 0, np = 0;
-        for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x) {
+        for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
             const UnitInfo u = unit_info(p, unit);
             if (u.N <= 0 || u.M <= 0) continue;
-            for (int I = u.T - 1; I >= 0 && ok; --I) {
+            for (int I = u.T - 1; I >= 0; --I) {
                 const uint32_t a = na & 1u;
-                if (!mbar_wait(&afull[a], (na >> 1) & 1u)) { ok = false; break; }
+                wait_all(&afull[a], (na >> 1) & 1u);
                 ++na;
-                {
+                if (ok) {
                     // 1 / max(||k_i||, 1e-12) of the row tile's rows (0 past N)
                     const uint8_t *hp = sA + a * kTileBytes + nhalf * kHalfBytes + row_t * 128;
                     float2 ss2 = make_float2(0.f, 0.f);
@@ -340,10 +348,11 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
 #pragma unroll
                 for (int r = 0; r < 4; ++r) inv_r[r] = sInv[I * 128 + row_of(r)];
                 float rrun = -INFINITY;
-                for (int J = I; J < u.T && ok; ++J) {
+                for (int J = I; J < u.T; ++J) {
                     const uint32_t t = np % kAcc;
-                    if (!mbar_wait(&tfull[t], (np / kAcc) & 1u)) { ok = false; break; }
+                    wait_all(&tfull[t], (np / kAcc) & 1u);
                     ++np;
+                    if (!ok) continue;
                     tc_fence_after();
                     uint32_t v0[32], v1[32];   // slab 0 (rows 0, 1), slab 1 (rows 2, 3)
                     const uint32_t tcol = tmem_base + t * 128u + 64u * ch;
@@ -441,10 +450,8 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
                         atomicMax(&sKey[cj + 1], ord_key(cm[1]));
                     }
                 }
-                if (!ok) break;
-                atomicMax(&sKey[I * 128 + myrow], ord_key(rrun));
+                if (ok) atomicMax(&sKey[I * 128 + myrow], ord_key(rrun));
             }
-            if (!ok) break;
             // every key of the unit is final: r = inv_i * u_i; then clear for the next unit
             epi_sync();
             float *ro = p.r_out + u.unit_g * p.cap;
