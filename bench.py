@@ -504,6 +504,8 @@ def run_rkv(args, w, red_mode):
         rdist.barrier(dev)
         torch.cuda.synchronize()
         t_start.record(stream)
+        # an NVTX range around the timed steps (profilers can restrict a capture to it)
+        torch.cuda.nvtx.range_push("timed_steps")
         for i in range(n_steps):
             if not fits:
                 restore(reps[0])
@@ -512,6 +514,7 @@ def run_rkv(args, w, red_mode):
                  sim_events=ev_sim[i] if (kernel_events and ev_sim) else None, **kw)
             if not fits:
                 st[i][1].record(stream)
+        torch.cuda.nvtx.range_pop()
         t_stop.record(stream)
         torch.cuda.synchronize()
         rdist.barrier(dev)
@@ -886,8 +889,10 @@ def run_mode(args, w, red_mode):
     rdist.barrier(dev)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
+    torch.cuda.nvtx.range_push("timed_steps")
     for i in range(args.steps):
         call(reps[args.warmup + i])
+    torch.cuda.nvtx.range_pop()
     b.record(stream)
     torch.cuda.synchronize()
     rdist.barrier(dev)

@@ -17,7 +17,8 @@ import torch
 __all__ = [
     "RKV_OK", "RKV_STATUS_DISABLED", "RKV_RED_MEAN", "RKV_RED_MAX", "RKV_GQA_MAX", "RKV_GQA_MEAN",
     "RkvError", "rkv_config", "rkv_step_options", "make_config", "library_path",
-    "rkv_status_string", "rkv_version", "rkv_workspace_size", "rkv_workspace_status",
+    "rkv_status_string", "rkv_version", "rkv_last_cuda_error", "rkv_workspace_size",
+    "rkv_workspace_status",
     "rkv_query_step_shape",
     "rkv_score_importance", "rkv_score_redundancy", "rkv_select_topk", "rkv_compact_kv",
     "rkv_compress_step", "rkv_append_kv",
@@ -95,6 +96,7 @@ def _load() -> ctypes.CDLL:
     sig = {
         "rkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "rkv_version": (I32, []),
+        "rkv_last_cuda_error": (I32, []),
         "rkv_workspace_size": (SZ, [CFG, I32, I32, I32]),
         "rkv_workspace_status": (ctypes.c_int, [P, P]),
         "rkv_query_step_shape": (ctypes.c_int, [CFG, I64, I32, ctypes.POINTER(I32),
@@ -135,7 +137,11 @@ _lib = _load()
 class RkvError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {rkv_status_string(status)} ({status})")
+        detail = ""
+        if status == -7:   # RKV_ERR_CUDA: name the CUDA error behind it
+            self.cuda_error = int(_lib.rkv_last_cuda_error())
+            detail = f"; cudaError {self.cuda_error}"
+        super().__init__(f"{where}: {rkv_status_string(status)} ({status}{detail})")
 
 
 def rkv_status_string(status: int) -> str:
@@ -144,6 +150,10 @@ def rkv_status_string(status: int) -> str:
 
 def rkv_version() -> int:
     return int(_lib.rkv_version())
+
+
+def rkv_last_cuda_error() -> int:
+    return int(_lib.rkv_last_cuda_error())
 
 
 def make_config(budget=1024, buffer=128, window=8, head_dim=128, n_kv_heads=8, n_q_heads=32,

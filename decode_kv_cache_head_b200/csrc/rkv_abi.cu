@@ -306,7 +306,14 @@ void fill_common(StepParams &p, const rkv_config *cfg, const Shape &s, int batch
     p.gqa_pool = cfg->gqa_pool;
 }
 
-rkv_status cuda_status(cudaError_t e) { return e == cudaSuccess ? RKV_OK : RKV_ERR_CUDA; }
+// The CUDA error behind the calling thread's latest RKV_ERR_CUDA.
+thread_local int32_t g_last_cuda_error = 0;
+
+rkv_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return RKV_OK;
+    g_last_cuda_error = static_cast<int32_t>(e);
+    return RKV_ERR_CUDA;
+}
 
 // Per-head entry points share this: one (sequence, layer), all KV heads.
 rkv_status run_per_head_scores(const rkv_config *cfg, const rkv_bf16 *q, const rkv_bf16 *k,
@@ -389,6 +396,8 @@ const char *rkv_status_string(rkv_status s) {
 
 int32_t rkv_version(void) { return kVersion; }
 
+int32_t rkv_last_cuda_error(void) { return g_last_cuda_error; }
+
 size_t rkv_workspace_size(const rkv_config *cfg, int32_t n_layers, int32_t batch, int32_t cap) {
     if (check_cfg(cfg) != RKV_OK || n_layers < 1 || batch < 1 || cap < 2) return 0;
     return ws_bytes_for(cfg, n_layers, batch, cap);
@@ -421,7 +430,7 @@ rkv_status rkv_workspace_status(const void *workspace, rkv_stream_t stream) {
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
-    if (e != cudaSuccess) return RKV_ERR_CUDA;
+    if (e != cudaSuccess) return cuda_status(e);
     if (word & kDevFlagTimeout) return RKV_STATUS_DEVICE_TIMEOUT;
     if (word) return RKV_ERR_DEVICE_INPUT;
     return RKV_OK;

@@ -50,13 +50,12 @@ __global__ void rkv_bump_len_kernel(int batch, int n_new, int cap, int32_t *cur_
 cudaError_t launch_append(const AppendParams &p, int n_layers, cudaStream_t stream) {
     const int nchunk = static_cast<int>((static_cast<int64_t>(p.n_new) * 16 + 255) / 256);
     const unsigned blocks = static_cast<unsigned>(n_layers * p.batch * p.n_kv) * nchunk;
-    rkv_append_kernel<<<blocks, 256, 0, stream>>>(p, nchunk);
-    return cudaGetLastError();
+    return launch_kernel(rkv_append_kernel, dim3(blocks), dim3(256), 0, stream, p, nchunk);
 }
 
 cudaError_t launch_bump(int batch, int n_new, int cap, int32_t *cur_len, cudaStream_t stream) {
-    rkv_bump_len_kernel<<<(batch + 127) / 128, 128, 0, stream>>>(batch, n_new, cap, cur_len);
-    return cudaGetLastError();
+    return launch_kernel(rkv_bump_len_kernel, dim3((batch + 127) / 128), dim3(128), 0, stream, batch,
+                         n_new, cap, cur_len);
 }
 
 }  // namespace rkv

@@ -117,9 +117,8 @@ cudaError_t launch_compact(const uint16_t *k_src, const uint16_t *v_src, const i
     if (!in_place) {
         const int64_t items = static_cast<int64_t>(budget) * 16;
         dim3 grid(static_cast<unsigned>((items + 255) / 256), static_cast<unsigned>(n_kv));
-        rkv_gather_kernel<<<grid, 256, 0, stream>>>(k_src, v_src, kept, k_dst, v_dst, head_stride,
-                                                    budget, n_tokens, status);
-        return cudaGetLastError();
+        return launch_kernel(rkv_gather_kernel, grid, dim3(256), 0, stream, k_src, v_src, kept, k_dst,
+                             v_dst, head_stride, budget, n_tokens, status);
     }
     const int rb = (budget + cs - 1) / cs;
     const size_t smem = static_cast<size_t>(rb) * 512u + 128u;

@@ -8,27 +8,30 @@
 //
 // With a_ij = k_i . k_j (bf16 products, fp32 accumulate on tcgen05) and
 // inv_i = 1 / max(||k_i||, 1e-12):  r_i = inv_i * u_i,  u_i = max_{j != i} a_ij inv_j.
-// The Gram matrix is symmetric, so only the tile pairs (I, J >= I) of 128 x 128
-// are computed: the accumulator of pair (I, J) gives u of the rows of tile I
-// (row maxima of a_ij inv_j) and u of the rows of tile J (column maxima of
-// a_ij inv_i).  The N x N matrix never leaves the chip, and the inverse norms
-// are computed here from the tiles already in shared memory: K is read once
-// from HBM (the tiles a unit reuses come from L2).
+// The Gram matrix is symmetric, so only the tile pairs (I <= J) of 128 x 128 are
+// computed: the accumulator of pair (I, J) gives u of the rows of tile I (row
+// maxima of a_ij inv_j) and of the rows of tile J (column maxima of a_ij inv_i).
+// The N x N matrix never leaves the chip, and the inverse norms are computed here
+// from the tiles already in shared memory: K is read once from HBM (the tiles a
+// unit reuses come from L2).
 //
-// Persistent CTAs (one per SM) walk the units; per unit the row tiles go from
-// last to first, so that when row I runs, the inverse norms of every tile
-// J >= I are known (tile J was the A operand of an earlier row).  Warp roles
-// (320 threads, one CTA per SM):
-//   warps 0-7  epilogue: inverse norms of each row tile; per pair, the
+// Persistent CTAs (one per SM) walk the units.  Per unit the column tiles J go
+// from first to last; tile J stays resident while the row tiles I = J (the
+// diagonal, from the resident tile itself), 0, 1, ..., J-1 stream past it, so
+// every row tile's inverse norms are known when it arrives, and the column
+// maxima of tile J build up in registers over the whole column and cross lanes
+// once.  Warp roles (320 threads, one CTA per SM):
+//   warps 0-7  epilogue: inverse norms of each column tile; per pair, the
 //              accumulator read with tcgen05.ld 16x256b (each thread holds 4
-//              rows x 16 columns), row and column maxima folded in registers,
-//              across 4 and 8 lanes by shuffles, then merged into per-row
-//              order-preserving keys in shared memory with atomicMax;
-//   warp 8     producer: TMA of the row tile (double-buffered A) and of the
-//              column tiles (three-stage B ring);
+//              rows x 16 columns); row maxima folded over the 16 columns and
+//              across the 4 lanes of a row group, merged into per-row
+//              order-preserving keys in shared memory with atomicMax; column
+//              maxima kept per thread until the column tile is done, then
+//              folded across the 8 lanes of a column group and merged the same way;
+//   warp 8     producer: TMA of the column tile (double-buffered) and of the
+//              row tiles (three-stage ring);
 //   warp 9     MMA issuer: 8 UMMAs (K = 128) per pair into one of four TMEM
-//              accumulators (128 columns each); the diagonal pair uses the A
-//              tile as both operands.
+//              accumulators (128 columns each).
 // Hand-offs are mbarriers; every wait is bounded and a timeout is recorded in
 // the status word (the CTA then drains what it issued and stops).
 #include <cuda.h>
@@ -46,8 +49,10 @@ namespace rkv {
 
 namespace {
 
-constexpr int kGramThreads = 320;
-constexpr int kEpiThreads = 256;
+constexpr int kEpiWarps = 16;                     // 4 TMEM quadrants x 4 column quarters
+constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int kGramThreads = kEpiThreads + 64;     // + producer warp + MMA warp
+constexpr int kProducerWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1;
 constexpr int kBStages = 3;
 constexpr int kAcc = 4;                            // TMEM accumulators of 128 columns
 constexpr uint32_t kTileBytes = 128u * 256u;       // 128 rows x 128 bf16
@@ -93,30 +98,19 @@ __device__ __forceinline__ float key_value(uint32_t k) {
     return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
-__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory"); }
 
-// 16 TMEM lanes x 64 fp32 columns (16x256b, 8 repetitions): thread t gets, for
+// 16 TMEM lanes x 32 fp32 columns (16x256b, 4 repetitions): thread t gets, for
 // repetition k, lane (t / 4) columns 8k + 2 (t % 4) + {0, 1} in r[4k], r[4k+1]
 // and lane (t / 4) + 8 the same columns in r[4k+2], r[4k+3].
-__device__ __forceinline__ void tmem_ld_16x256b_x8(uint32_t taddr, uint32_t (&r)[32]) {
+__device__ __forceinline__ void tmem_ld_16x256b_x4(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile(
-        "tcgen05.ld.sync.aligned.16x256b.x8.b32"
-        " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15,"
-        " %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32"
+        " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
           "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-          "=r"(r[31])
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
-}
-
-__device__ __forceinline__ void reg_tie32(uint32_t (&r)[32]) {
-#pragma unroll
-    for (int i = 0; i < 32; i += 8)
-        asm volatile("" : "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]),
-                     "+r"(r[i + 4]), "+r"(r[i + 5]), "+r"(r[i + 6]), "+r"(r[i + 7])::"memory");
 }
 
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
@@ -181,7 +175,7 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
         }
         for (int t = 0; t < kAcc; ++t) {
             mbar_init(&tfull[t], 1);
-            mbar_init(&tempty[t], 8);        // one arrival per epilogue warp
+            mbar_init(&tempty[t], kEpiWarps);   // one arrival per epilogue warp
         }
         fence_mbar_init();
     }
@@ -193,8 +187,9 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
     bool ok = true;
-    if (warp == 8) {
-        // ---------------- producer: per unit, row tiles T-1 .. 0 into A, column tiles into B
+    // buffers: sA = the resident column tiles (double-buffered), sB = the row-tile ring
+    if (warp == kProducerWarp) {
+        // ---------------- producer: per unit, column tiles 0 .. T-1; row tiles 0 .. J-1 of each
         uint32_t na = 0, nb = 0;
         for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x) {
             const UnitInfo u = unit_info(p, unit);
@@ -224,23 +219,23 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
                     }
                 }
             };
-            for (int I = u.T - 1; I >= 0 && ok; --I) {
+            for (int J = 0; J < u.T && ok; ++J) {
                 if (lane == 0) {
                     const uint32_t a = na & 1u;
                     if (na >= 2 && !mbar_wait(&aempty[a], ((na >> 1) - 1) & 1u)) ok = false;
                     if (ok) {
                         mbar_arrive_expect_tx(&afull[a], kTileBytes);
-                        load_tile(sA + a * kTileBytes, &afull[a], I);
+                        load_tile(sA + a * kTileBytes, &afull[a], J);
                     }
                     ++na;
-                    for (int J = I + 1; J < u.T && ok; ++J) {
+                    for (int I = 0; I < J && ok; ++I) {
                         const uint32_t s = nb % kBStages;
                         if (nb >= kBStages && !mbar_wait(&bempty[s], ((nb / kBStages) - 1) & 1u)) {
                             ok = false;
                             break;
                         }
                         mbar_arrive_expect_tx(&bfull[s], kTileBytes);
-                        load_tile(sB + s * kTileBytes, &bfull[s], J);
+                        load_tile(sB + s * kTileBytes, &bfull[s], I);
                         ++nb;
                     }
                 }
@@ -254,38 +249,40 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
             for (uint32_t i = nb >= kBStages ? nb - kBStages : 0; i < nb; ++i)
                 (void)mbar_wait(&bfull[i % kBStages], (i / kBStages) & 1u);
         }
-    } else if (warp == 9) {
-        // ---------------- MMA issuer
+    } else if (warp == kMmaWarp) {
+        // ---------------- MMA issuer: D[i][j] = K_I[i] . K_J[j]; A = the row tile, B = the column tile
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
             uint32_t na = 0, nb = 0, np = 0;
             for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x) {
                 const UnitInfo u = unit_info(p, unit);
                 if (u.N <= 0 || u.M <= 0) continue;
-                for (int I = u.T - 1; I >= 0 && ok; --I) {
+                for (int J = 0; J < u.T && ok; ++J) {
                     const uint32_t a = na & 1u;
                     if (!mbar_wait(&afull[a], (na >> 1) & 1u)) { ok = false; break; }
                     ++na;
-                    const uint32_t a_base = smem_u32(sA + a * kTileBytes);
-                    for (int J = I; J < u.T && ok; ++J) {
+                    const uint32_t col_base = smem_u32(sA + a * kTileBytes);
+                    // the diagonal pair first (both operands the resident tile), then I = 0 .. J-1
+                    for (int step = 0; step <= J && ok; ++step) {
+                        const bool diag = step == 0;
                         const uint32_t t = np % kAcc;
                         if (np >= kAcc && !mbar_wait(&tempty[t], ((np / kAcc) - 1) & 1u)) { ok = false; break; }
-                        uint32_t b_base = a_base, s = 0;
-                        if (J > I) {
+                        uint32_t row_base = col_base, s = 0;
+                        if (!diag) {
                             s = nb % kBStages;
                             if (!mbar_wait(&bfull[s], (nb / kBStages) & 1u)) { ok = false; break; }
-                            b_base = smem_u32(sB + s * kTileBytes);
+                            row_base = smem_u32(sB + s * kTileBytes);
                         }
                         tc_fence_after();
 #pragma unroll
                         for (int ks = 0; ks < 8; ++ks) {
                             const uint32_t off = (ks >> 2) * kHalfBytes + (ks & 3) * 32u;
-                            umma_bf16(tmem_base + t * 128u, desc_kmajor_sw128(a_base + off),
-                                      desc_kmajor_sw128(b_base + off), idesc, ks > 0 ? 1u : 0u);
+                            umma_bf16(tmem_base + t * 128u, desc_kmajor_sw128(row_base + off),
+                                      desc_kmajor_sw128(col_base + off), idesc, ks > 0 ? 1u : 0u);
                         }
                         umma_commit(&tfull[t]);
                         ++np;
-                        if (J > I) {
+                        if (!diag) {
                             umma_commit(&bempty[s]);
                             ++nb;
                         }
@@ -297,14 +294,15 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
             if (!ok && np > 0) (void)mbar_wait(&tfull[(np - 1) % kAcc], ((np - 1) / kAcc) & 1u);
         }
     } else {
-        // ---------------- epilogue warps 0-7: quadrant qd of TMEM lanes, column half ch
-        const int qd = warp & 3, ch = warp >> 2;
+        // ---------------- epilogue warps 0-15: quadrant qd of TMEM lanes, column quarter cq
+        const int qd = warp & 3, cq = warp >> 2;
         const int g = lane >> 2, q = lane & 3;
-        // this thread's 4 tile rows 32 qd + g + 8 r (r = 0, 1: the first 16-lane slab,
-        // r = 2, 3: the second) and the row it keeps after the 4-lane fold (r = q)
+        // this thread's 4 accumulator rows 32 qd + g + 8 r (r = 0, 1: the first 16-lane
+        // slab, r = 2, 3: the second) and the row it keeps after the 4-lane fold (r = q);
+        // its 8 columns 32 cq + 8 k + 2 q + e (k = 0..3, e = 0, 1)
         auto row_of = [&](int r) { return 32 * qd + g + 8 * r; };
         const int myrow = row_of(q);
-        // norms: two threads per row, 64 columns each
+        // norms (warps 0-7): two threads per row, 64 columns each
         const int nrow = (lane & 7) + 8 * (lane >> 4), nhalf = (lane >> 3) & 1;
         const int row_t = 16 * warp + nrow;
         // A wait that runs out makes `ok` false for the whole warp (so the warp's
@@ -319,12 +317,12 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
         for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
             const UnitInfo u = unit_info(p, unit);
             if (u.N <= 0 || u.M <= 0) continue;
-            for (int I = u.T - 1; I >= 0; --I) {
+            for (int J = 0; J < u.T; ++J) {
                 const uint32_t a = na & 1u;
                 wait_all(&afull[a], (na >> 1) & 1u);
                 ++na;
-                if (ok) {
-                    // 1 / max(||k_i||, 1e-12) of the row tile's rows (0 past N)
+                if (ok && warp < 8) {
+                    // 1 / max(||k_j||, 1e-12) of the column tile's rows (0 past N)
                     const uint8_t *hp = sA + a * kTileBytes + nhalf * kHalfBytes + row_t * 128;
                     float2 ss2 = make_float2(0.f, 0.f);
 #pragma unroll
@@ -339,28 +337,38 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
                     }
                     const float ssh = ss2.x + ss2.y;
                     const float ss = ssh + __shfl_xor_sync(kFull, ssh, 8);
-                    const int i = I * 128 + row_t;
+                    const int i = J * 128 + row_t;
                     if (nhalf == 0) sInv[i] = i < u.N ? 1.0f / fmaxf(sqrtf(ss), 1e-12f) : 0.f;
                 }
                 epi_sync();
-                if (tid == 0) mbar_arrive(&aempty[a]);   // the epilogue is done reading A
-                float inv_r[4];
+                if (tid == 0) mbar_arrive(&aempty[a]);   // the epilogue is done reading the tile
+                const int c0 = J * 128 + 32 * cq + 2 * q;    // unit row of this thread's column (k, e) = (0, 0)
+                float inv_c[8];
 #pragma unroll
-                for (int r = 0; r < 4; ++r) inv_r[r] = sInv[I * 128 + row_of(r)];
-                float rrun = -INFINITY;
-                for (int J = I; J < u.T; ++J) {
+                for (int k = 0; k < 4; ++k) {
+                    const float2 iv = *reinterpret_cast<const float2 *>(&sInv[c0 + 8 * k]);
+                    inv_c[2 * k] = iv.x;
+                    inv_c[2 * k + 1] = iv.y;
+                }
+                const bool tail = (J + 1) * 128 > u.N;       // columns past N in this tile
+                float colrun[8];                             // max over the rows seen of a_ij inv_i
+#pragma unroll
+                for (int c = 0; c < 8; ++c) colrun[c] = -INFINITY;
+                for (int step = 0; step <= J; ++step) {
+                    const bool diag = step == 0;
+                    const int I = diag ? J : step - 1;
                     const uint32_t t = np % kAcc;
                     wait_all(&tfull[t], (np / kAcc) & 1u);
                     ++np;
                     if (!ok) continue;
                     tc_fence_after();
-                    uint32_t v0[32], v1[32];   // slab 0 (rows 0, 1), slab 1 (rows 2, 3)
-                    const uint32_t tcol = tmem_base + t * 128u + 64u * ch;
-                    tmem_ld_16x256b_x8(tcol + ((32u * qd) << 16), v0);
-                    tmem_ld_16x256b_x8(tcol + ((32u * qd + 16u) << 16), v1);
+                    uint32_t v0[16], v1[16];   // slab 0 (rows 0, 1), slab 1 (rows 2, 3)
+                    const uint32_t tcol = tmem_base + t * 128u + 32u * cq;
+                    tmem_ld_16x256b_x4(tcol + ((32u * qd) << 16), v0);
+                    tmem_ld_16x256b_x4(tcol + ((32u * qd + 16u) << 16), v1);
                     tmem_wait_ld();
-                    reg_tie32(v0);
-                    reg_tie32(v1);
+                    reg_tie16(v0);
+                    reg_tie16(v1);
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&tempty[t]);   // the accumulator may be reused
@@ -369,22 +377,13 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
                         const uint32_t x = (r < 2) ? v0[4 * k + 2 * (r & 1) + e] : v1[4 * k + 2 * (r & 1) + e];
                         return __uint_as_float(x);
                     };
-                    const int c0 = J * 128 + 64 * ch + 2 * q;    // unit row of column (k = 0, e = 0)
-                    float inv_c[16];
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const float2 iv = *reinterpret_cast<const float2 *>(&sInv[c0 + 8 * k]);
-                        inv_c[2 * k] = iv.x;
-                        inv_c[2 * k + 1] = iv.y;
-                    }
-                    // ---- rows of tile I: max over this pair's columns of a_ij inv_j
-                    const bool diag = J == I, tail = (J + 1) * 128 > u.N;
+                    // ---- rows of tile I: max over this tile's columns of a_ij inv_j
                     float rm[4];
 #pragma unroll
                     for (int r = 0; r < 4; ++r) {
-                        float x[16];
+                        float x[8];
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) {
+                        for (int k = 0; k < 4; ++k) {
                             const float2 pr = __fmul2_rn(make_float2(av(r, k, 0), av(r, k, 1)),
                                                          make_float2(inv_c[2 * k], inv_c[2 * k + 1]));
                             x[2 * k] = pr.x;
@@ -393,20 +392,17 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
                         if (diag || tail) {
                             const int ri = I * 128 + row_of(r);
 #pragma unroll
-                            for (int k = 0; k < 8; ++k)
+                            for (int k = 0; k < 4; ++k)
 #pragma unroll
                                 for (int e = 0; e < 2; ++e) {
                                     const int cj = c0 + 8 * k + e;
                                     if (cj == ri || cj >= u.N) x[2 * k + e] = -INFINITY;
                                 }
                         }
-                        const float m0 = fmax3(x[0], x[1], x[2]), m1 = fmax3(x[3], x[4], x[5]);
-                        const float m2 = fmax3(x[6], x[7], x[8]), m3 = fmax3(x[9], x[10], x[11]);
-                        const float m4 = fmax3(x[12], x[13], x[14]);
-                        rm[r] = fmax3(fmax3(m0, m1, m2), fmax3(m3, m4, x[15]), -INFINITY);
+                        rm[r] = fmax3(fmax3(x[0], x[1], x[2]), fmax3(x[3], x[4], x[5]), fmaxf(x[6], x[7]));
                     }
-                    // fold across the 4 lanes of a row group: lane q keeps row q
                     {
+                        // fold across the 4 lanes of a row group: lane q keeps row q
                         const bool up = (q & 2) != 0;
                         const float s0 = up ? rm[0] : rm[2], s1 = up ? rm[1] : rm[3];
                         float k0 = up ? rm[2] : rm[0], k1 = up ? rm[3] : rm[1];
@@ -416,41 +412,43 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
                         const float s2 = up1 ? k0 : k1;
                         float kk = up1 ? k1 : k0;
                         kk = fmaxf(kk, __shfl_xor_sync(kFull, s2, 1));
-                        rrun = fmaxf(rrun, kk);
+                        atomicMax(&sKey[I * 128 + myrow], ord_key(kk));
                     }
                     if (!diag) {
-                        // ---- rows of tile J (columns here): max over tile I's rows of a_ij inv_i
-                        float cm[16];
+                        // ---- rows of tile J (this tile's columns): max over tile I's rows of
+                        // a_ij inv_i, kept per thread until the column tile is done
+                        float inv_r[4];
 #pragma unroll
-                        for (int k = 0; k < 8; ++k)
+                        for (int r = 0; r < 4; ++r) inv_r[r] = sInv[I * 128 + row_of(r)];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
 #pragma unroll
                             for (int e = 0; e < 2; ++e) {
                                 const float2 pa = __fmul2_rn(make_float2(av(0, k, e), av(1, k, e)),
                                                              make_float2(inv_r[0], inv_r[1]));
                                 const float2 pb = __fmul2_rn(make_float2(av(2, k, e), av(3, k, e)),
                                                              make_float2(inv_r[2], inv_r[3]));
-                                cm[2 * k + e] = fmax3(fmaxf(pa.x, pa.y), pb.x, pb.y);
+                                colrun[2 * k + e] = fmax3(colrun[2 * k + e], fmax3(pa.x, pa.y, pb.x), pb.y);
                             }
-                        // fold across the 8 lanes of a column group: lane g keeps columns
-                        // 2g, 2g + 1 of its 16 (k = g)
-#pragma unroll
-                        for (int lvl = 0; lvl < 3; ++lvl) {
-                            const int half = 8 >> lvl;              // values kept after this round
-                            const int bit = 4 >> lvl;               // lane bit (of g) exchanged
-                            const bool upper = (g & bit) != 0;
-#pragma unroll
-                            for (int i = 0; i < half; ++i) {
-                                const float send = upper ? cm[i] : cm[i + half];
-                                const float keep = upper ? cm[i + half] : cm[i];
-                                cm[i] = fmaxf(keep, __shfl_xor_sync(kFull, send, bit * 4));
-                            }
-                        }
-                        const int cj = c0 + 8 * g;
-                        atomicMax(&sKey[cj], ord_key(cm[0]));
-                        atomicMax(&sKey[cj + 1], ord_key(cm[1]));
                     }
                 }
-                if (ok) atomicMax(&sKey[I * 128 + myrow], ord_key(rrun));
+                if (ok && J > 0) {
+                    // fold the column maxima across the 8 lanes of a column group: lane g keeps
+                    // column (k, e) = (g >> 1, g & 1) of its 8
+#pragma unroll
+                    for (int lvl = 0; lvl < 3; ++lvl) {
+                        const int half = 4 >> lvl;              // values kept after this round
+                        const int bit = 4 >> lvl;               // lane bit (of g) exchanged
+                        const bool upper = (g & bit) != 0;
+#pragma unroll
+                        for (int i = 0; i < half; ++i) {
+                            const float send = upper ? colrun[i] : colrun[i + half];
+                            const float keep = upper ? colrun[i + half] : colrun[i];
+                            colrun[i] = fmaxf(keep, __shfl_xor_sync(kFull, send, bit * 4));
+                        }
+                    }
+                    atomicMax(&sKey[c0 + 8 * (g >> 1) + (g & 1)], ord_key(colrun[0]));
+                }
             }
             // every key of the unit is final: r = inv_i * u_i; then clear for the next unit
             epi_sync();

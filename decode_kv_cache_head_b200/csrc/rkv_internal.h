@@ -8,6 +8,7 @@
 #include <atomic>
 #include <cstddef>
 #include <cstdint>
+#include <utility>
 
 #include "../../include/rkv.h"
 
@@ -114,6 +115,20 @@ __host__ __device__ inline SmemLayout make_layout(int rp, int rmax, int cap, int
     L.bars = o;   o += 64u;
     L.total = o + 1024u;
     return L;
+}
+
+// Launches `kernel` and returns that launch's own status.  (A <<< >>> launch has to be
+// checked with cudaGetLastError, which would also report an error some unrelated
+// earlier call of the caller left behind.)
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                 cudaStream_t stream, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 // Raises a kernel's dynamic shared-memory limit only when a launch needs more

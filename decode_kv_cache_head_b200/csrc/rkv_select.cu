@@ -64,8 +64,8 @@ cudaError_t launch_select(const float *I, const float *R, int n_kv, int M, int N
     static std::atomic<int> granted{0};
     cudaError_t e = ensure_smem_attr(rkv_select_kernel, smem, granted);
     if (e != cudaSuccess) return e;
-    rkv_select_kernel<<<n_kv, kSelThreads, smem, stream>>>(I, R, M, N, budget, lambda, kept, Z);
-    return cudaGetLastError();
+    return launch_kernel(rkv_select_kernel, dim3(n_kv), dim3(kSelThreads), smem, stream, I, R, M, N,
+                         budget, lambda, kept, Z);
 }
 
 }  // namespace rkv

@@ -96,9 +96,8 @@ cudaError_t launch_plan(int batch, const int32_t *budgets, int32_t budget_cfg, i
                         int32_t window, int32_t cap, int32_t *cur_len, int32_t *n_eff,
                         uint32_t *status, cudaStream_t stream, bool update,
                         const RaggedLayout &rg) {
-    rkv_plan_kernel<<<1, 256, 0, stream>>>(batch, budgets, budget_cfg, buffer, window, cap,
-                                           cur_len, n_eff, status, update ? 1 : 0, rg);
-    return cudaGetLastError();
+    return launch_kernel(rkv_plan_kernel, dim3(1), dim3(256), 0, stream, batch, budgets, budget_cfg,
+                         buffer, window, cap, cur_len, n_eff, status, update ? 1 : 0, rg);
 }
 
 // ----------------------------------------------------------------------------

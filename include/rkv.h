@@ -120,6 +120,11 @@ RKV_API const char *rkv_status_string(rkv_status status);
 /* Library version, major * 10000 + minor * 100 + patch. */
 RKV_API int32_t rkv_version(void);
 
+/* The CUDA runtime error code (a cudaError_t value) behind the most recent
+ * RKV_ERR_CUDA that a call of this library returned on the calling thread, or 0
+ * when there was none.  Host-only; it does not touch the device. */
+RKV_API int32_t rkv_last_cuda_error(void);
+
 /*
  * Bytes of device workspace every call below needs for the given shapes
  * (n_layers = batch = 1 and cap = the per-head row count for the per-head

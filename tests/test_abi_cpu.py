@@ -216,3 +216,10 @@ def test_ragged_layout_helpers():
     Y = unpack_ragged(P, [10, 3, 7], 2, 10)
     assert torch.equal(Y[:, 0], X[:, 0])
     assert torch.equal(Y[:, 2, :, :7], X[:, 2, :, :7]) and not Y[:, 2, :, 7:].any()
+
+
+def test_max_redundancy_row_limit():
+    """MAX redundancy keeps per-row keys and norms of a whole unit in the similarity
+    kernel's shared memory: caches longer than 7680 rows are refused on the host."""
+    cm = rkv.make_config(redundancy_mode=rkv.RKV_RED_MAX)
+    assert _step(cm, cap=7808, ws_bytes=1 << 30) == -6
