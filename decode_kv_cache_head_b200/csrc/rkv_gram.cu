@@ -58,6 +58,7 @@ constexpr int kAcc = 4;                            // TMEM accumulators of 128 c
 constexpr uint32_t kTileBytes = 128u * 256u;       // 128 rows x 128 bf16
 constexpr uint32_t kHalfBytes = kTileBytes / 2;
 constexpr uint32_t kTmemCols = 128u * kAcc;
+constexpr uint32_t kBackoffNs = 64;              // producer / MMA polling interval
 
 struct GramLayout {
     uint32_t a, b, key, inv, pages, bars, total;
@@ -222,7 +223,7 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
             for (int J = 0; J < u.T && ok; ++J) {
                 if (lane == 0) {
                     const uint32_t a = na & 1u;
-                    if (na >= 2 && !mbar_wait(&aempty[a], ((na >> 1) - 1) & 1u)) ok = false;
+                    if (na >= 2 && !mbar_wait_backoff(&aempty[a], ((na >> 1) - 1) & 1u, kBackoffNs)) ok = false;
                     if (ok) {
                         mbar_arrive_expect_tx(&afull[a], kTileBytes);
                         load_tile(sA + a * kTileBytes, &afull[a], J);
@@ -230,7 +231,7 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
                     ++na;
                     for (int I = 0; I < J && ok; ++I) {
                         const uint32_t s = nb % kBStages;
-                        if (nb >= kBStages && !mbar_wait(&bempty[s], ((nb / kBStages) - 1) & 1u)) {
+                        if (nb >= kBStages && !mbar_wait_backoff(&bempty[s], ((nb / kBStages) - 1) & 1u, kBackoffNs)) {
                             ok = false;
                             break;
                         }
@@ -259,18 +260,18 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
                 if (u.N <= 0 || u.M <= 0) continue;
                 for (int J = 0; J < u.T && ok; ++J) {
                     const uint32_t a = na & 1u;
-                    if (!mbar_wait(&afull[a], (na >> 1) & 1u)) { ok = false; break; }
+                    if (!mbar_wait_backoff(&afull[a], (na >> 1) & 1u, kBackoffNs)) { ok = false; break; }
                     ++na;
                     const uint32_t col_base = smem_u32(sA + a * kTileBytes);
                     // the diagonal pair first (both operands the resident tile), then I = 0 .. J-1
                     for (int step = 0; step <= J && ok; ++step) {
                         const bool diag = step == 0;
                         const uint32_t t = np % kAcc;
-                        if (np >= kAcc && !mbar_wait(&tempty[t], ((np / kAcc) - 1) & 1u)) { ok = false; break; }
+                        if (np >= kAcc && !mbar_wait_backoff(&tempty[t], ((np / kAcc) - 1) & 1u, kBackoffNs)) { ok = false; break; }
                         uint32_t row_base = col_base, s = 0;
                         if (!diag) {
                             s = nb % kBStages;
-                            if (!mbar_wait(&bfull[s], (nb / kBStages) & 1u)) { ok = false; break; }
+                            if (!mbar_wait_backoff(&bfull[s], (nb / kBStages) & 1u, kBackoffNs)) { ok = false; break; }
                             row_base = smem_u32(sB + s * kTileBytes);
                         }
                         tc_fence_after();
@@ -417,19 +418,23 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
                     if (!diag) {
                         // ---- rows of tile J (this tile's columns): max over tile I's rows of
                         // a_ij inv_i, kept per thread until the column tile is done
-                        float inv_r[4];
+                        // (the packed products pair the two adjacent columns of one row, whose
+                        // accumulator values sit in adjacent registers)
+                        float2 inv_r2[4];
 #pragma unroll
-                        for (int r = 0; r < 4; ++r) inv_r[r] = sInv[I * 128 + row_of(r)];
+                        for (int r = 0; r < 4; ++r) {
+                            const float v = sInv[I * 128 + row_of(r)];
+                            inv_r2[r] = make_float2(v, v);
+                        }
 #pragma unroll
-                        for (int k = 0; k < 4; ++k)
+                        for (int k = 0; k < 4; ++k) {
+                            float2 y[4];
 #pragma unroll
-                            for (int e = 0; e < 2; ++e) {
-                                const float2 pa = __fmul2_rn(make_float2(av(0, k, e), av(1, k, e)),
-                                                             make_float2(inv_r[0], inv_r[1]));
-                                const float2 pb = __fmul2_rn(make_float2(av(2, k, e), av(3, k, e)),
-                                                             make_float2(inv_r[2], inv_r[3]));
-                                colrun[2 * k + e] = fmax3(colrun[2 * k + e], fmax3(pa.x, pa.y, pb.x), pb.y);
-                            }
+                            for (int r = 0; r < 4; ++r)
+                                y[r] = __fmul2_rn(make_float2(av(r, k, 0), av(r, k, 1)), inv_r2[r]);
+                            colrun[2 * k] = fmax3(fmax3(colrun[2 * k], y[0].x, y[1].x), y[2].x, y[3].x);
+                            colrun[2 * k + 1] = fmax3(fmax3(colrun[2 * k + 1], y[0].y, y[1].y), y[2].y, y[3].y);
+                        }
                     }
                 }
                 if (ok && J > 0) {
