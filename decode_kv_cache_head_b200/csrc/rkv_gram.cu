@@ -11,27 +11,30 @@
 // The Gram matrix is symmetric, so only the tile pairs (I <= J) of 128 x 128 are
 // computed: the accumulator of pair (I, J) gives u of the rows of tile I (row
 // maxima of a_ij inv_j) and of the rows of tile J (column maxima of a_ij inv_i).
-// The N x N matrix never leaves the chip, and the inverse norms are computed here
-// from the tiles already in shared memory: K is read once from HBM (the tiles a
-// unit reuses come from L2).
+// The N x N matrix never leaves the chip, and the inverse norms come from its
+// diagonal (||k_j||^2 = a_jj of the diagonal pair (J, J)): K is read once from
+// HBM (the tiles a unit reuses come from L2).
 //
 // Persistent CTAs (one per SM) walk the units.  Per unit the column tiles J go
 // from first to last; tile J stays resident while the row tiles I = J (the
 // diagonal, from the resident tile itself), 0, 1, ..., J-1 stream past it, so
 // every row tile's inverse norms are known when it arrives, and the column
 // maxima of tile J build up in registers over the whole column and cross lanes
-// once.  Warp roles (320 threads, one CTA per SM):
-//   warps 0-7  epilogue: inverse norms of each column tile; per pair, the
-//              accumulator read with tcgen05.ld 16x256b (each thread holds 4
-//              rows x 16 columns); row maxima folded over the 16 columns and
-//              across the 4 lanes of a row group, merged into per-row
-//              order-preserving keys in shared memory with atomicMax; column
-//              maxima kept per thread until the column tile is done, then
-//              folded across the 8 lanes of a column group and merged the same way;
-//   warp 8     producer: TMA of the column tile (double-buffered) and of the
+// once.  Warp roles (576 threads, one CTA per SM):
+//   warps 0-15 epilogue, warp w on TMEM lane quadrant w % 4 and column quarter
+//              w / 4: per pair, the accumulator read with tcgen05.ld 16x256b
+//              (each thread holds 4 rows x 8 columns); row maxima folded over
+//              the 8 columns and across the 4 lanes of a row group, merged into
+//              per-row order-preserving keys in shared memory with atomicMax;
+//              column maxima kept per thread until the column tile is done,
+//              then folded across the 8 lanes of a column group and merged the
+//              same way.  On the diagonal pair of each column tile the four
+//              warps with qd == cq turn its diagonal into the tile's inverse
+//              norms, published to all epilogue warps by one named barrier;
+//   warp 16    producer: TMA of the column tile (double-buffered) and of the
 //              row tiles (three-stage ring);
-//   warp 9     MMA issuer: 8 UMMAs (K = 128) per pair into one of four TMEM
-//              accumulators (128 columns each).
+//   warp 17    MMA issuer: 8 UMMAs (K = 128) per pair, issued from one asm
+//              block, into one of four TMEM accumulators (128 columns each).
 // Hand-offs are mbarriers; every wait is bounded and a timeout is recorded in
 // the status word (the CTA then drains what it issued and stops).
 #include <cuda.h>
@@ -168,7 +171,7 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
     if (tid == 32) {
         for (int i = 0; i < 2; ++i) {
             mbar_init(&afull[i], 1);
-            mbar_init(&aempty[i], 2);        // the row's last UMMA + the epilogue's norm pass
+            mbar_init(&aempty[i], 1);        // the column tile's last UMMA
         }
         for (int s = 0; s < kBStages; ++s) {
             mbar_init(&bfull[s], 1);
@@ -262,25 +265,20 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
                     const uint32_t a = na & 1u;
                     if (!mbar_wait_backoff(&afull[a], (na >> 1) & 1u, kBackoffNs)) { ok = false; break; }
                     ++na;
-                    const uint32_t col_base = smem_u32(sA + a * kTileBytes);
+                    const uint32_t col_lo = desc_lo_sw128(smem_u32(sA + a * kTileBytes));
                     // the diagonal pair first (both operands the resident tile), then I = 0 .. J-1
                     for (int step = 0; step <= J && ok; ++step) {
                         const bool diag = step == 0;
                         const uint32_t t = np % kAcc;
                         if (np >= kAcc && !mbar_wait_backoff(&tempty[t], ((np / kAcc) - 1) & 1u, kBackoffNs)) { ok = false; break; }
-                        uint32_t row_base = col_base, s = 0;
+                        uint32_t row_lo = col_lo, s = 0;
                         if (!diag) {
                             s = nb % kBStages;
                             if (!mbar_wait_backoff(&bfull[s], (nb / kBStages) & 1u, kBackoffNs)) { ok = false; break; }
-                            row_base = smem_u32(sB + s * kTileBytes);
+                            row_lo = desc_lo_sw128(smem_u32(sB + s * kTileBytes));
                         }
                         tc_fence_after();
-#pragma unroll
-                        for (int ks = 0; ks < 8; ++ks) {
-                            const uint32_t off = (ks >> 2) * kHalfBytes + (ks & 3) * 32u;
-                            umma_bf16(tmem_base + t * 128u, desc_kmajor_sw128(row_base + off),
-                                      desc_kmajor_sw128(col_base + off), idesc, ks > 0 ? 1u : 0u);
-                        }
+                        umma_bf16_k128_sw128(tmem_base + t * 128u, row_lo, col_lo, idesc);
                         umma_commit(&tfull[t]);
                         ++np;
                         if (!diag) {
@@ -303,55 +301,25 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
         // its 8 columns 32 cq + 8 k + 2 q + e (k = 0..3, e = 0, 1)
         auto row_of = [&](int r) { return 32 * qd + g + 8 * r; };
         const int myrow = row_of(q);
-        // norms (warps 0-7): two threads per row, 64 columns each
-        const int nrow = (lane & 7) + 8 * (lane >> 4), nhalf = (lane >> 3) & 1;
-        const int row_t = 16 * warp + nrow;
+        // the diagonal of the 32 x 32 block of a warp with qd == cq: lane (g, q = g / 2)
+        // holds a_jj of columns 32 cq + 8 r + g (r = 0..3) in register e = g % 2 of (r, k = r)
+        const bool diag_lane = qd == cq && q == (g >> 1);
         // A wait that runs out makes `ok` false for the whole warp (so the warp's
         // .sync.aligned TMEM loads never diverge); a failed warp skips the work but keeps
         // every named barrier of the schedule, so the other epilogue warps never wait
         // on it at a barrier without a time limit.
         auto wait_all = [&](uint64_t *bar, uint32_t parity) {
-            const bool w = ok ? mbar_wait(bar, parity) : false;
+            const bool w = ok && (mbar_test_wait(bar, parity) || mbar_wait(bar, parity));
             ok = __all_sync(kFull, w) != 0;
         };
-        uint32_t na = 0, np = 0;
+        uint32_t np = 0;
         for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
             const UnitInfo u = unit_info(p, unit);
             if (u.N <= 0 || u.M <= 0) continue;
             for (int J = 0; J < u.T; ++J) {
-                const uint32_t a = na & 1u;
-                wait_all(&afull[a], (na >> 1) & 1u);
-                ++na;
-                if (ok && warp < 8) {
-                    // 1 / max(||k_j||, 1e-12) of the column tile's rows (0 past N)
-                    const uint8_t *hp = sA + a * kTileBytes + nhalf * kHalfBytes + row_t * 128;
-                    float2 ss2 = make_float2(0.f, 0.f);
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const uint4 raw = *reinterpret_cast<const uint4 *>(hp + ((c ^ (row_t & 7)) << 4));
-                        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 f = __bfloat1622float2(h2[e]);
-                            ss2 = __ffma2_rn(f, f, ss2);
-                        }
-                    }
-                    const float ssh = ss2.x + ss2.y;
-                    const float ss = ssh + __shfl_xor_sync(kFull, ssh, 8);
-                    const int i = J * 128 + row_t;
-                    if (nhalf == 0) sInv[i] = i < u.N ? 1.0f / fmaxf(sqrtf(ss), 1e-12f) : 0.f;
-                }
-                epi_sync();
-                if (tid == 0) mbar_arrive(&aempty[a]);   // the epilogue is done reading the tile
                 const int c0 = J * 128 + 32 * cq + 2 * q;    // unit row of this thread's column (k, e) = (0, 0)
-                float inv_c[8];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float2 iv = *reinterpret_cast<const float2 *>(&sInv[c0 + 8 * k]);
-                    inv_c[2 * k] = iv.x;
-                    inv_c[2 * k + 1] = iv.y;
-                }
                 const bool tail = (J + 1) * 128 > u.N;       // columns past N in this tile
+                float inv_c[8];                              // inverse norms of this thread's columns
                 float colrun[8];                             // max over the rows seen of a_ij inv_i
 #pragma unroll
                 for (int c = 0; c < 8; ++c) colrun[c] = -INFINITY;
@@ -361,23 +329,46 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
                     const uint32_t t = np % kAcc;
                     wait_all(&tfull[t], (np / kAcc) & 1u);
                     ++np;
-                    if (!ok) continue;
-                    tc_fence_after();
                     uint32_t v0[16], v1[16];   // slab 0 (rows 0, 1), slab 1 (rows 2, 3)
-                    const uint32_t tcol = tmem_base + t * 128u + 32u * cq;
-                    tmem_ld_16x256b_x4(tcol + ((32u * qd) << 16), v0);
-                    tmem_ld_16x256b_x4(tcol + ((32u * qd + 16u) << 16), v1);
-                    tmem_wait_ld();
-                    reg_tie16(v0);
-                    reg_tie16(v1);
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&tempty[t]);   // the accumulator may be reused
+                    if (ok) {
+                        tc_fence_after();
+                        const uint32_t tcol = tmem_base + t * 128u + 32u * cq;
+                        tmem_ld_16x256b_x4(tcol + ((32u * qd) << 16), v0);
+                        tmem_ld_16x256b_x4(tcol + ((32u * qd + 16u) << 16), v1);
+                        tmem_wait_ld();
+                        reg_tie16(v0);
+                        reg_tie16(v1);
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&tempty[t]);   // the accumulator may be reused
+                    }
                     // a(row r, column k, e): slab r >> 1, register 4k + 2 (r & 1) + e
                     auto av = [&](int r, int k, int e) -> float {
                         const uint32_t x = (r < 2) ? v0[4 * k + 2 * (r & 1) + e] : v1[4 * k + 2 * (r & 1) + e];
                         return __uint_as_float(x);
                     };
+                    if (diag) {
+                        // 1 / max(||k_j||, 1e-12) of the column tile's rows (0 past N), with
+                        // ||k_j||^2 = a_jj read off the diagonal of the tile's own Gram block;
+                        // the barrier publishes them to every epilogue warp (rows of a later
+                        // row tile are read by other warps than the one that wrote them)
+                        if (ok && diag_lane) {
+#pragma unroll
+                            for (int r = 0; r < 4; ++r) {
+                                const float ss = (g & 1) ? av(r, r, 1) : av(r, r, 0);
+                                const int j = J * 128 + 32 * cq + 8 * r + g;
+                                sInv[j] = j < u.N ? 1.0f / fmaxf(sqrtf(ss), 1e-12f) : 0.f;
+                            }
+                        }
+                        epi_sync();
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const float2 iv = *reinterpret_cast<const float2 *>(&sInv[c0 + 8 * k]);
+                            inv_c[2 * k] = iv.x;
+                            inv_c[2 * k + 1] = iv.y;
+                        }
+                    }
+                    if (!ok) continue;
                     // ---- rows of tile I: max over this tile's columns of a_ij inv_j
                     float rm[4];
 #pragma unroll

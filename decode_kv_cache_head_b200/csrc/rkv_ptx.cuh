@@ -62,6 +62,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// One non-blocking test of phase `parity` (the thread is never suspended).  On a
+// phase that has already completed it answers sooner than mbar_try_wait, so a wait
+// that is usually satisfied on arrival tests first.  A true answer orders like a
+// completed wait.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Waits for phase `parity` of `bar` to complete; gives up after kWaitLimitNs
 // and returns false (the caller records kDevFlagTimeout).
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
@@ -158,6 +174,51 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// D = A B^T over K = 128 for two 128 x 128 bf16 tiles stored K-major with the
+// 128-byte swizzle as two 64-column halves 16 KB apart (the layout of a 2-D TMA
+// box pair): eight UMMAs of K = 16 issued back to back from one asm block, the
+// first overwriting D.  `a_lo` / `b_lo` are the low descriptor words of the
+// tiles' first bytes (desc_lo_sw128); the K steps advance them by 32 bytes
+// inside a half and by 16 KB between halves, so no descriptor is rebuilt
+// between issues.
+__device__ __forceinline__ uint32_t desc_lo_sw128(uint32_t smem_addr) {
+    return ((smem_addr >> 4) & 0x3FFFu) | (1u << 16);
+}
+constexpr uint32_t kDescHiSw128 = (1024u >> 4) | (1u << 14) | (2u << 29);
+
+__device__ __forceinline__ void umma_bf16_k128_sw128(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
+                                                     uint32_t idesc) {
+    asm volatile(
+        "{\n\t.reg .pred pf, pt;\n\t.reg .b64 da, db;\n\t.reg .b32 al, bl;\n\t"
+        "setp.ne.b32 pf, %1, %1;\n\t"
+        "setp.eq.b32 pt, %1, %1;\n\t"
+        "mov.b64 da, {%1, %3};\n\tmov.b64 db, {%2, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, pf;\n\t"
+        "add.u32 al, %1, 2;\n\tadd.u32 bl, %2, 2;\n\t"
+        "mov.b64 da, {al, %3};\n\tmov.b64 db, {bl, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, pt;\n\t"
+        "add.u32 al, %1, 4;\n\tadd.u32 bl, %2, 4;\n\t"
+        "mov.b64 da, {al, %3};\n\tmov.b64 db, {bl, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, pt;\n\t"
+        "add.u32 al, %1, 6;\n\tadd.u32 bl, %2, 6;\n\t"
+        "mov.b64 da, {al, %3};\n\tmov.b64 db, {bl, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, pt;\n\t"
+        "add.u32 al, %1, 1024;\n\tadd.u32 bl, %2, 1024;\n\t"
+        "mov.b64 da, {al, %3};\n\tmov.b64 db, {bl, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, pt;\n\t"
+        "add.u32 al, %1, 1026;\n\tadd.u32 bl, %2, 1026;\n\t"
+        "mov.b64 da, {al, %3};\n\tmov.b64 db, {bl, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, pt;\n\t"
+        "add.u32 al, %1, 1028;\n\tadd.u32 bl, %2, 1028;\n\t"
+        "mov.b64 da, {al, %3};\n\tmov.b64 db, {bl, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, pt;\n\t"
+        "add.u32 al, %1, 1030;\n\tadd.u32 bl, %2, 1030;\n\t"
+        "mov.b64 da, {al, %3};\n\tmov.b64 db, {bl, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, pt;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_lo), "r"(b_lo), "r"(kDescHiSw128), "r"(idesc)
         : "memory");
 }
 
