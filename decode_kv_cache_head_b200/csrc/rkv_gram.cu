@@ -309,7 +309,7 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
         // every named barrier of the schedule, so the other epilogue warps never wait
         // on it at a barrier without a time limit.
         auto wait_all = [&](uint64_t *bar, uint32_t parity) {
-            const bool w = ok && (mbar_test_wait(bar, parity) || mbar_wait(bar, parity));
+            const bool w = ok && mbar_wait(bar, parity);
             ok = __all_sync(kFull, w) != 0;
         };
         uint32_t np = 0;

@@ -81,6 +81,7 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
 // Waits for phase `parity` of `bar` to complete; gives up after kWaitLimitNs
 // and returns false (the caller records kDevFlagTimeout).
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+    if (mbar_test_wait(bar, parity)) return true;   // usually complete on arrival
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
