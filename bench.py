@@ -57,7 +57,7 @@ def parse_args():
     ap.add_argument("--impl", default="rkv", choices=["rkv", "reference"])
     ap.add_argument("--workload", default="ragged_batch", choices=sorted(WORKLOADS))
     ap.add_argument("--redundancy", default="mean", choices=["mean", "max"])
-    ap.add_argument("--e2e-steps", type=int, default=6)
+    ap.add_argument("--e2e-steps", type=int, default=12)
     ap.add_argument("--layers", type=int, default=0,
                     help="run the workload with this many layers instead of its own (a smaller "
                          "case of the same shape, for profiler captures); 0 = the workload's")
