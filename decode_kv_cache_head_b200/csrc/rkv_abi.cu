@@ -173,7 +173,8 @@ cudaError_t launch_unit_layers(const rkv_config *cfg, int32_t n_layers, int32_t 
                                int32_t *kept_out, float *scores_out, float *z_heads,
                                uint32_t *status, const UnitShape &us, int nqp, cudaStream_t strm,
                                const PagedArgs &pg = PagedArgs{nullptr, 0, 0, 0},
-                               const RaggedLayout &rg = RaggedLayout{}) {
+                               const RaggedLayout &rg = RaggedLayout{},
+                               const int32_t *order = nullptr) {
     UnitParams *up = new UnitParams();
     std::memset(up, 0, sizeof(*up));
     up->batch = batch;
@@ -192,6 +193,7 @@ cudaError_t launch_unit_layers(const rkv_config *cfg, int32_t n_layers, int32_t 
     up->budgets = budgets;
     up->lambdas = lambdas;
     up->n_eff = n_eff;
+    up->order = order;
     up->r_ext = r_ext;
     up->kept_out = kept_out;
     up->scores_out = scores_out;
@@ -237,7 +239,8 @@ cudaError_t launch_gram_layers(const rkv_config *cfg, int32_t n_layers, int32_t 
                                uint32_t *status, cudaStream_t strm, cudaEvent_t sim_begin = nullptr,
                                cudaEvent_t sim_end = nullptr,
                                const RaggedLayout &rg = RaggedLayout{},
-                               const PagedArgs &pg = PagedArgs{nullptr, 0, 0, 0}) {
+                               const PagedArgs &pg = PagedArgs{nullptr, 0, 0, 0},
+                               const int32_t *order = nullptr) {
     GramParams *gp = new GramParams();
     std::memset(gp, 0, sizeof(*gp));
     gp->batch = batch;
@@ -245,6 +248,7 @@ cudaError_t launch_gram_layers(const rkv_config *cfg, int32_t n_layers, int32_t 
     gp->window = cfg->window;
     gp->cap = cap;
     gp->n_eff = n_eff;
+    gp->order = order;
     gp->seq_row = rg.seq_row;
     gp->seq_cap = rg.seq_cap;
     gp->block_table = pg.block_table;
@@ -286,6 +290,17 @@ size_t ws_bytes_for(const rkv_config *cfg, int32_t n_layers, int32_t batch, int3
 size_t ws_bytes_shared(const rkv_config *cfg, int32_t n_layers, int32_t batch, int32_t cap) {
     const size_t units = static_cast<size_t>(n_layers) * batch * cfg->n_kv_heads;
     return ws_bytes_for(cfg, n_layers, batch, cap) + align256(units * cap * 4);
+}
+
+// Past the part a call needs (`base` bytes), a workspace may hold the plan kernel's
+// order of the sequences by decreasing length (one int32 each); the batched kernels
+// then start the longest sequences' units first.  rkv_workspace_size and
+// rkv_workspace_size_shared include that room; a workspace without it runs the units in
+// layer-major order (same results).
+size_t order_bytes(int32_t batch) { return align256(static_cast<size_t>(batch) * 4); }
+
+int32_t *order_slot(uint8_t *ws, size_t ws_bytes, size_t base, int32_t batch) {
+    return ws_bytes >= base + order_bytes(batch) ? reinterpret_cast<int32_t *>(ws + base) : nullptr;
 }
 
 void fill_common(StepParams &p, const rkv_config *cfg, const Shape &s, int batch, int cap) {
@@ -375,6 +390,19 @@ rkv_status run_per_head_scores(const rkv_config *cfg, const rkv_bf16 *q, const r
 
 }  // namespace
 
+// The part of a step's workspace the call cannot run without (no room for the order of
+// the sequences); 0 for an invalid configuration.
+namespace rkv {
+size_t workspace_required_bytes(const rkv_config *cfg, int32_t n_layers, int32_t batch,
+                                int32_t cap);
+}  // namespace rkv
+
+size_t rkv::workspace_required_bytes(const rkv_config *cfg, int32_t n_layers, int32_t batch,
+                                     int32_t cap) {
+    if (check_cfg(cfg) != RKV_OK || n_layers < 1 || batch < 1 || cap < 2) return 0;
+    return ws_bytes_for(cfg, n_layers, batch, cap);
+}
+
 extern "C" {
 
 const char *rkv_status_string(rkv_status s) {
@@ -400,7 +428,7 @@ int32_t rkv_last_cuda_error(void) { return g_last_cuda_error; }
 
 size_t rkv_workspace_size(const rkv_config *cfg, int32_t n_layers, int32_t batch, int32_t cap) {
     if (check_cfg(cfg) != RKV_OK || n_layers < 1 || batch < 1 || cap < 2) return 0;
-    return ws_bytes_for(cfg, n_layers, batch, cap);
+    return ws_bytes_for(cfg, n_layers, batch, cap) + order_bytes(batch);
 }
 
 rkv_status rkv_query_step_shape(const rkv_config *cfg, int64_t n_units, int32_t cap,
@@ -585,6 +613,8 @@ rkv_status rkv_compress_step(const rkv_config *cfg, int32_t n_layers, int32_t ba
     int32_t *n_eff = reinterpret_cast<int32_t *>(ws + kStatusBytes);
     float *r_ext = reinterpret_cast<float *>(ws + kStatusBytes + align256(static_cast<size_t>(batch) * 4));
     const bool red_max = cfg->redundancy_mode == RKV_RED_MAX;
+    int32_t *order = unit_path ? order_slot(ws, ws_bytes, ws_bytes_for(cfg, n_layers, batch, cap), batch)
+                               : nullptr;
 
     StepParams *pp = new StepParams();
     StepParams &p = *pp;
@@ -601,18 +631,19 @@ rkv_status rkv_compress_step(const rkv_config *cfg, int32_t n_layers, int32_t ba
 
     // the plan kernel clears the status words first
     cudaError_t e = launch_plan(batch, budgets, cfg->budget, cfg->buffer, cfg->window, cap, cur_len,
-                                n_eff, status, strm);
+                                n_eff, status, strm, true, RaggedLayout{}, order);
     if (red_max && e == cudaSuccess)   // raw r of every candidate: the tcgen05 similarity kernel
         e = launch_gram_layers(cfg, n_layers, batch, cap,
                                const_cast<const rkv_bf16 *const *>(k_layers), n_eff, r_ext, status,
                                strm, opts ? reinterpret_cast<cudaEvent_t>(opts->sim_begin) : nullptr,
-                               opts ? reinterpret_cast<cudaEvent_t>(opts->sim_end) : nullptr);
+                               opts ? reinterpret_cast<cudaEvent_t>(opts->sim_end) : nullptr,
+                               RaggedLayout{}, PagedArgs{nullptr, 0, 0, 0}, order);
     if (e == cudaSuccess && opts && opts->main_begin)
         e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->main_begin), strm);
     if (unit_path && e == cudaSuccess)
         e = launch_unit_layers(cfg, n_layers, batch, cap, k_layers, v_layers, q_layers, budgets,
                                lambdas, n_eff, p.r_ext, p.kept_out, p.scores_out, nullptr, status,
-                               us, nqp, strm);
+                               us, nqp, strm, PagedArgs{nullptr, 0, 0, 0}, RaggedLayout{}, order);
     for (int l0 = 0; !unit_path && e == cudaSuccess && l0 < n_layers; l0 += kMaxLayersPerLaunch) {
         const int nl = (n_layers - l0 < kMaxLayersPerLaunch) ? n_layers - l0 : kMaxLayersPerLaunch;
         p.n_layers = nl;
@@ -692,7 +723,7 @@ rkv_status rkv_append_kv(const rkv_config *cfg, int32_t n_layers, int32_t batch,
 size_t rkv_workspace_size_shared(const rkv_config *cfg, int32_t n_layers, int32_t batch,
                                  int32_t cap) {
     if (check_cfg(cfg) != RKV_OK || n_layers < 1 || batch < 1 || cap < 2) return 0;
-    return ws_bytes_shared(cfg, n_layers, batch, cap);
+    return ws_bytes_shared(cfg, n_layers, batch, cap) + order_bytes(batch);
 }
 
 }  // extern "C"
@@ -758,15 +789,19 @@ rkv_status rkv_score_shared(const rkv_config *cfg, int32_t n_layers, int32_t bat
     float *r_ext = reinterpret_cast<float *>(ws + kStatusBytes + align256(static_cast<size_t>(batch) * 4));
     float *z_heads = reinterpret_cast<float *>(ws + base);
     const bool red_max = cfg->redundancy_mode == RKV_RED_MAX;
+    int32_t *order = order_slot(ws, ws_bytes, ws_bytes_shared(cfg, n_layers, batch, cap), batch);
     // the plan kernel clears the status words first
     cudaError_t e = launch_plan(batch, budgets, cfg->budget, cfg->buffer, cfg->window, cap,
-                                const_cast<int32_t *>(cur_len), n_eff, status, strm, false);
+                                const_cast<int32_t *>(cur_len), n_eff, status, strm, false,
+                                RaggedLayout{}, order);
     if (red_max && e == cudaSuccess)
-        e = launch_gram_layers(cfg, n_layers, batch, cap, k_layers, n_eff, r_ext, status, strm);
+        e = launch_gram_layers(cfg, n_layers, batch, cap, k_layers, n_eff, r_ext, status, strm,
+                               nullptr, nullptr, RaggedLayout{}, PagedArgs{nullptr, 0, 0, 0}, order);
     if (e == cudaSuccess)
         e = launch_unit_layers(cfg, n_layers, batch, cap, k_layers, nullptr, q_layers, budgets,
                                lambdas, n_eff, red_max ? r_ext : nullptr, nullptr, nullptr, z_heads,
-                               status, us, nqp, strm);
+                               status, us, nqp, strm, PagedArgs{nullptr, 0, 0, 0}, RaggedLayout{},
+                               order);
     SharedParams sp;
     std::memset(&sp, 0, sizeof(sp));
     sp.batch = batch;
@@ -870,15 +905,16 @@ rkv_status rkv_compress_step_paged(const rkv_config *cfg, int32_t n_layers, int3
     float *r_ext = reinterpret_cast<float *>(ws + kStatusBytes + align256(static_cast<size_t>(batch) * 4));
     const bool red_max = cfg->redundancy_mode == RKV_RED_MAX;
     const PagedArgs pa{pg->block_table, pg->max_blocks, P, pg->num_pages};
+    int32_t *order = order_slot(ws, ws_bytes, ws_bytes_for(cfg, n_layers, batch, cap), batch);
     // the plan kernel clears the status words first
     cudaError_t e = launch_plan(batch, budgets, cfg->budget, cfg->buffer, cfg->window, cap, cur_len,
-                                n_eff, status, strm, true);
+                                n_eff, status, strm, true, RaggedLayout{}, order);
     if (red_max && e == cudaSuccess)   // raw r of every candidate, through the block table
         e = launch_gram_layers(cfg, n_layers, batch, cap,
                                const_cast<const rkv_bf16 *const *>(k_pools), n_eff, r_ext, status,
                                strm, opts ? reinterpret_cast<cudaEvent_t>(opts->sim_begin) : nullptr,
                                opts ? reinterpret_cast<cudaEvent_t>(opts->sim_end) : nullptr,
-                               RaggedLayout{}, pa);
+                               RaggedLayout{}, pa, order);
     if (e == cudaSuccess)
         e = launch_freed_pages(batch, budgets, cfg->budget, n_eff, pg->block_table, pg->max_blocks,
                                P, pg->freed_pages, pg->n_freed, strm);
@@ -889,7 +925,8 @@ rkv_status rkv_compress_step_paged(const rkv_config *cfg, int32_t n_layers, int3
                                const_cast<const rkv_bf16 *const *>(k_pools), v_pools, q_layers,
                                budgets, lambdas, n_eff, red_max ? r_ext : nullptr,
                                opts ? opts->kept_out : nullptr,
-                               opts ? opts->scores_out : nullptr, nullptr, status, us, nqp, strm, pa);
+                               opts ? opts->scores_out : nullptr, nullptr, status, us, nqp, strm, pa,
+                               RaggedLayout{}, order);
     if (e == cudaSuccess && opts && opts->main_end)
         e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->main_end), strm);
     return cuda_status(e);
@@ -941,15 +978,17 @@ rkv_status rkv_compress_step_ragged(const rkv_config *cfg, int32_t n_layers, int
     lay.seq_cap = rg->seq_cap;
     lay.pool_rows = rg->pool_rows;
     lay.n_kv = cfg->n_kv_heads;
+    int32_t *order = order_slot(ws, ws_bytes, ws_bytes_for(cfg, n_layers, batch, cap), batch);
     // the plan kernel clears the status words first, then checks every due sequence's
     // block against the pool
     cudaError_t e = launch_plan(batch, budgets, cfg->budget, cfg->buffer, cfg->window, cap, cur_len,
-                                n_eff, status, strm, true, lay);
+                                n_eff, status, strm, true, lay, order);
     if (red_max && e == cudaSuccess)
         e = launch_gram_layers(cfg, n_layers, batch, cap,
                                const_cast<const rkv_bf16 *const *>(k_pools), n_eff, r_ext, status,
                                strm, opts ? reinterpret_cast<cudaEvent_t>(opts->sim_begin) : nullptr,
-                               opts ? reinterpret_cast<cudaEvent_t>(opts->sim_end) : nullptr, lay);
+                               opts ? reinterpret_cast<cudaEvent_t>(opts->sim_end) : nullptr, lay,
+                               PagedArgs{nullptr, 0, 0, 0}, order);
     if (e == cudaSuccess && opts && opts->main_begin)
         e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->main_begin), strm);
     if (e == cudaSuccess)
@@ -957,7 +996,8 @@ rkv_status rkv_compress_step_ragged(const rkv_config *cfg, int32_t n_layers, int
                                const_cast<const rkv_bf16 *const *>(k_pools), v_pools, q_layers,
                                budgets, lambdas, n_eff, red_max ? r_ext : nullptr,
                                opts ? opts->kept_out : nullptr, opts ? opts->scores_out : nullptr,
-                               nullptr, status, us, nqp, strm, PagedArgs{nullptr, 0, 0, 0}, lay);
+                               nullptr, status, us, nqp, strm, PagedArgs{nullptr, 0, 0, 0}, lay,
+                               order);
     if (e == cudaSuccess && opts && opts->main_end)
         e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->main_end), strm);
     return cuda_status(e);

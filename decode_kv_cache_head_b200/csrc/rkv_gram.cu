@@ -127,11 +127,12 @@ struct UnitInfo {
     int64_t unit_g, krow0;
 };
 
-__device__ __forceinline__ UnitInfo unit_info(const GramParams &p, int unit) {
+__device__ __forceinline__ UnitInfo unit_info(const GramParams &p, int unit, int n_units) {
     UnitInfo u;
-    u.h = unit % p.n_kv;
-    u.b = (unit / p.n_kv) % p.batch;
-    u.l = unit / (p.n_kv * p.batch);
+    const UnitCoord c = unit_coord(unit, p.n_kv, p.batch, n_units / (p.n_kv * p.batch), p.order);
+    u.h = c.h;
+    u.b = c.b;
+    u.l = c.l;
     u.N = p.n_tokens_fixed > 0 ? p.n_tokens_fixed : p.n_eff[u.b];
     u.M = u.N - p.window;
     u.T = (u.N + 127) / 128;
@@ -196,7 +197,7 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
         // ---------------- producer: per unit, column tiles 0 .. T-1; row tiles 0 .. J-1 of each
         uint32_t na = 0, nb = 0;
         for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x) {
-            const UnitInfo u = unit_info(p, unit);
+            const UnitInfo u = unit_info(p, unit, n_units);
             if (u.N <= 0 || u.M <= 0) continue;
             const CUtensorMap *map = &p.tmap[u.l];
             if (paged) {
@@ -259,7 +260,7 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
             constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
             uint32_t na = 0, nb = 0, np = 0;
             for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x) {
-                const UnitInfo u = unit_info(p, unit);
+                const UnitInfo u = unit_info(p, unit, n_units);
                 if (u.N <= 0 || u.M <= 0) continue;
                 for (int J = 0; J < u.T && ok; ++J) {
                     const uint32_t a = na & 1u;
@@ -314,7 +315,7 @@ __global__ void __launch_bounds__(kGramThreads, 1) rkv_gram_max_kernel(const __g
         };
         uint32_t np = 0;
         for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
-            const UnitInfo u = unit_info(p, unit);
+            const UnitInfo u = unit_info(p, unit, n_units);
             if (u.N <= 0 || u.M <= 0) continue;
             for (int J = 0; J < u.T; ++J) {
                 const int c0 = J * 128 + 32 * cq + 2 * q;    // unit row of this thread's column (k, e) = (0, 0)

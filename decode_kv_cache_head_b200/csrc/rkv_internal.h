@@ -170,7 +170,28 @@ __device__ __forceinline__ int64_t unit_first_row(const int64_t *seq_row, const 
 cudaError_t launch_plan(int batch, const int32_t *budgets, int32_t budget_cfg, int32_t buffer,
                         int32_t window, int32_t cap, int32_t *cur_len, int32_t *n_eff,
                         uint32_t *status, cudaStream_t stream, bool update = true,
-                        const RaggedLayout &rg = RaggedLayout{});
+                        const RaggedLayout &rg = RaggedLayout{}, int32_t *order = nullptr);
+
+// Unit `pos` of a launch over `n_layers` layers x `batch` sequences x `n_kv` heads, in
+// the launch's order: by default layer-major (l, b, h); with `order` (the plan kernel's
+// sequences by decreasing length) sequence-major (rank, l, h), so that the units of the
+// longest sequences start first and a launch of many units ends on short ones.
+struct UnitCoord {
+    int l, b, h;
+};
+__host__ __device__ inline UnitCoord unit_coord(int pos, int n_kv, int batch, int n_layers,
+                                                const int32_t *order) {
+    UnitCoord c;
+    c.h = pos % n_kv;
+    if (order == nullptr) {
+        c.b = (pos / n_kv) % batch;
+        c.l = pos / (n_kv * batch);
+    } else {
+        c.l = (pos / n_kv) % n_layers;
+        c.b = order[pos / (n_kv * n_layers)];
+    }
+    return c;
+}
 cudaError_t launch_step(const StepParams &p, int n_units, int nqp, size_t smem,
                         cudaStream_t stream);
 size_t step_smem_bytes(int rp, int rmax, int cap, int nqp, int cs);
@@ -200,6 +221,7 @@ struct alignas(64) UnitParams {
     const int32_t *budgets;
     const float *lambdas;
     const int32_t *n_eff;
+    const int32_t *order;  // sequences by decreasing length (plan kernel), or null: launch order
     const float *r_ext;
     int32_t *kept_out;
     float *scores_out;
@@ -285,6 +307,7 @@ struct alignas(64) GramParams {
     int32_t layer_base, batch, n_kv, window, cap;
     int32_t n_tokens_fixed;  // > 0: per-head entry point, N fixed
     const int32_t *n_eff;
+    const int32_t *order;    // sequences by decreasing length (plan kernel), or null
     const int64_t *seq_row;  // per-sequence capacities, as in UnitParams (or null)
     const int32_t *seq_cap;
     const int32_t *block_table;   // paged caches, as in UnitParams (or null)

@@ -19,6 +19,12 @@
 
 #include "../../include/rkv.h"
 
+namespace rkv {
+// The part of a step's workspace the call cannot run without (rkv_abi.cu).
+size_t workspace_required_bytes(const rkv_config *cfg, int32_t n_layers, int32_t batch,
+                                int32_t cap);
+}  // namespace rkv
+
 namespace {
 
 constexpr size_t kScratchBytes = RKV_NOALLOC_SCRATCH_BYTES;
@@ -60,7 +66,7 @@ extern "C" rkv_status rkv_compress_step_noalloc(const rkv_config *cfg, int32_t n
                                                 rkv_stream_t stream) {
     if (!cfg) return RKV_ERR_NULL;
     if (n_layers < 1 || batch < 1 || cap < 2) return RKV_ERR_INVALID;
-    const size_t need = rkv_workspace_size(cfg, n_layers, batch, cap);
+    const size_t need = rkv::workspace_required_bytes(cfg, n_layers, batch, cap);
     if (need == 0)   // invalid config: let the step report exactly what is wrong
         return rkv_compress_step(cfg, n_layers, batch, cap, k_layers, v_layers, q_layers, budgets,
                                  lambdas, cur_len, opts, nullptr, 0, stream);

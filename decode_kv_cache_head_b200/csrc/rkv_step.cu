@@ -57,14 +57,15 @@ namespace rkv {
 
 // ----------------------------------------------------------------------------
 // Plan: clear the status words; which sequences are due; snapshot their length;
-// set cur_len = budget.  One CTA, so the clearing precedes every flag it records.
+// set cur_len = budget; optionally order the sequences by decreasing length.  One
+// CTA, so the clearing precedes every flag it records.
 // ----------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) rkv_plan_kernel(int batch, const int32_t *__restrict__ budgets,
                                                        int32_t budget_cfg, int32_t buffer, int32_t window,
                                                        int32_t cap, int32_t *__restrict__ cur_len,
                                                        int32_t *__restrict__ n_eff,
                                                        uint32_t *__restrict__ status, int update,
-                                                       RaggedLayout rg) {
+                                                       RaggedLayout rg, int32_t *__restrict__ order) {
     // the kernel that follows may be scheduled now; it waits for this one to finish
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     for (int i = threadIdx.x; i < static_cast<int>(kStatusBytes / 4); i += blockDim.x) status[i] = 0u;
@@ -90,14 +91,40 @@ __global__ void __launch_bounds__(256) rkv_plan_kernel(int batch, const int32_t 
         n_eff[b] = due ? n : 0;
         if (due && update) cur_len[b] = bud;
     }
+    if (order == nullptr) return;
+    // The sequences by decreasing tile count (ceil(N / 128), 0 when not due): a launch
+    // that takes its units in this order starts the longest first and ends on the
+    // shortest.  A counting sort over the tile counts; the order inside one count is
+    // whichever the atomics give, which changes no result (units are independent).
+    constexpr int kBins = 64;
+    __shared__ uint32_t cnt[kBins];
+    for (int i = threadIdx.x; i < kBins; i += blockDim.x) cnt[i] = 0u;
+    __syncthreads();   // also: every n_eff above is written
+    auto bin_of = [&](int b) {
+        const int n = n_eff[b];
+        return n > 0 ? min((n + 127) / 128, kBins - 1) : 0;
+    };
+    for (int b = threadIdx.x; b < batch; b += blockDim.x) atomicAdd(&cnt[bin_of(b)], 1u);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t run = 0;   // start of each bin, the highest bin first
+        for (int i = kBins - 1; i >= 0; --i) {
+            const uint32_t c = cnt[i];
+            cnt[i] = run;
+            run += c;
+        }
+    }
+    __syncthreads();
+    for (int b = threadIdx.x; b < batch; b += blockDim.x)
+        order[atomicAdd(&cnt[bin_of(b)], 1u)] = b;
 }
 
 cudaError_t launch_plan(int batch, const int32_t *budgets, int32_t budget_cfg, int32_t buffer,
                         int32_t window, int32_t cap, int32_t *cur_len, int32_t *n_eff,
                         uint32_t *status, cudaStream_t stream, bool update,
-                        const RaggedLayout &rg) {
+                        const RaggedLayout &rg, int32_t *order) {
     return launch_kernel(rkv_plan_kernel, dim3(1), dim3(256), 0, stream, batch, budgets, budget_cfg,
-                         buffer, window, cap, cur_len, n_eff, status, update ? 1 : 0, rg);
+                         buffer, window, cap, cur_len, n_eff, status, update ? 1 : 0, rg, order);
 }
 
 // ----------------------------------------------------------------------------

@@ -117,15 +117,14 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
     uint8_t *base = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
 
-    const int unit = blockIdx.x;
-    const int h = unit % p.n_kv;
-    const int b = (unit / p.n_kv) % p.batch;
-    const int l = unit / (p.n_kv * p.batch);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wg = warp >> 2;
 
     // launched as a programmatic dependent of the plan kernel: nothing it wrote (or that
     // ran before it) is read before this wait
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    const UnitCoord uc = unit_coord(static_cast<int>(blockIdx.x), p.n_kv, p.batch,
+                                    static_cast<int>(gridDim.x) / (p.n_kv * p.batch), p.order);
+    const int h = uc.h, b = uc.b, l = uc.l;
     const int N = p.n_eff[b];
     if (N <= 0) return;   // not due
 

@@ -129,7 +129,11 @@ RKV_API int32_t rkv_last_cuda_error(void);
  * Bytes of device workspace every call below needs for the given shapes
  * (n_layers = batch = 1 and cap = the per-head row count for the per-head
  * entry points).  Returns 0 for an invalid config.  The workspace needs
- * 256-byte alignment, holds no state between calls and may be reused.
+ * 256-byte alignment, holds no state between calls and may be reused.  The
+ * size includes room for one int32 per sequence in which the batched steps
+ * order the sequences by decreasing length, so that their units start with the
+ * longest; a workspace short of exactly that room (256-byte rounded) is still
+ * accepted, and the units then run in launch order (the results are the same).
  */
 RKV_API size_t rkv_workspace_size(const rkv_config *cfg, int32_t n_layers, int32_t batch, int32_t cap);
 

@@ -157,7 +157,9 @@ def test_shared_selection_host_validation():
     assert L.rkv_score_shared(cfgp, 2, 1, 1152, k, None, None, None, cur, z, ws, need, None) == -1
     assert L.rkv_score_shared(cfgp, 2, 1, 1152, k, q, None, None, cur, None, ws, need, None) == -1
     assert L.rkv_score_shared(cfgp, 2, 1, 1152, k, q, None, None, cur, z, None, need, None) == -5
-    assert L.rkv_score_shared(cfgp, 2, 1, 1152, k, q, None, None, cur, z, ws, need - 256, None) == -5
+    # (the size includes 256 bytes of room for the order of the sequences, which a call
+    # can do without; 512 short is below what it needs)
+    assert L.rkv_score_shared(cfgp, 2, 1, 1152, k, q, None, None, cur, z, ws, need - 512, None) == -5
     assert L.rkv_score_shared(cfgp, 2, 1, 1152, k, q, None, None, cur, z + 4, ws, need, None) == -3
     assert L.rkv_score_shared(ctypes.byref(rkv.make_config(buffer=0)), 2, 1, 1152, k, q, None,
                               None, cur, z, ws, need, None) == 1
@@ -197,7 +199,7 @@ def test_ragged_step_host_validation():
     assert call(rkv.rkv_ragged_kv(A, A, 100000, 9000)) == -6                 # one CTA cannot hold it
     assert call(cfg=ctypes.byref(rkv.make_config(buffer=0))) == 1            # disabled
     assert call(ws_=None) == -5
-    assert call(ws_bytes=need - 256) == -5
+    assert call(ws_bytes=need - 512) == -5                                   # below the required part
     assert call(ws_=ws + 16) == -3
     assert call(vv=arr(A + 4096, A + (1 << 36))) == -4                       # K pool overlaps V pool
     opts = rkv.rkv_step_options(None, None, None, None, 8)
