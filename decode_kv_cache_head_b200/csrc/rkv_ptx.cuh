@@ -190,37 +190,52 @@ __device__ __forceinline__ uint32_t desc_lo_sw128(uint32_t smem_addr) {
 }
 constexpr uint32_t kDescHiSw128 = (1024u >> 4) | (1u << 14) | (2u << 29);
 
-__device__ __forceinline__ void umma_bf16_k128_sw128(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
-                                                     uint32_t idesc) {
+// The general form: A's K steps advance its descriptor by kAStep within a half and by kAHalf
+// between halves (16-byte units; a K-major A: 2 and 1024, an MN-major A: 128 and 512), B's by
+// 2 and kBHalf.  The first UMMA accumulates onto D when `accumulate` is nonzero.
+template <uint32_t kAStep, uint32_t kAHalf, uint32_t kBHalf>
+__device__ __forceinline__ void umma_bf16_k128(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
+                                               uint32_t idesc, uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred pf, pt;\n\t.reg .b64 da, db;\n\t.reg .b32 al, bl;\n\t"
-        "setp.ne.b32 pf, %1, %1;\n\t"
+        "setp.ne.b32 pf, %5, 0;\n\t"
         "setp.eq.b32 pt, %1, %1;\n\t"
         "mov.b64 da, {%1, %3};\n\tmov.b64 db, {%2, %3};\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, pf;\n\t"
-        "add.u32 al, %1, 2;\n\tadd.u32 bl, %2, 2;\n\t"
+        "add.u32 al, %1, %6;\n\tadd.u32 bl, %2, 2;\n\t"
         "mov.b64 da, {al, %3};\n\tmov.b64 db, {bl, %3};\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, pt;\n\t"
-        "add.u32 al, %1, 4;\n\tadd.u32 bl, %2, 4;\n\t"
+        "add.u32 al, %1, %7;\n\tadd.u32 bl, %2, 4;\n\t"
         "mov.b64 da, {al, %3};\n\tmov.b64 db, {bl, %3};\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, pt;\n\t"
-        "add.u32 al, %1, 6;\n\tadd.u32 bl, %2, 6;\n\t"
+        "add.u32 al, %1, %8;\n\tadd.u32 bl, %2, 6;\n\t"
         "mov.b64 da, {al, %3};\n\tmov.b64 db, {bl, %3};\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, pt;\n\t"
-        "add.u32 al, %1, 1024;\n\tadd.u32 bl, %2, 1024;\n\t"
+        "add.u32 al, %1, %9;\n\tadd.u32 bl, %2, %13;\n\t"
         "mov.b64 da, {al, %3};\n\tmov.b64 db, {bl, %3};\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, pt;\n\t"
-        "add.u32 al, %1, 1026;\n\tadd.u32 bl, %2, 1026;\n\t"
+        "add.u32 al, %1, %10;\n\tadd.u32 bl, %2, %14;\n\t"
         "mov.b64 da, {al, %3};\n\tmov.b64 db, {bl, %3};\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, pt;\n\t"
-        "add.u32 al, %1, 1028;\n\tadd.u32 bl, %2, 1028;\n\t"
+        "add.u32 al, %1, %11;\n\tadd.u32 bl, %2, %15;\n\t"
         "mov.b64 da, {al, %3};\n\tmov.b64 db, {bl, %3};\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, pt;\n\t"
-        "add.u32 al, %1, 1030;\n\tadd.u32 bl, %2, 1030;\n\t"
+        "add.u32 al, %1, %12;\n\tadd.u32 bl, %2, %16;\n\t"
         "mov.b64 da, {al, %3};\n\tmov.b64 db, {bl, %3};\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, pt;\n\t}\n" ::"r"(d_tmem),
-        "r"(a_lo), "r"(b_lo), "r"(kDescHiSw128), "r"(idesc)
+        "r"(a_lo), "r"(b_lo), "r"(kDescHiSw128), "r"(idesc), "r"(accumulate),
+        "n"(kAStep), "n"(2u * kAStep), "n"(3u * kAStep), "n"(kAHalf), "n"(kAHalf + kAStep),
+        "n"(kAHalf + 2u * kAStep), "n"(kAHalf + 3u * kAStep), "n"(kBHalf), "n"(kBHalf + 2u),
+        "n"(kBHalf + 4u), "n"(kBHalf + 6u)
         : "memory");
+}
+
+// Both operands K-major: D = A B^T (the first UMMA overwrites D).  kBHalf: B's second
+// 64-column half in 16-byte units past its first (A's is always 16 KB).
+template <uint32_t kBHalf = 1024u>
+__device__ __forceinline__ void umma_bf16_k128_sw128(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
+                                                     uint32_t idesc) {
+    umma_bf16_k128<2u, 1024u, kBHalf>(d_tmem, a_lo, b_lo, idesc, 0u);
 }
 
 // Arrives once on `bar` when every UMMA issued so far by this thread has completed.

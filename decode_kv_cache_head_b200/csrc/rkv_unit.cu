@@ -250,14 +250,11 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
         tc_fence_after();
         const bool with_s = g >= T && !red_max;
         const uint32_t idesc = with_s ? idesc_bf16_f32(128, NQP + 16) : idesc_bf16_f32(128, NQP);
-        const uint32_t a_base = smem_u32(sStage + (g & 1) * kStageBytes), b_base = smem_u32(sB);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t half = ks >> 2, koff = (ks & 3) * 32u;
-            const uint64_t ad = desc_kmajor_sw128(a_base + half * kHalfBytes + koff);
-            const uint64_t bd = desc_kmajor_sw128(b_base + half * kBRows * 128u + koff);
-            umma_bf16(tmem_base + static_cast<uint32_t>((g & 1) * SLOT), ad, bd, idesc, ks > 0 ? 1u : 0u);
-        }
+        // A: the tile's two 64-column halves 16 KB apart; B: the queries (and split S), halves
+        // kBRows x 128 bytes apart; eight K steps issued from one asm block
+        umma_bf16_k128_sw128<kBRows * 8u>(tmem_base + static_cast<uint32_t>((g & 1) * SLOT),
+                                          desc_lo_sw128(smem_u32(sStage + (g & 1) * kStageBytes)),
+                                          desc_lo_sw128(smem_u32(sB)), idesc);
         umma_commit(&mmab[g & 1]);
     };
     if (tid == 0) {
@@ -366,13 +363,11 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
                     // 64-column blocks 16 KB apart, 8-row groups 1 KB apart), B = inv split
                     tc_fence_after();
                     constexpr uint32_t idesc_s = idesc_bf16_f32_amn(128, 16);
-                    const uint32_t a_base = smem_u32(stg), b_base = smem_u32(sBs + s * 4096);
-#pragma unroll
-                    for (int ks = 0; ks < 8; ++ks) {
-                        const uint64_t ad = desc_mnmajor_sw128(a_base + ks * 2048u, kHalfBytes, 1024u);
-                        const uint64_t bd = desc_kmajor_sw128(b_base + (ks >> 2) * 2048u + (ks & 3) * 32u);
-                        umma_bf16(tmem_base + scol, ad, bd, idesc_s, (g > 0 || ks > 0) ? 1u : 0u);
-                    }
+                    // A MN-major: K steps of 16 rows are 2 KB apart; B: 64-row halves 2 KB apart
+                    const uint32_t a_lo = static_cast<uint32_t>(desc_mnmajor_sw128(smem_u32(stg), kHalfBytes, 1024u));
+                    umma_bf16_k128<128u, 512u, 128u>(tmem_base + scol, a_lo,
+                                                     desc_lo_sw128(smem_u32(sBs + s * 4096)), idesc_s,
+                                                     g > 0 ? 1u : 0u);
                     umma_commit(&smma[s]);
                 }
             }
