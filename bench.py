@@ -110,6 +110,7 @@ KERNEL_SOURCES = {
                         "rkv_ptx.cuh"),
     "rkv_step_kernel": ("rkv_step.cu", "rkv_block.cuh", "rkv_internal.h", "rkv_post.cuh",
                         "rkv_ptx.cuh"),
+    "rkv_gram_max_kernel": ("rkv_gram.cu", "rkv_block.cuh", "rkv_internal.h", "rkv_ptx.cuh"),
 }
 
 
@@ -667,7 +668,10 @@ def run_rkv(args, w, red_mode):
         t_ach = alg_flops / (sim_ms / 1e3) / 1e12
         roofline_unit = roofline
         roofline = {"bound": "tensor", "achieved": t_ach, "peak": tpeak, "unit": "TFLOP/s",
-                    "frac": t_ach / tpeak, "traffic": None, "kernel": "rkv_gram_max_kernel",
+                    "frac": t_ach / tpeak,
+                    "traffic": profiled_traffic("rkv_gram_max_kernel", w.name, units),
+                    "kernel": "rkv_gram_max_kernel",
+                    "kernel_source_sha256_16": kernel_source_digest("rkv_gram_max_kernel"),
                     "kernel_us_per_launch": sim_ms * 1e3, "algorithmic_flops_per_launch": alg_flops,
                     "executed_flops_per_launch": exe_flops,
                     "executed_tflops": exe_flops / (sim_ms / 1e3) / 1e12, "peak_source": tkind}
