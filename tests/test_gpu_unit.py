@@ -125,6 +125,18 @@ def test_max_redundancy_step(rkv, lam):
     verify(w, x, out, all_units(w), w.budget_of, lambda b: lam, red_mode=1)
 
 
+@pytest.mark.parametrize("red_mode", [0, 1], ids=["mean", "max"])
+def test_longest_cache(rkv, red_mode):
+    """The longest cache the unit kernel and the similarity kernel take: N = 7680 rows
+    (60 tiles; 7672 candidates, 30 per thread in the select; one CTA per SM)."""
+    w = Workload("longest", 1, 1, 2, 8, 128, (7552,), buffer=128, seed=79)
+    assert w.cap == 7680
+    x = make_inputs(w)
+    out = run_step(rkv, w, x, red_mode=red_mode, cluster_size=1)
+    verify(w, x, out, all_units(w), w.budget_of, lambda b: w.mix_lambda, red_mode=red_mode)
+    assert out["cur_len"].tolist() == [7552]
+
+
 def test_automatic_choice_at_many_units(rkv):
     """With one unit per SM or more the step picks this kernel by itself; the result
     is identical to forcing it."""
