@@ -45,8 +45,12 @@ from rkv_synth import WORKLOADS, bf16_bits, make_inputs, pack_ragged  # noqa: E4
 
 METRIC = "cached tokens compressed/sec (all layers×heads); µs per compress step"
 UNIT = "tokens/s"
-def profile_traffic_path(kernel, workload):
-    return os.path.join(ROOT, "profiles", f"{kernel}.{workload}.traffic.txt")
+def profile_traffic_path(kernel, workload, variant=""):
+    """The committed ncu traffic summary of `kernel` on `workload`; `variant` ("max")
+    names a run whose kernel does different work (the step kernel reading r in MAX
+    mode instead of computing the MEAN row sums)."""
+    tag = f".{variant}" if variant else ""
+    return os.path.join(ROOT, "profiles", f"{kernel}.{workload}{tag}.traffic.txt")
 
 
 def parse_args():
@@ -125,10 +129,10 @@ def kernel_source_digest(kernel):
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kernel, workload, units_per_launch):
+def profiled_traffic(kernel, workload, units_per_launch, variant=""):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
     the current kernel sources (else None)."""
-    path = profile_traffic_path(kernel, workload)
+    path = profile_traffic_path(kernel, workload, variant)
     if not os.path.exists(path):
         return None
     kv = {}
@@ -647,10 +651,16 @@ def run_rkv(args, w, red_mode):
 
     peak, peak_kind = measured_peaks()
     achieved = alg_bytes / (kern_ms / 1e3) / 1e9
+    # a step launches the main kernel once per 32-layer chunk: the per-launch figures
+    # are the step's totals over its launches (their ratio, `achieved`, is the same)
+    n_chunks = (L + 31) // 32
+    traffic = profiled_traffic(kernel_name, w.name, units, "max" if red_mode else "")
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": profiled_traffic(kernel_name, w.name, units),
-                "kernel": kernel_name, "kernel_us_per_launch": kern_ms * 1e3,
-                "algorithmic_bytes_per_launch": alg_bytes,
+                "frac": achieved / peak,
+                "traffic": traffic / n_chunks if traffic is not None else None,
+                "kernel": kernel_name, "launches_per_step": n_chunks,
+                "kernel_us_per_launch": kern_ms * 1e3 / n_chunks,
+                "algorithmic_bytes_per_launch": alg_bytes / n_chunks,
                 "algorithmic_bytes_definition": ALG_BYTES_DEFINITION,
                 "moved_rows": moved, "kept_rows": L * H * sum(w.budget_of(b) for b in range(B)),
                 "peak_source": peak_kind,
@@ -667,13 +677,16 @@ def run_rkv(args, w, red_mode):
         tpeak, tkind = measured_bf16_tflops()
         t_ach = alg_flops / (sim_ms / 1e3) / 1e12
         roofline_unit = roofline
+        n_sim = n_chunks * gram_launches_per_chunk()
+        sim_traffic = profiled_traffic("rkv_gram_max_kernel", w.name, units)
         roofline = {"bound": "tensor", "achieved": t_ach, "peak": tpeak, "unit": "TFLOP/s",
                     "frac": t_ach / tpeak,
-                    "traffic": profiled_traffic("rkv_gram_max_kernel", w.name, units),
+                    "traffic": sim_traffic / n_sim if sim_traffic is not None else None,
                     "kernel": "rkv_gram_max_kernel",
                     "kernel_source_sha256_16": kernel_source_digest("rkv_gram_max_kernel"),
-                    "kernel_us_per_launch": sim_ms * 1e3, "algorithmic_flops_per_launch": alg_flops,
-                    "executed_flops_per_launch": exe_flops,
+                    "launches_per_step": n_sim, "kernel_us_per_launch": sim_ms * 1e3 / n_sim,
+                    "algorithmic_flops_per_launch": alg_flops / n_sim,
+                    "executed_flops_per_launch": exe_flops / n_sim,
                     "executed_tflops": exe_flops / (sim_ms / 1e3) / 1e12, "peak_source": tkind}
 
     cpu = cpu1 = None
