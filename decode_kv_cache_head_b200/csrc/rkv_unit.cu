@@ -21,7 +21,7 @@
 //   between the passes: the column pairs are merged over the CTA; S is split
 //     into three bf16 terms (hi + mid + lo carries its fp32 value) and written
 //     as three extra rows of the UMMA B operand.
-//   pass 2 (the same tiles, now from L2): the UMMA gives the logits again and,
+//   pass 2 (the same tiles, last to first, now from L2): the UMMA gives the logits again and,
 //     in three more columns, k_i . S; per row p = exp(s - max) / sum, the mean
 //     over the window queries and the max over the group (Ihat_i), and
 //     r_i = (khat_i . S - khat_i . khat_i) / (N - 1) (MEAN) or r_i from the
@@ -222,9 +222,13 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
     // last tile / logits UMMA / S UMMA issued (thread 0's copies), for the error path
     int tma_last = 1, mma_last = -1;
     const CUtensorMap *mk = &p.tmap_k[l];
-    auto issue_tile = [&](int g) {   // global tile g: pass 1 for g < T, pass 2 after
+    // global tile g: pass 1 takes tiles 0 .. T-1, pass 2 the same tiles from T-1 down to 0,
+    // so it starts on the tiles pass 1 read last (the most likely still in L2) and ends on the
+    // first ones, which the compaction reads first
+    auto tile_of = [&](int g) { return g < T ? g : 2 * T - 1 - g; };
+    auto issue_tile = [&](int g) {
         tma_last = g;
-        const int tt = g < T ? g : g - T;
+        const int tt = tile_of(g);
         uint8_t *stg = sStage + (g & 1) * kStageBytes;
         // K tiles are kept in L2 (evict last): pass 2 and the compaction read them again
         const uint64_t pol = policy_evict_last();
@@ -291,7 +295,7 @@ __global__ void __launch_bounds__(kUnitThreads, 2) rkv_unit_kernel(const __grid_
     int g = 0;
     for (; g < 2 * T; ++g) {
         const bool pass2 = g >= T;
-        const int tt = pass2 ? g - T : g;
+        const int tt = tile_of(g);
         const int s = g & 1;
         const uint32_t par = static_cast<uint32_t>((g >> 1) & 1);
         uint8_t *stg = sStage + s * kStageBytes;
