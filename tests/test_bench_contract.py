@@ -63,3 +63,35 @@ def test_reference_arm_prints_one_json_line_with_the_contract_keys():
     e2e = d["e2e"]
     assert e2e["value"] == d["value"] and e2e["unit"] == d["unit"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+
+
+def test_profiled_traffic_follows_the_kernel_sources(tmp_path, monkeypatch):
+    # a committed ncu summary counts only while the kernel's sources hash to its digest
+    path = tmp_path / "summary.traffic.txt"
+    monkeypatch.setattr(bench, "profile_traffic_path", lambda kernel, workload, variant="": str(path))
+    digest = bench.kernel_source_digest("rkv_unit_kernel")
+    path.write_text("# dram bytes\nkernel_source_sha256_16: %s\nunits_per_launch: 8\n"
+                    "dram_bytes_per_unit: 1000\n" % digest)
+    assert bench.profiled_traffic("rkv_unit_kernel", "w", 16) == 16000
+    path.write_text("kernel_source_sha256_16: %s\ndram_bytes_per_unit: 1000\n" % ("0" * 16))
+    assert bench.profiled_traffic("rkv_unit_kernel", "w", 16) is None
+    path.unlink()
+    assert bench.profiled_traffic("rkv_unit_kernel", "w", 16) is None
+
+
+def test_committed_traffic_summaries_name_a_known_kernel_and_their_units():
+    # every summary under profiles/ parses, names a timed kernel and gives a per-unit figure
+    prof = os.path.join(ROOT, "profiles")
+    names = [n for n in os.listdir(prof) if n.endswith(".traffic.txt")]
+    assert names
+    for n in names:
+        kernel = n.split(".")[0]
+        assert kernel in bench.KERNEL_SOURCES, n
+        kv = {}
+        with open(os.path.join(prof, n)) as f:
+            for line in f:
+                if ":" in line and not line.startswith("#"):
+                    k, v = line.split(":", 1)
+                    kv[k.strip()] = v.strip()
+        assert len(kv["kernel_source_sha256_16"]) == 16, n
+        assert int(kv["units_per_launch"]) > 0 and int(kv["dram_bytes_per_unit"]) > 0, n
