@@ -109,14 +109,15 @@ def test_ablation_extremes(rkv, lam, pool):
     verify(w, x, out, all_units(w), w.budget_of, lambda b: lam, pool=pool)
 
 
-def test_group_of_five_and_ragged_lengths(rkv):
+@pytest.mark.parametrize("red_mode", [0, 1], ids=["mean", "max"])
+def test_group_of_five_and_ragged_lengths(rkv, red_mode):
     """Qwen-14B-like group (G = 5, 40 query columns padded to 48) and lengths that
-    are not multiples of 16, several sequences per batch."""
+    are not multiples of 16, several sequences per batch, in both redundancy modes."""
     w = Workload("g5", 2, 3, 2, 10, 128, (900, 1500, 333), buffer=97, seed=63)
     x = make_inputs(w)
     budgets = torch.tensor([w.budget_of(b) for b in range(3)], dtype=torch.int32, device="cuda")
-    out = run_step(rkv, w, x, budgets=budgets)
-    verify(w, x, out, all_units(w), w.budget_of, lambda b: w.mix_lambda)
+    out = run_step(rkv, w, x, budgets=budgets, red_mode=red_mode)
+    verify(w, x, out, all_units(w), w.budget_of, lambda b: w.mix_lambda, red_mode=red_mode)
     assert out["cur_len"].tolist() == [900, 1500, 333]
 
 

@@ -50,16 +50,19 @@ def test_ablation_extremes(rkv, lam, pool):
     verify(w, x, out, all_units(w), w.budget_of, lambda b: lam, pool=pool)
 
 
+@pytest.mark.parametrize("red_mode", [0, 1], ids=["mean", "max"])
 @pytest.mark.parametrize("n_q,window", [(10, 8), (16, 8), (12, 4), (8, 3), (4, 16)])
-def test_groups_and_windows(rkv, n_q, window):
+def test_groups_and_windows(rkv, n_q, window, red_mode):
     """G = 5 (40 query columns padded to 48), G = 8 (64 columns), and windows other
-    than 8 (the runtime-window kernel), with ragged lengths and several sequences."""
+    than 8 (the runtime-window kernel), with ragged lengths and several sequences, in
+    both redundancy modes."""
     w = Workload("gw", 2, 3, 2, n_q, 128, (900, 1500, 333), buffer=97, window=window, seed=63)
     x = make_inputs(w)
     budgets = torch.tensor([w.budget_of(b) for b in range(3)], dtype=torch.int32, device="cuda")
     for pool in (0, 1):
-        out = run_step(rkv, w, x, budgets=budgets, pool=pool, cluster_size=1)
-        verify(w, x, out, all_units(w), w.budget_of, lambda b: w.mix_lambda, pool=pool)
+        out = run_step(rkv, w, x, budgets=budgets, pool=pool, cluster_size=1, red_mode=red_mode)
+        verify(w, x, out, all_units(w), w.budget_of, lambda b: w.mix_lambda, pool=pool,
+               red_mode=red_mode)
 
 
 def test_per_sequence_budgets_lambdas_and_not_due(rkv):
