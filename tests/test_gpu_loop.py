@@ -1,6 +1,6 @@
-"""The decode-time cycle on the GPU: tokens are appended (rkv_append_kv) until the
-buffer is full, the step compresses back to the budget (rkv_compress_step),
-and so on.  Every compression is checked against the oracle on the cache as it
+"""The decode-time cycle on the GPU, in both redundancy modes: tokens are appended
+(rkv_append_kv) until the buffer is full, the step compresses back to the budget
+(rkv_compress_step), and so on.  Every compression is checked against the oracle on the cache as it
 was just before the step; the whole cycle is also captured in a CUDA graph and
 must replay bit for bit like the eager calls."""
 import numpy as np
@@ -45,11 +45,12 @@ def _trace(seed, T):
     return k.to(torch.bfloat16), v.to(torch.bfloat16), q.to(torch.bfloat16)
 
 
-def test_append_then_compress_cycles_match_the_oracle(rkv):
+@pytest.mark.parametrize("red_mode", [0, 1], ids=["mean", "max"])
+def test_append_then_compress_cycles_match_the_oracle(rkv, red_mode):
     dev = torch.device("cuda")
     T = CAP + 5 * BUFFER
     kt, vt, qt = _trace(81, T)
-    cfg = rkv.make_config(BUDGET, BUFFER, WINDOW, D, H, H * G, 0.1)
+    cfg = rkv.make_config(BUDGET, BUFFER, WINDOW, D, H, H * G, 0.1, redundancy_mode=red_mode)
     K = torch.zeros((L, B, H, CAP, D), dtype=torch.bfloat16, device=dev)
     V = torch.zeros_like(K)
     cur = torch.zeros(B, dtype=torch.int32, device=dev)
@@ -76,7 +77,8 @@ def test_append_then_compress_cycles_match_the_oracle(rkv):
         for l in range(L):
             for b in range(B):
                 for h in range(H):
-                    o = oracle.unit(qb[l, b, h * G:(h + 1) * G], kb[l, b, h], CAP, BUDGET, 0.1)
+                    o = oracle.unit(qb[l, b, h * G:(h + 1) * G], kb[l, b, h], CAP, BUDGET, 0.1,
+                                    red_mode=red_mode)
                     kp = kh[l, b, h, :BUDGET]
                     gc.check_kept_layout(kp, CAP - WINDOW, CAP, BUDGET)
                     gc.boundary_check(o["Z"], kp[:BUDGET - WINDOW], BUDGET - WINDOW)
@@ -86,10 +88,11 @@ def test_append_then_compress_cycles_match_the_oracle(rkv):
     assert steps == 6
 
 
-def test_the_cycle_replays_in_a_cuda_graph(rkv):
+@pytest.mark.parametrize("red_mode", [0, 1], ids=["mean", "max"])
+def test_the_cycle_replays_in_a_cuda_graph(rkv, red_mode):
     dev = torch.device("cuda")
     kt, vt, qt = _trace(82, CAP + 4 * BUFFER)
-    cfg = rkv.make_config(BUDGET, BUFFER, WINDOW, D, H, H * G, 0.1)
+    cfg = rkv.make_config(BUDGET, BUFFER, WINDOW, D, H, H * G, 0.1, redundancy_mode=red_mode)
 
     def fresh():
         K = torch.zeros((L, B, H, CAP, D), dtype=torch.bfloat16, device=dev)
